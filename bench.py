@@ -1,0 +1,401 @@
+"""Benchmark of the RDA core on B200: prefill tokens/s and decode state GB/s.
+
+One JSON line on stdout (rank 0).  A "step" is one call of the prefill entry
+point over the nano-shaped workload (bf16 q/k/v, B=1, T=4096, H=16,
+Dk=Dv=128, 64-token chunks, nonzero fp32 initial state, final state returned)
+with its inputs resident in HBM; L2 is flushed (a 256 MiB write) between
+timed steps and each step is timed alone with CUDA events on the launching
+stream.  ``e2e`` times the same call with host (pinned) inputs and outputs,
+copies included.  ``decode`` times 128 consecutive decode steps over
+B=256 sequences (state 256 MiB, larger than L2).
+
+Multi-GPU (torchrun): the path does not shard within one problem; every rank
+runs its own replica (weak scaling), timing is the max over ranks.
+
+``--impl reference`` times the fp64 CPU oracle instead (rank 0 only), on a
+bounded sample of the same workload.
+"""
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "RDA prefill tokens/s (H=16,D=128) and decode state GB/s on 1 B200 vs roofline"
+WORKLOAD = "nano_prefill_b1_t4096_h16_d128"
+CHUNK = 64
+
+
+# ------------------------------------------------------------------ algorithmic counts
+
+def prefill_flops_per_token_head(Dk=128, Dv=128, C=CHUNK):
+    """QK^T, KK^T, T.(beta K): 2 C Dk each; T.(beta V), P.U: 2 C Dv each;
+    W.S, Q.S, K^T.U: 2 Dk Dv each; the UT solve: C^2/3 per token."""
+    return 6 * C * Dk + 4 * C * Dv + 6 * Dk * Dv + C * C / 3.0
+
+
+def prefill_bytes_per_token_head(Dk=128, Dv=128, elem=2):
+    """q, k, v read and o written in the I/O dtype; log alpha and beta (fp32) read."""
+    return (2 * Dk + Dv) * elem + Dv * elem + 8
+
+
+def state_bytes(H, Dk, Dv):
+    return H * Dk * Dv * 4
+
+
+def decode_bytes_per_seq_head(Dk=128, Dv=128, elem=2):
+    """State read + written once (fp32) plus the token's q, k, v, o and gates."""
+    return 2 * Dk * Dv * 4 + prefill_bytes_per_token_head(Dk, Dv, elem)
+
+
+# ------------------------------------------------------------------ helpers
+
+def load_peaks():
+    try:
+        with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
+            p = json.load(f)
+        return float(p["hbm_gbs"]), float(p["bf16_tflops"]), float(p.get("bf16_tflops_sustained", 0)), "measured"
+    except Exception:
+        return 6650.0, 1590.0, 1400.0, "fallback"
+
+
+class ClockSampler:
+    """Samples SM clocks and throttle reasons with nvidia-smi in the background."""
+    FIELDS = ["clocks.sm", "clocks.max.sm", "power.draw", "clocks_event_reasons.hw_slowdown",
+              "clocks_event_reasons.hw_thermal_slowdown", "clocks_event_reasons.sw_thermal_slowdown",
+              "clocks_event_reasons.sw_power_cap"]
+    REASONS = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+
+    def __init__(self, gpu_id, interval_ms=20):
+        self.samples = []
+        self.proc = None
+        self.thread = None
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", gpu_id, f"--query-gpu={','.join(self.FIELDS)}",
+                 "--format=csv,noheader,nounits", f"-lms={interval_ms}"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            self.thread = threading.Thread(target=self._read, daemon=True)
+            self.thread.start()
+        except Exception:
+            self.proc = None
+
+    def _read(self):
+        for line in self.proc.stdout:
+            parts = [p.strip() for p in line.split(",")]
+            if len(parts) != len(self.FIELDS):
+                continue
+            try:
+                self.samples.append((time.time(), float(parts[0]), float(parts[1]), parts[3:]))
+            except ValueError:
+                pass
+
+    def stop(self):
+        if self.proc:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except Exception:
+                self.proc.kill()
+
+    def summary(self, t0, t1):
+        inside = [s for s in self.samples if t0 <= s[0] <= t1]
+        if len(inside) < 3:  # short windows: widen to the nearest samples around it
+            inside = [s for s in self.samples if t0 - 0.25 <= s[0] <= t1 + 0.25] or self.samples[-5:]
+        if not inside:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [], "samples": 0}
+        reasons = sorted({self.REASONS[i] for s in inside for i, r in enumerate(s[3])
+                          if r.lower().startswith("active")})
+        return {"sm_mhz": statistics.median(s[1] for s in inside),
+                "sm_max_mhz": max(s[2] for s in inside), "reasons": reasons,
+                "samples": len(inside)}
+
+
+def gpu_id_for(device):
+    import torch
+    try:
+        return "GPU-" + str(torch.cuda.get_device_properties(device).uuid)
+    except Exception:
+        return str(device.index or 0)
+
+
+# ------------------------------------------------------------------ our arm
+
+def run_ours(args, rank, world, device):
+    import torch
+    import gated_delta_rule_rda_b200 as rda
+    import rda_gen
+
+    torch.cuda.set_device(device)
+    stream = torch.cuda.current_stream(device)
+    dist = None
+    if world > 1:
+        import torch.distributed as dist
+
+    inp = rda_gen.workload(WORKLOAD)
+    B, T, H, Dk = inp.q.shape
+    Dv = inp.v.shape[-1]
+    d = inp.to(device)
+    out = torch.empty((B, T, H, Dv), dtype=d.q.dtype, device=device)
+    sf = torch.empty((B, H, Dk, Dv), dtype=torch.float32, device=device)
+    ws = rda.new_workspace(rda.rda_prefill_workspace_bytes(B, T, H, Dk, Dv, 0), device)
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device=device)
+
+    def step():
+        rda.rda_prefill_chunked(d.q, d.k, d.v, d.log_alpha, d.beta,
+                                initial_state=d.initial_state, out=out, final_state=sf,
+                                workspace=ws)
+
+    sampler = ClockSampler(gpu_id_for(device)) if rank == 0 else None
+    for _ in range(args.warmup):
+        flush.zero_()
+        step()
+    torch.cuda.synchronize()
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+          for _ in range(args.steps)]
+    if dist:
+        dist.barrier()
+    torch.cuda.synchronize()
+    t_wall0 = time.time()
+    for s, e in ev:
+        flush.zero_()
+        s.record(stream)
+        step()
+        e.record(stream)
+    torch.cuda.synchronize()
+    t_wall1 = time.time()
+    if dist:
+        dist.barrier()
+    step_ms = [s.elapsed_time(e) for s, e in ev]
+    ms_per_step = sum(step_ms) / len(step_ms)
+    if dist:
+        t = torch.tensor([ms_per_step], device=device)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        ms_per_step = float(t.item())
+    assert rda.rda_read_device_error(ws) == 0, "device error word set during the benchmark"
+
+    # ---- e2e: host (pinned) inputs and outputs, copies inside the timed region
+    host_in = [t.pin_memory() for t in (inp.q, inp.k, inp.v, inp.log_alpha, inp.beta, inp.initial_state)]
+    dev_in = [torch.empty_like(t, device=device) for t in host_in]
+    host_out = torch.empty((B, T, H, Dv), dtype=inp.q.dtype).pin_memory()
+    host_sf = torch.empty((B, H, Dk, Dv), dtype=torch.float32).pin_memory()
+    h2d = sum(t.numel() * t.element_size() for t in host_in)
+    d2h = host_out.numel() * host_out.element_size() + host_sf.numel() * host_sf.element_size()
+
+    def e2e_step():
+        for hd, dd in zip(host_in, dev_in):
+            dd.copy_(hd, non_blocking=True)
+        q, k, v, la, be, s0 = dev_in
+        rda.rda_prefill_chunked(q, k, v, la, be, initial_state=s0, out=out, final_state=sf,
+                                workspace=ws)
+        host_out.copy_(out, non_blocking=True)
+        host_sf.copy_(sf, non_blocking=True)
+
+    e2e_steps = max(3, min(args.steps, 50))
+    for _ in range(3):
+        e2e_step()
+    torch.cuda.synchronize()
+    if dist:
+        dist.barrier()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(e2e_steps):
+        e2e_step()
+    e1.record(stream)
+    torch.cuda.synchronize()
+    e2e_ms = e0.elapsed_time(e1) / e2e_steps
+    if dist:
+        t = torch.tensor([e2e_ms], device=device)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        e2e_ms = float(t.item())
+
+    # ---- decode: 128 consecutive steps over B=256 (state larger than L2)
+    dec = None
+    if not args.no_decode:
+        din = rda_gen.workload("decode_b256_h16_d128_128steps").to(device)
+        st = din.state.clone()
+        dout = torch.empty((din.q.shape[1], H, Dv), dtype=din.q.dtype, device=device)
+        nsteps = din.q.shape[0]
+
+        def dec_rep():
+            for t in range(nsteps):
+                rda.rda_decode_step(din.q[t], din.k[t], din.v[t], din.log_alpha[t], din.beta[t],
+                                    st, out=dout)
+        dec_rep()
+        torch.cuda.synchronize()
+        reps = 3
+        d0, d1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        if dist:
+            dist.barrier()
+        d0.record(stream)
+        for _ in range(reps):
+            dec_rep()
+        d1.record(stream)
+        torch.cuda.synchronize()
+        dms = d0.elapsed_time(d1) / (reps * nsteps)
+        if dist:
+            t = torch.tensor([dms], device=device)
+            dist.all_reduce(t, op=dist.ReduceOp.MAX)
+            dms = float(t.item())
+        Bd = din.q.shape[1]
+        bytes_step = Bd * H * decode_bytes_per_seq_head(Dk, Dv, 2)
+        hbm, _, _, src = load_peaks()
+        gbs = bytes_step / (dms * 1e-3) / 1e9
+        dec = {"workload": "decode_b256_h16_d128_128steps", "ms_per_decode_step": dms,
+               "state_gbs": gbs * world, "bytes_per_step": bytes_step,
+               "hbm_frac": gbs / hbm, "peak_gbs": hbm, "peak_source": src,
+               "tokens_per_s": Bd * world / (dms * 1e-3)}
+        del din, st
+
+    clocks = None
+    if sampler:
+        sampler.stop()
+        clocks = sampler.summary(t_wall0, t_wall1)
+
+    hbm, tf, tf_sus, src = load_peaks()
+    tokens = B * T
+    alg_bytes = tokens * H * prefill_bytes_per_token_head(Dk, Dv, 2) + 2 * B * state_bytes(H, Dk, Dv)
+    alg_flops = tokens * H * prefill_flops_per_token_head(Dk, Dv)
+    gbs = alg_bytes / (ms_per_step * 1e-3) / 1e9
+    tflops = alg_flops / (ms_per_step * 1e-3) / 1e12
+    return {
+        "metric": METRIC,
+        "value": tokens * world / (ms_per_step * 1e-3),
+        "unit": "tokens/s",
+        "n_gpus": world,
+        "steps": args.steps,
+        "warmup": args.warmup,
+        "ms_per_step": ms_per_step,
+        "higher_is_better": True,
+        "scaling": "weak",
+        "vs_baseline": None,
+        "dtype": "bf16",
+        "data": "synthetic",
+        "config": {"workload": WORKLOAD, "B": B, "T": T, "H": H, "Dk": Dk, "Dv": Dv,
+                   "chunk": CHUNK, "state": "fp32, nonzero initial, final returned",
+                   "l2": "flushed between timed steps (256 MiB write)",
+                   "parallelism": f"replicas x{world}"},
+        "roofline": {"bound": "hbm", "achieved": gbs, "peak": hbm, "unit": "GB/s",
+                     "frac": gbs / hbm, "traffic": None, "peak_source": src,
+                     "algorithmic_bytes_per_launch": alg_bytes,
+                     "tensor": {"achieved_tflops": tflops, "peak_tflops": tf,
+                                "frac": tflops / tf, "algorithmic_flops_per_launch": alg_flops}},
+        "e2e": {"value": tokens * world / (e2e_ms * 1e-3), "unit": "tokens/s",
+                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms},
+        "gpu_launches": args.steps,
+        "clocks": clocks,
+        "decode": dec,
+    }
+
+
+# ------------------------------------------------------------------ oracle timing
+
+_ORACLE_INPUTS = []
+
+
+def oracle_sample_rate(T_sample, threads):
+    """Times the oracle on the first T_sample tokens of the workload, all 16
+    heads; returns (tokens/s, seconds, cores used)."""
+    import oracle
+    import rda_gen
+    if not _ORACLE_INPUTS:
+        _ORACLE_INPUTS.append(rda_gen.workload(WORKLOAD))
+    inp = _ORACLE_INPUTS[0]
+    sl = lambda t: t[:, :T_sample]
+    H = inp.q.shape[2]
+    t0 = time.perf_counter()
+    oracle.forward(sl(inp.q), sl(inp.k), sl(inp.v), sl(inp.log_alpha), sl(inp.beta),
+                   initial_state=inp.initial_state, num_threads=threads)
+    dt = time.perf_counter() - t0
+    return T_sample / dt, dt, min(threads, H)
+
+
+def cpu_baseline(target_s=10.0):
+    import oracle
+    threads = oracle.max_threads()
+    rate, dt, cores = oracle_sample_rate(64, threads)
+    T_sample = int(min(4096, max(64, rate * target_s)))
+    rate, dt, cores = oracle_sample_rate(T_sample, threads)
+    return {"value": rate, "unit": "tokens/s", "cores": cores, "kind": "oracle",
+            "sample": f"fp64 token-sequential oracle on the first {T_sample} tokens of "
+                      f"{WORKLOAD} (all 16 heads, one OpenMP thread per head), {dt:.1f} s"}
+
+
+def run_reference(args):
+    import oracle
+    threads = oracle.max_threads()
+    rate, _, _ = oracle_sample_rate(16, threads)
+    per_step_s = max(0.5, min(3.0, 120.0 / max(1, args.steps + args.warmup)))
+    T_sample = int(min(4096, max(16, rate * per_step_s)))
+    for _ in range(args.warmup):
+        oracle_sample_rate(T_sample, threads)
+    times = []
+    cores = 1
+    for _ in range(args.steps):
+        _, dt, cores = oracle_sample_rate(T_sample, threads)
+        times.append(dt)
+    ms = 1e3 * sum(times) / len(times)
+    value = T_sample / (ms * 1e-3)
+    sample = (f"fp64 token-sequential oracle, first {T_sample} tokens of {WORKLOAD} per step "
+              f"(all 16 heads)")
+    return {
+        "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": 0, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "f64", "data": "synthetic", "impl": "reference",
+        "config": {"workload": WORKLOAD, "B": 1, "T": 4096, "H": 16, "Dk": 128, "Dv": 128,
+                   "chunk": CHUNK, "sample_T": T_sample},
+        "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": cores, "kind": "oracle",
+                         "sample": sample},
+        "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=1000)
+    ap.add_argument("--warmup", type=int, default=20)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--no-decode", action="store_true")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        ap.error("--warmup must be >= 3")
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+
+    if args.impl == "reference":
+        if rank == 0:
+            print(json.dumps(run_reference(args)), flush=True)
+        return
+
+    import torch
+    device = torch.device("cuda", local)
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        torch.cuda.set_device(device)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=device)
+    try:
+        line = run_ours(args, rank, world, device)
+        if rank == 0 and world == 1 and not args.no_cpu_baseline:
+            line["cpu_baseline"] = cpu_baseline()
+        if rank == 0:
+            print(json.dumps(line), flush=True)
+    finally:
+        if world > 1:
+            import torch.distributed as dist
+            dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,216 @@
+"""Python binding of the RDA core C-ABI library (``librda.so``).
+
+Argument marshalling only: every step of the recurrence runs in the library's
+CUDA kernels.  PyTorch supplies device memory and the current stream.  There is
+no CPU fallback: importing this package fails loudly when ``librda.so`` has not
+been built, and every call requires CUDA tensors.
+
+Functions mirror the C entry points of ``include/rda.h``:
+
+- :func:`rda_prefill_chunked` -- fixed-length prefill ``[B,T,H,D]``;
+- :func:`rda_prefill_varlen` -- packed sequences with ``cu_seqlens``;
+- :func:`rda_decode_step` -- one token per sequence, state updated in place;
+- :func:`rda_read_device_error`, :func:`rda_prefill_workspace_bytes`.
+
+The raw ctypes handle is :data:`lib` (``lib.rda_prefill_chunked(...)`` takes
+plain pointers and sizes, including host-pointer use for the varlen schedule).
+"""
+import ctypes
+import os
+
+import torch
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "librda.so")
+
+if not os.path.exists(LIB_PATH):
+    raise ImportError(
+        f"{LIB_PATH} is missing: build it with `python -m gated_delta_rule_rda_b200.build` "
+        "(or __graft_entry__.build()); there is no fallback implementation")
+
+lib = ctypes.CDLL(LIB_PATH)
+
+_vp = ctypes.c_void_p
+_i = ctypes.c_int
+_f = ctypes.c_float
+_sz = ctypes.c_size_t
+
+lib.rda_status_string.argtypes = [_i]
+lib.rda_status_string.restype = ctypes.c_char_p
+lib.rda_version.argtypes = []
+lib.rda_version.restype = ctypes.c_char_p
+lib.rda_prefill_workspace_bytes.argtypes = [_i] * 6
+lib.rda_prefill_workspace_bytes.restype = _sz
+lib.rda_prefill_chunked.argtypes = [_vp] * 9 + [_i] * 6 + [_f, _vp, _sz, _vp]
+lib.rda_prefill_chunked.restype = _i
+lib.rda_prefill_varlen.argtypes = [_vp] * 8 + [_i, _i, _vp, _vp, _vp, _i, _i, _i, _i, _f, _vp, _sz, _vp]
+lib.rda_prefill_varlen.restype = _i
+lib.rda_decode_step.argtypes = [_vp] * 8 + [_i] * 5 + [_f, _vp]
+lib.rda_decode_step.restype = _i
+lib.rda_read_device_error.argtypes = [_vp, ctypes.POINTER(_i), _vp]
+lib.rda_read_device_error.restype = _i
+
+RDA_OK = 0
+RDA_F32 = 0
+RDA_BF16 = 1
+STATUS_NAMES = {0: "RDA_OK", 1: "RDA_ERR_INVALID_ARG", 2: "RDA_ERR_UNSUPPORTED",
+                3: "RDA_ERR_MISALIGNED", 4: "RDA_ERR_WORKSPACE", 5: "RDA_ERR_CUDA",
+                6: "RDA_ERR_TIMEOUT"}
+
+
+class RdaError(RuntimeError):
+    def __init__(self, code, where):
+        self.code = code
+        super().__init__(f"{where}: {lib.rda_status_string(code).decode()}")
+
+
+def _check(code, where):
+    if code != RDA_OK:
+        raise RdaError(code, where)
+
+
+def version() -> str:
+    return lib.rda_version().decode()
+
+
+def _dtype_code(t: torch.Tensor) -> int:
+    if t.dtype == torch.float32:
+        return RDA_F32
+    if t.dtype == torch.bfloat16:
+        return RDA_BF16
+    raise TypeError(f"q/k/v must be float32 or bfloat16, got {t.dtype}")
+
+
+def _ptr(t):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _need_cuda(*ts):
+    for t in ts:
+        if t is not None:
+            if not t.is_cuda:
+                raise ValueError("rda: tensors must be CUDA tensors (no CPU path exists)")
+            if not t.is_contiguous():
+                raise ValueError("rda: tensors must be contiguous")
+
+
+def _need_f32(*ts):
+    for t in ts:
+        if t is not None and t.dtype != torch.float32:
+            raise TypeError(f"rda: gates and states must be float32, got {t.dtype}")
+
+
+def _stream(stream):
+    s = torch.cuda.current_stream() if stream is None else stream
+    return ctypes.c_void_p(s.cuda_stream)
+
+
+def rda_prefill_workspace_bytes(B, T, H, Dk, Dv, num_seqs=0) -> int:
+    return int(lib.rda_prefill_workspace_bytes(B, T, H, Dk, Dv, num_seqs))
+
+
+def new_workspace(nbytes, device) -> torch.Tensor:
+    """A zeroed workspace (256-byte aligned by the caching allocator)."""
+    return torch.zeros(max(int(nbytes), 256), dtype=torch.uint8, device=device)
+
+
+def rda_prefill_chunked(q, k, v, log_alpha, beta, write_gate=None, initial_state=None,
+                        scale=1.0, out=None, final_state=None, return_final_state=True,
+                        workspace=None, stream=None):
+    """Fixed-length prefill.  q, k ``[B,T,H,Dk]``; v ``[B,T,H,Dv]``; gates fp32
+    ``[B,T,H]``; initial_state fp32 ``[B,H,Dk,Dv]`` or None.
+
+    Returns ``(out [B,T,H,Dv], final_state [B,H,Dk,Dv] or None)``.
+    """
+    B, T, H, Dk = q.shape
+    Dv = v.shape[-1]
+    _need_cuda(q, k, v, log_alpha, beta, write_gate, initial_state, out, final_state, workspace)
+    _need_f32(log_alpha, beta, write_gate, initial_state, final_state)
+    dt = _dtype_code(q)
+    if k.dtype != q.dtype or v.dtype != q.dtype:
+        raise TypeError("rda: q, k and v must share a dtype")
+    if k.shape != q.shape or v.shape[:3] != (B, T, H) or log_alpha.shape != (B, T, H) \
+            or beta.shape != (B, T, H):
+        raise ValueError("rda: inconsistent shapes")
+    if out is None:
+        out = torch.empty((B, T, H, Dv), dtype=q.dtype, device=q.device)
+    if final_state is None and return_final_state:
+        final_state = torch.empty((B, H, Dk, Dv), dtype=torch.float32, device=q.device)
+    if workspace is None:
+        workspace = new_workspace(rda_prefill_workspace_bytes(B, T, H, Dk, Dv, 0), q.device)
+    code = lib.rda_prefill_chunked(_ptr(q), _ptr(k), _ptr(v), _ptr(log_alpha), _ptr(beta),
+                                   _ptr(write_gate), _ptr(initial_state), _ptr(final_state),
+                                   _ptr(out), dt, B, T, H, Dk, Dv, float(scale),
+                                   _ptr(workspace), workspace.numel(), _stream(stream))
+    _check(code, "rda_prefill_chunked")
+    return out, final_state
+
+
+def rda_prefill_varlen(q, k, v, log_alpha, beta, cu_seqlens, write_gate=None,
+                       initial_states=None, scale=1.0, out=None, final_states=None,
+                       return_final_states=True, cu_seqlens_host=None, workspace=None,
+                       stream=None):
+    """Packed prefill.  q, k ``[total,H,Dk]``; v ``[total,H,Dv]``; gates
+    ``[total,H]``; cu_seqlens int32 CUDA ``[N+1]``; cu_seqlens_host optional
+    int32 CPU mirror (enables longest-first scheduling).
+
+    Returns ``(out [total,H,Dv], final_states [N,H,Dk,Dv] or None)``.
+    """
+    total, H, Dk = q.shape
+    Dv = v.shape[-1]
+    N = cu_seqlens.numel() - 1
+    _need_cuda(q, k, v, log_alpha, beta, cu_seqlens, write_gate, initial_states, out,
+               final_states, workspace)
+    _need_f32(log_alpha, beta, write_gate, initial_states, final_states)
+    if cu_seqlens.dtype != torch.int32:
+        raise TypeError("rda: cu_seqlens must be int32")
+    dt = _dtype_code(q)
+    if out is None:
+        out = torch.empty((total, H, Dv), dtype=q.dtype, device=q.device)
+    if final_states is None and return_final_states:
+        final_states = torch.empty((N, H, Dk, Dv), dtype=torch.float32, device=q.device)
+    if workspace is None:
+        workspace = new_workspace(rda_prefill_workspace_bytes(1, total, H, Dk, Dv, N), q.device)
+    host_ptr = None
+    if cu_seqlens_host is not None:
+        cu_seqlens_host = cu_seqlens_host.to(torch.int32).contiguous()
+        if cu_seqlens_host.is_cuda:
+            raise ValueError("rda: cu_seqlens_host must be a CPU tensor")
+        host_ptr = ctypes.c_void_p(cu_seqlens_host.data_ptr())
+    code = lib.rda_prefill_varlen(_ptr(q), _ptr(k), _ptr(v), _ptr(log_alpha), _ptr(beta),
+                                  _ptr(write_gate), _ptr(cu_seqlens), host_ptr, N, total,
+                                  _ptr(initial_states), _ptr(final_states), _ptr(out), dt, H, Dk,
+                                  Dv, float(scale), _ptr(workspace), workspace.numel(),
+                                  _stream(stream))
+    _check(code, "rda_prefill_varlen")
+    return out, final_states
+
+
+def rda_decode_step(q, k, v, log_alpha, beta, state, write_gate=None, scale=1.0, out=None,
+                    stream=None):
+    """One decode step.  q, k ``[B,H,Dk]``; v ``[B,H,Dv]``; gates fp32 ``[B,H]``;
+    state fp32 ``[B,H,Dk,Dv]`` updated in place.  Returns ``out [B,H,Dv]``."""
+    B, H, Dk = q.shape
+    Dv = v.shape[-1]
+    _need_cuda(q, k, v, log_alpha, beta, state, write_gate, out)
+    _need_f32(log_alpha, beta, state, write_gate)
+    dt = _dtype_code(q)
+    if out is None:
+        out = torch.empty((B, H, Dv), dtype=q.dtype, device=q.device)
+    code = lib.rda_decode_step(_ptr(q), _ptr(k), _ptr(v), _ptr(log_alpha), _ptr(beta),
+                               _ptr(write_gate), _ptr(state), _ptr(out), dt, B, H, Dk, Dv,
+                               float(scale), _stream(stream))
+    _check(code, "rda_decode_step")
+    return out
+
+
+def rda_read_device_error(workspace, stream=None) -> int:
+    code = _i(0)
+    _check(lib.rda_read_device_error(_ptr(workspace), ctypes.byref(code), _stream(stream)),
+           "rda_read_device_error")
+    return int(code.value)
+
+
+__all__ = ["rda_prefill_chunked", "rda_prefill_varlen", "rda_decode_step",
+           "rda_read_device_error", "rda_prefill_workspace_bytes", "new_workspace", "version",
+           "RdaError", "lib", "LIB_PATH"]

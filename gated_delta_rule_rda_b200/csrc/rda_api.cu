@@ -1,0 +1,207 @@
+// C-ABI entry points (include/rda.h): argument validation on the host, then
+// dispatch to the kernels on the caller's stream.  Nothing here allocates
+// device memory; nothing here computes any part of the recurrence.
+#include <algorithm>
+#include <cstring>
+#include <numeric>
+#include <vector>
+
+#include "rda_internal.h"
+
+using namespace rda;
+
+namespace {
+
+bool aligned(const void *p, size_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
+
+bool dims_ok(int Dk, int Dv) { return (Dk == 64 || Dk == 128) && (Dv == 64 || Dv == 128); }
+
+// Largest element count of any one tensor must stay below 2^31.
+bool sizes_ok(long long tokens, int H, int Dk, int Dv) {
+    const long long m = tokens * H * std::max(Dk, Dv);
+    return tokens >= 0 && H > 0 && m < (1LL << 31);
+}
+
+rda_status_t check_io_ptrs(const void *q, const void *k, const void *v, const float *la,
+                           const float *be, const void *out) {
+    if (!q || !k || !v || !la || !be || !out) return RDA_ERR_INVALID_ARG;
+    if (!aligned(q, 16) || !aligned(k, 16) || !aligned(v, 16) || !aligned(out, 16))
+        return RDA_ERR_MISALIGNED;
+    if (!aligned(la, 4) || !aligned(be, 4)) return RDA_ERR_MISALIGNED;
+    return RDA_OK;
+}
+
+size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
+
+// Workspace layout: [0, 256) error word; then, for packed batches, the
+// longest-first schedule (int32 per sequence).
+size_t workspace_bytes(int num_seqs) {
+    size_t b = kErrorWordBytes;
+    if (num_seqs > 0) b += align_up(sizeof(int32_t) * (size_t)num_seqs, 256);
+    return b;
+}
+
+}  // namespace
+
+extern "C" {
+
+const char *rda_status_string(rda_status_t s) {
+    switch (s) {
+        case RDA_OK: return "RDA_OK";
+        case RDA_ERR_INVALID_ARG: return "RDA_ERR_INVALID_ARG: null required pointer, negative size or bad cu_seqlens";
+        case RDA_ERR_UNSUPPORTED: return "RDA_ERR_UNSUPPORTED: Dk and Dv must be 64 or 128; dtype must be RDA_F32 or RDA_BF16";
+        case RDA_ERR_MISALIGNED: return "RDA_ERR_MISALIGNED: q, k, v, out, state and workspace must be 16-byte aligned (workspace 256)";
+        case RDA_ERR_WORKSPACE: return "RDA_ERR_WORKSPACE: workspace missing or smaller than rda_prefill_workspace_bytes()";
+        case RDA_ERR_CUDA: return "RDA_ERR_CUDA: a CUDA runtime call or kernel launch failed";
+        case RDA_ERR_TIMEOUT: return "RDA_ERR_TIMEOUT: a bounded device-side wait ran out";
+    }
+    return "RDA_ERR_UNKNOWN";
+}
+
+const char *rda_version(void) { return "0.1.0"; }
+
+size_t rda_prefill_workspace_bytes(int B, int T, int H, int Dk, int Dv, int num_seqs) {
+    if (B < 0 || T < 0 || H <= 0 || num_seqs < 0 || !dims_ok(Dk, Dv)) return 0;
+    return workspace_bytes(num_seqs);
+}
+
+rda_status_t rda_prefill_chunked(const void *q, const void *k, const void *v,
+                                 const float *log_alpha, const float *beta,
+                                 const float *write_gate,
+                                 const float *initial_state, float *final_state,
+                                 void *out, rda_dtype_t dtype,
+                                 int B, int T, int H, int Dk, int Dv, float scale,
+                                 void *workspace, size_t workspace_bytes_given, void *stream) {
+    if (dtype != RDA_F32 && dtype != RDA_BF16) return RDA_ERR_UNSUPPORTED;
+    if (B < 0 || T < 0 || H <= 0) return RDA_ERR_INVALID_ARG;
+    if (!dims_ok(Dk, Dv)) return RDA_ERR_UNSUPPORTED;
+    if (!sizes_ok((long long)B * T, H, Dk, Dv)) return RDA_ERR_INVALID_ARG;
+    if ((long long)B * H * Dk * Dv >= (1LL << 31)) return RDA_ERR_INVALID_ARG;
+    if (!workspace || workspace_bytes_given < workspace_bytes(0)) return RDA_ERR_WORKSPACE;
+    if (!aligned(workspace, 256)) return RDA_ERR_MISALIGNED;
+    if ((initial_state && !aligned(initial_state, 16)) || (final_state && !aligned(final_state, 16)))
+        return RDA_ERR_MISALIGNED;
+    if (write_gate && !aligned(write_gate, 4)) return RDA_ERR_MISALIGNED;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    const bool empty = (B == 0 || T == 0);
+    if (!empty) {
+        rda_status_t st = check_io_ptrs(q, k, v, log_alpha, beta, out);
+        if (st != RDA_OK) return st;
+    }
+    if (empty) {
+        if (B > 0 && final_state) {
+            const size_t bytes = sizeof(float) * (size_t)B * H * Dk * Dv;
+            cudaError_t e = initial_state
+                ? (initial_state == final_state ? cudaSuccess
+                   : cudaMemcpyAsync(final_state, initial_state, bytes, cudaMemcpyDeviceToDevice, s))
+                : cudaMemsetAsync(final_state, 0, bytes, s);
+            if (e != cudaSuccess) return RDA_ERR_CUDA;
+        }
+        return RDA_OK;
+    }
+    PrefillArgs a{};
+    a.q = q; a.k = k; a.v = v;
+    a.log_alpha = log_alpha; a.beta = beta; a.gamma = write_gate;
+    a.s0 = initial_state; a.sf = final_state; a.out = out;
+    a.cu_seqlens = nullptr; a.order = nullptr;
+    a.num_seqs = B; a.T = T; a.total_T = B * T;
+    a.H = H; a.Dk = Dk; a.Dv = Dv; a.scale = scale;
+    a.err = static_cast<int32_t *>(workspace);
+    cudaError_t e = chunked_supported(dtype, Dk, Dv) ? launch_chunked(a, s)
+                                                     : launch_recurrent(a, dtype, s);
+    return e == cudaSuccess ? RDA_OK : RDA_ERR_CUDA;
+}
+
+rda_status_t rda_prefill_varlen(const void *q, const void *k, const void *v,
+                                const float *log_alpha, const float *beta,
+                                const float *write_gate,
+                                const int32_t *cu_seqlens, const int32_t *cu_seqlens_host,
+                                int num_seqs, int total_T,
+                                const float *initial_states, float *final_states,
+                                void *out, rda_dtype_t dtype,
+                                int H, int Dk, int Dv, float scale,
+                                void *workspace, size_t workspace_bytes_given, void *stream) {
+    if (dtype != RDA_F32 && dtype != RDA_BF16) return RDA_ERR_UNSUPPORTED;
+    if (num_seqs < 0 || total_T < 0 || H <= 0) return RDA_ERR_INVALID_ARG;
+    if (!dims_ok(Dk, Dv)) return RDA_ERR_UNSUPPORTED;
+    if (!sizes_ok(total_T, H, Dk, Dv)) return RDA_ERR_INVALID_ARG;
+    if ((long long)num_seqs * H * Dk * Dv >= (1LL << 31)) return RDA_ERR_INVALID_ARG;
+    if (num_seqs > 0 && !cu_seqlens) return RDA_ERR_INVALID_ARG;
+    if (!workspace || workspace_bytes_given < workspace_bytes(num_seqs)) return RDA_ERR_WORKSPACE;
+    if (!aligned(workspace, 256)) return RDA_ERR_MISALIGNED;
+    if ((initial_states && !aligned(initial_states, 16)) || (final_states && !aligned(final_states, 16)))
+        return RDA_ERR_MISALIGNED;
+    if (cu_seqlens && !aligned(cu_seqlens, 4)) return RDA_ERR_MISALIGNED;
+    if (total_T > 0) {
+        rda_status_t st = check_io_ptrs(q, k, v, log_alpha, beta, out);
+        if (st != RDA_OK) return st;
+    }
+    if (write_gate && !aligned(write_gate, 4)) return RDA_ERR_MISALIGNED;
+    if (num_seqs == 0) return RDA_OK;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+
+    int32_t *order = nullptr;
+    if (cu_seqlens_host) {
+        if (cu_seqlens_host[0] != 0 || cu_seqlens_host[num_seqs] != total_T) return RDA_ERR_INVALID_ARG;
+        for (int n = 0; n < num_seqs; ++n)
+            if (cu_seqlens_host[n + 1] < cu_seqlens_host[n]) return RDA_ERR_INVALID_ARG;
+        // Longest sequences first, so that the long tails start early.
+        std::vector<int32_t> perm(num_seqs);
+        std::iota(perm.begin(), perm.end(), 0);
+        std::stable_sort(perm.begin(), perm.end(), [&](int32_t x, int32_t y) {
+            return cu_seqlens_host[x + 1] - cu_seqlens_host[x] > cu_seqlens_host[y + 1] - cu_seqlens_host[y];
+        });
+        order = reinterpret_cast<int32_t *>(static_cast<char *>(workspace) + kErrorWordBytes);
+        // Pageable source: the copy is staged before cudaMemcpyAsync returns.
+        if (cudaMemcpyAsync(order, perm.data(), sizeof(int32_t) * num_seqs, cudaMemcpyHostToDevice, s) != cudaSuccess)
+            return RDA_ERR_CUDA;
+    }
+    PrefillArgs a{};
+    a.q = q; a.k = k; a.v = v;
+    a.log_alpha = log_alpha; a.beta = beta; a.gamma = write_gate;
+    a.s0 = initial_states; a.sf = final_states; a.out = out;
+    a.cu_seqlens = cu_seqlens; a.order = order;
+    a.num_seqs = num_seqs; a.T = 0; a.total_T = total_T;
+    a.H = H; a.Dk = Dk; a.Dv = Dv; a.scale = scale;
+    a.err = static_cast<int32_t *>(workspace);
+    cudaError_t e = chunked_supported(dtype, Dk, Dv) ? launch_chunked(a, s)
+                                                     : launch_recurrent(a, dtype, s);
+    return e == cudaSuccess ? RDA_OK : RDA_ERR_CUDA;
+}
+
+rda_status_t rda_decode_step(const void *q, const void *k, const void *v,
+                             const float *log_alpha, const float *beta,
+                             const float *write_gate,
+                             float *state, void *out, rda_dtype_t dtype,
+                             int B, int H, int Dk, int Dv, float scale, void *stream) {
+    if (dtype != RDA_F32 && dtype != RDA_BF16) return RDA_ERR_UNSUPPORTED;
+    if (B < 0 || H <= 0) return RDA_ERR_INVALID_ARG;
+    if (!dims_ok(Dk, Dv)) return RDA_ERR_UNSUPPORTED;
+    if ((long long)B * H * Dk * Dv >= (1LL << 31)) return RDA_ERR_INVALID_ARG;
+    if (B == 0) return RDA_OK;
+    rda_status_t st = check_io_ptrs(q, k, v, log_alpha, beta, out);
+    if (st != RDA_OK) return st;
+    if (!state) return RDA_ERR_INVALID_ARG;
+    if (!aligned(state, 16)) return RDA_ERR_MISALIGNED;
+    if (write_gate && !aligned(write_gate, 4)) return RDA_ERR_MISALIGNED;
+    DecodeArgs a{};
+    a.q = q; a.k = k; a.v = v;
+    a.log_alpha = log_alpha; a.beta = beta; a.gamma = write_gate;
+    a.state = state; a.out = out;
+    a.B = B; a.H = H; a.Dk = Dk; a.Dv = Dv; a.scale = scale;
+    return launch_decode(a, dtype, static_cast<cudaStream_t>(stream)) == cudaSuccess ? RDA_OK : RDA_ERR_CUDA;
+}
+
+rda_status_t rda_read_device_error(void *workspace, int *code, void *stream) {
+    if (!workspace || !code) return RDA_ERR_INVALID_ARG;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    int32_t host = 0;
+    if (cudaMemcpyAsync(&host, workspace, sizeof(int32_t), cudaMemcpyDeviceToHost, s) != cudaSuccess)
+        return RDA_ERR_CUDA;
+    if (cudaStreamSynchronize(s) != cudaSuccess) return RDA_ERR_CUDA;
+    if (cudaMemsetAsync(workspace, 0, sizeof(int32_t), s) != cudaSuccess) return RDA_ERR_CUDA;
+    *code = host;
+    return RDA_OK;
+}
+
+}  // extern "C"

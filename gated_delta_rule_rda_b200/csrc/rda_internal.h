@@ -1,0 +1,52 @@
+// Internal launch interface shared by the C-ABI layer and the kernels.
+// Not installed; the public interface is include/rda.h.
+#pragma once
+
+#include <cstddef>
+#include <cstdint>
+
+#include <cuda_runtime.h>
+
+#include "rda.h"
+
+namespace rda {
+
+// Device error word: first 4 bytes of the caller's workspace.
+constexpr size_t kErrorWordBytes = 256;
+
+// Arguments common to every prefill launch.  Token rows are addressed as
+// (global token index) * H + head; fixed-length batches use seq_start = b * T,
+// packed batches read cu_seqlens.
+struct PrefillArgs {
+    const void *q, *k, *v;
+    const float *log_alpha, *beta, *gamma;
+    const float *s0;
+    float *sf;
+    void *out;
+    const int32_t *cu_seqlens;   // null for fixed-length batches
+    const int32_t *order;        // optional schedule: sequence index per grid z, or null
+    int num_seqs;                // B (fixed) or N (packed)
+    int T;                       // tokens per sequence (fixed only)
+    int total_T;                 // B*T or packed total
+    int H, Dk, Dv;
+    float scale;
+    int32_t *err;                // device error word
+};
+
+struct DecodeArgs {
+    const void *q, *k, *v;
+    const float *log_alpha, *beta, *gamma;
+    float *state;
+    void *out;
+    int B, H, Dk, Dv;
+    float scale;
+};
+
+cudaError_t launch_recurrent(const PrefillArgs &a, rda_dtype_t dtype, cudaStream_t s);
+cudaError_t launch_decode(const DecodeArgs &a, rda_dtype_t dtype, cudaStream_t s);
+// Chunked tensor-core prefill (bf16, Dk = 128).  Returns cudaErrorNotSupported
+// when the sizes are outside what it handles; the caller then falls back.
+cudaError_t launch_chunked(const PrefillArgs &a, cudaStream_t s);
+bool chunked_supported(rda_dtype_t dtype, int Dk, int Dv);
+
+}  // namespace rda

@@ -1,0 +1,180 @@
+/*
+ * rda.h -- C ABI of the RDA (Raon Delta Attention) core for NVIDIA B200 (sm_100a).
+ *
+ * WHAT IS COMPUTED
+ *   Per sequence and head, the gated delta rule.  The article "Raon-1 nano:
+ *   half of a 3.1B model is a lookup table, and a 99M model keeps one too",
+ *   section "The other 1.5B: a hybrid built to forget", describes the
+ *   reference recurrence: it decays the state, computes the error between the
+ *   value and the state's prediction for the key, writes that error with
+ *   strength beta, and rescales the value with a separate write gate.  In
+ *   matrix form, with the math-orientation state S (Dv x Dk):
+ *
+ *       S_t = alpha_t * S_{t-1} * (I - beta_t k_t k_t^T) + beta_t (gamma_t v_t) k_t^T
+ *       o_t = scale * S_t q_t                       (post-update read)
+ *
+ *   alpha_t = exp(log_alpha_t) is a scalar per (token, head); gamma_t is the
+ *   optional write gate (NULL means 1).  Preconditions, not checked: log_alpha
+ *   in [-5, 0] (the article bounds the decay below by -5 in log space),
+ *   beta in [0, 1], all inputs finite.  Outside them the result is unspecified
+ *   but the call still terminates.
+ *
+ * STATE
+ *   fp32, as the blog post on the Raon-1 mini vLLM pull request lists for its
+ *   fast kernels (FP32 recurrent state) and as the nano article sizes it
+ *   (16 heads x 128 x 128 fp32 per layer).  Stored as [.., H, Dk, Dv]
+ *   row-major: element [i][j] is S[j][i] (i indexes the key dimension, j the
+ *   value dimension).
+ *
+ * LAYOUTS (all row-major, contiguous, no padding)
+ *   q, k   [B, T, H, Dk]        (varlen: [total_T, H, Dk])
+ *   v, out [B, T, H, Dv]        (varlen: [total_T, H, Dv])
+ *   log_alpha, beta, write_gate  fp32 [B, T, H]  (varlen: [total_T, H])
+ *   states fp32 [B, H, Dk, Dv]  (varlen: [num_seqs, H, Dk, Dv])
+ *   q, k, v and out share one element type, rda_dtype_t.
+ *
+ * OWNERSHIP AND ORDERING
+ *   Every pointer named "device" is device memory owned by the caller; the
+ *   library allocates no device memory and keeps no per-call state.  Each call
+ *   enqueues its work on `stream` (a cudaStream_t, passed as void*; NULL is the
+ *   legacy default stream) and returns without synchronising.  Calls are
+ *   thread-safe.  Input buffers must not be modified, and outputs not read,
+ *   until the stream has reached the call.
+ *
+ * ALIASING
+ *   final_state may equal initial_state (updated in place).  No other output
+ *   may overlap any input or another output.
+ *
+ * ERRORS
+ *   Argument errors are detected on the host before anything is enqueued and
+ *   returned synchronously; nothing is launched then.  A failed launch returns
+ *   RDA_ERR_CUDA.  Kernels never trap: a device-side wait that exceeds its
+ *   bound records RDA_ERR_TIMEOUT in the workspace error word, stops the
+ *   affected work and returns; read it with rda_read_device_error().
+ *
+ * SUPPORTED SHAPES
+ *   Dk, Dv in {64, 128}.  B, T, H >= 0 with B*T*H*max(Dk,Dv) < 2^31 per
+ *   tensor.  T = 0 (or B = 0) is a no-op that copies initial to final state.
+ */
+#ifndef RDA_H_
+#define RDA_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+    RDA_OK = 0,
+    RDA_ERR_INVALID_ARG = 1,   /* null required pointer, negative size, bad cu_seqlens */
+    RDA_ERR_UNSUPPORTED = 2,   /* Dk or Dv outside {64, 128}, unknown dtype          */
+    RDA_ERR_MISALIGNED = 3,    /* a pointer breaks the 16-byte alignment rule        */
+    RDA_ERR_WORKSPACE = 4,     /* workspace missing or smaller than required         */
+    RDA_ERR_CUDA = 5,          /* a CUDA runtime call or kernel launch failed        */
+    RDA_ERR_TIMEOUT = 6        /* a bounded device-side wait ran out                 */
+} rda_status_t;
+
+typedef enum {
+    RDA_F32 = 0,               /* q, k, v, out are float                             */
+    RDA_BF16 = 1               /* q, k, v, out are bfloat16 (raw 16-bit words)       */
+} rda_dtype_t;
+
+/* Static, human-readable name of a status code.  Never NULL. */
+const char *rda_status_string(rda_status_t status);
+
+/* Library version string, e.g. "0.1.0". */
+const char *rda_version(void);
+
+/*
+ * Bytes of device workspace that rda_prefill_chunked (num_seqs = 0) or
+ * rda_prefill_varlen (num_seqs = N) needs for these sizes.  Always >= 256
+ * (the first 256 bytes hold the device error word).  The workspace must be
+ * 256-byte aligned.  Returns 0 for unsupported sizes.
+ */
+size_t rda_prefill_workspace_bytes(int B, int T, int H, int Dk, int Dv, int num_seqs);
+
+/*
+ * Fixed-length prefill over B sequences of T tokens each.
+ *
+ * Defined by the gated delta rule above; the chunked form it uses (64-token
+ * chunks, a UT transform of each chunk, tensor-core products, a sequential
+ * scan of fp32 states across chunks) reaches the same result up to rounding.
+ * bf16 inputs take the chunked tensor-core path when Dk = 128; fp32 inputs,
+ * and bf16 with Dk = 64, take a token-sequential fp32 path (fp32 inputs are
+ * held to fp32 accuracy, which bf16 tensor-core operands cannot give).
+ *
+ *   q, k, v        device, dtype, layouts above, 16-byte aligned
+ *   log_alpha      device fp32 [B,T,H]; beta device fp32 [B,T,H]
+ *   write_gate     device fp32 [B,T,H] or NULL (gamma = 1)
+ *   initial_state  device fp32 [B,H,Dk,Dv] or NULL (zero state)
+ *   final_state    device fp32 [B,H,Dk,Dv] or NULL (not returned)
+ *   out            device, dtype, [B,T,H,Dv], 16-byte aligned
+ *   scale          multiplies the output only
+ *   workspace      device, >= rda_prefill_workspace_bytes(B,T,H,Dk,Dv,0)
+ */
+rda_status_t rda_prefill_chunked(const void *q, const void *k, const void *v,
+                                 const float *log_alpha, const float *beta,
+                                 const float *write_gate,
+                                 const float *initial_state, float *final_state,
+                                 void *out, rda_dtype_t dtype,
+                                 int B, int T, int H, int Dk, int Dv, float scale,
+                                 void *workspace, size_t workspace_bytes, void *stream);
+
+/*
+ * Variable-length prefill over num_seqs sequences packed along the token axis.
+ * Sequence n owns tokens [cu_seqlens[n], cu_seqlens[n+1]); chunks restart at
+ * every sequence start and never cross a boundary.  A zero-length sequence
+ * copies its initial state to its final state.
+ *
+ *   cu_seqlens       device int32 [num_seqs+1], non-decreasing, cu_seqlens[0] = 0,
+ *                    cu_seqlens[num_seqs] = total_T
+ *   cu_seqlens_host  host int32 [num_seqs+1] mirror of cu_seqlens, or NULL.  When
+ *                    given, it is validated and used to schedule the longest
+ *                    sequences first; it is read before the call returns.
+ *   initial_states   device fp32 [num_seqs,H,Dk,Dv] or NULL (zero states)
+ *   final_states     device fp32 [num_seqs,H,Dk,Dv] or NULL
+ *   other arguments  as rda_prefill_chunked, with B*T replaced by total_T
+ *   workspace        device, >= rda_prefill_workspace_bytes(1,total_T,H,Dk,Dv,num_seqs)
+ */
+rda_status_t rda_prefill_varlen(const void *q, const void *k, const void *v,
+                                const float *log_alpha, const float *beta,
+                                const float *write_gate,
+                                const int32_t *cu_seqlens, const int32_t *cu_seqlens_host,
+                                int num_seqs, int total_T,
+                                const float *initial_states, float *final_states,
+                                void *out, rda_dtype_t dtype,
+                                int H, int Dk, int Dv, float scale,
+                                void *workspace, size_t workspace_bytes, void *stream);
+
+/*
+ * One decode step for B independent sequences (one new token each), state
+ * updated in place.  It is the T = 1 case of the rule above, evaluated in one
+ * pass over the state: with a = S_old k and b = S_old q,
+ *   e = gamma v - alpha a,  o = scale (alpha b + beta (k.q) e),
+ *   S_new = alpha S_old + beta e k^T.
+ *
+ *   q, k   device, dtype, [B,H,Dk];  v device, dtype, [B,H,Dv]
+ *   log_alpha, beta  device fp32 [B,H];  write_gate device fp32 [B,H] or NULL
+ *   state  device fp32 [B,H,Dk,Dv], read and overwritten, 16-byte aligned
+ *   out    device, dtype, [B,H,Dv]
+ */
+rda_status_t rda_decode_step(const void *q, const void *k, const void *v,
+                             const float *log_alpha, const float *beta,
+                             const float *write_gate,
+                             float *state, void *out, rda_dtype_t dtype,
+                             int B, int H, int Dk, int Dv, float scale, void *stream);
+
+/*
+ * Waits for `stream`, then reads and clears the device error word at the start
+ * of `workspace`.  Writes RDA_OK or the recorded code to *code.  Returns
+ * RDA_ERR_CUDA if the copy fails.
+ */
+rda_status_t rda_read_device_error(void *workspace, int *code, void *stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* RDA_H_ */
