@@ -110,8 +110,11 @@ def rda_prefill_workspace_bytes(B, T, H, Dk, Dv, num_seqs=0) -> int:
 
 
 def new_workspace(nbytes, device) -> torch.Tensor:
-    """A zeroed workspace (256-byte aligned by the caching allocator)."""
-    return torch.zeros(max(int(nbytes), 256), dtype=torch.uint8, device=device)
+    """A workspace of ``nbytes`` (256-byte aligned by the caching allocator)
+    whose device error word (first 256 bytes) starts cleared."""
+    ws = torch.empty(max(int(nbytes), 256), dtype=torch.uint8, device=device)
+    ws[:256].zero_()
+    return ws
 
 
 def rda_prefill_chunked(q, k, v, log_alpha, beta, write_gate=None, initial_state=None,

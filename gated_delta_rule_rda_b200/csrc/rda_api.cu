@@ -34,10 +34,14 @@ rda_status_t check_io_ptrs(const void *q, const void *k, const void *v, const fl
 size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
 
 // Workspace layout: [0, 256) error word; then, for packed batches, the
-// longest-first schedule (int32 per sequence).
-size_t workspace_bytes(int num_seqs) {
-    size_t b = kErrorWordBytes;
-    if (num_seqs > 0) b += align_up(sizeof(int32_t) * (size_t)num_seqs, 256);
+// longest-first schedule (int32 per sequence); then, when the chunked
+// tensor-core path can run (Dk = 128), its per-chunk prep scratch.
+size_t order_bytes(int num_seqs) { return num_seqs > 0 ? align_up(sizeof(int32_t) * (size_t)num_seqs, 256) : 0; }
+
+size_t workspace_bytes(int B, long T, int H, int Dk, int Dv, int num_seqs) {
+    size_t b = kErrorWordBytes + order_bytes(num_seqs);
+    if (chunked_supported(RDA_BF16, Dk, Dv))
+        b += align_up(chunked_workspace_bytes(num_seqs > 0 ? T : (long)B * T, (int)T, B, H, Dv, num_seqs), 256);
     return b;
 }
 
@@ -62,7 +66,7 @@ const char *rda_version(void) { return "0.1.0"; }
 
 size_t rda_prefill_workspace_bytes(int B, int T, int H, int Dk, int Dv, int num_seqs) {
     if (B < 0 || T < 0 || H <= 0 || num_seqs < 0 || !dims_ok(Dk, Dv)) return 0;
-    return workspace_bytes(num_seqs);
+    return workspace_bytes(B, T, H, Dk, Dv, num_seqs);
 }
 
 rda_status_t rda_prefill_chunked(const void *q, const void *k, const void *v,
@@ -77,7 +81,9 @@ rda_status_t rda_prefill_chunked(const void *q, const void *k, const void *v,
     if (!dims_ok(Dk, Dv)) return RDA_ERR_UNSUPPORTED;
     if (!sizes_ok((long long)B * T, H, Dk, Dv)) return RDA_ERR_INVALID_ARG;
     if ((long long)B * H * Dk * Dv >= (1LL << 31)) return RDA_ERR_INVALID_ARG;
-    if (!workspace || workspace_bytes_given < workspace_bytes(0)) return RDA_ERR_WORKSPACE;
+    const bool chunked = chunked_supported(dtype, Dk, Dv);
+    const size_t need = chunked ? workspace_bytes(B, T, H, Dk, Dv, 0) : kErrorWordBytes;
+    if (!workspace || workspace_bytes_given < need) return RDA_ERR_WORKSPACE;
     if (!aligned(workspace, 256)) return RDA_ERR_MISALIGNED;
     if ((initial_state && !aligned(initial_state, 16)) || (final_state && !aligned(final_state, 16)))
         return RDA_ERR_MISALIGNED;
@@ -107,8 +113,8 @@ rda_status_t rda_prefill_chunked(const void *q, const void *k, const void *v,
     a.num_seqs = B; a.T = T; a.total_T = B * T;
     a.H = H; a.Dk = Dk; a.Dv = Dv; a.scale = scale;
     a.err = static_cast<int32_t *>(workspace);
-    cudaError_t e = chunked_supported(dtype, Dk, Dv) ? launch_chunked(a, s)
-                                                     : launch_recurrent(a, dtype, s);
+    cudaError_t e = chunked ? launch_chunked(a, static_cast<char *>(workspace) + kErrorWordBytes, s)
+                            : launch_recurrent(a, dtype, s);
     return e == cudaSuccess ? RDA_OK : RDA_ERR_CUDA;
 }
 
@@ -127,7 +133,10 @@ rda_status_t rda_prefill_varlen(const void *q, const void *k, const void *v,
     if (!sizes_ok(total_T, H, Dk, Dv)) return RDA_ERR_INVALID_ARG;
     if ((long long)num_seqs * H * Dk * Dv >= (1LL << 31)) return RDA_ERR_INVALID_ARG;
     if (num_seqs > 0 && !cu_seqlens) return RDA_ERR_INVALID_ARG;
-    if (!workspace || workspace_bytes_given < workspace_bytes(num_seqs)) return RDA_ERR_WORKSPACE;
+    const bool chunked = chunked_supported(dtype, Dk, Dv);
+    const size_t need = chunked ? workspace_bytes(1, total_T, H, Dk, Dv, num_seqs)
+                                : kErrorWordBytes + order_bytes(num_seqs);
+    if (!workspace || workspace_bytes_given < need) return RDA_ERR_WORKSPACE;
     if (!aligned(workspace, 256)) return RDA_ERR_MISALIGNED;
     if ((initial_states && !aligned(initial_states, 16)) || (final_states && !aligned(final_states, 16)))
         return RDA_ERR_MISALIGNED;
@@ -164,8 +173,9 @@ rda_status_t rda_prefill_varlen(const void *q, const void *k, const void *v,
     a.num_seqs = num_seqs; a.T = 0; a.total_T = total_T;
     a.H = H; a.Dk = Dk; a.Dv = Dv; a.scale = scale;
     a.err = static_cast<int32_t *>(workspace);
-    cudaError_t e = chunked_supported(dtype, Dk, Dv) ? launch_chunked(a, s)
-                                                     : launch_recurrent(a, dtype, s);
+    cudaError_t e = chunked
+        ? launch_chunked(a, static_cast<char *>(workspace) + kErrorWordBytes + order_bytes(num_seqs), s)
+        : launch_recurrent(a, dtype, s);
     return e == cudaSuccess ? RDA_OK : RDA_ERR_CUDA;
 }
 

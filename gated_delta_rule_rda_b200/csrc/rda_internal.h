@@ -31,6 +31,10 @@ struct PrefillArgs {
     int H, Dk, Dv;
     float scale;
     int32_t *err;                // device error word
+    // chunked path only (filled by launch_chunked)
+    const int32_t *chunk_base;   // packed: first global chunk of each sequence [N+1]
+    uint8_t *workspace_chunks;   // per (chunk, head) prep results
+    size_t chunk_bytes;          // bytes per (chunk, head)
 };
 
 struct DecodeArgs {
@@ -44,9 +48,11 @@ struct DecodeArgs {
 
 cudaError_t launch_recurrent(const PrefillArgs &a, rda_dtype_t dtype, cudaStream_t s);
 cudaError_t launch_decode(const DecodeArgs &a, rda_dtype_t dtype, cudaStream_t s);
-// Chunked tensor-core prefill (bf16, Dk = 128).  Returns cudaErrorNotSupported
-// when the sizes are outside what it handles; the caller then falls back.
-cudaError_t launch_chunked(const PrefillArgs &a, cudaStream_t s);
+// Chunked tensor-core prefill (bf16, Dk = 128, Dv in {64, 128}).  `scratch`
+// points at chunked_workspace_bytes() bytes of device memory (256-aligned).
+cudaError_t launch_chunked(const PrefillArgs &a, void *scratch, cudaStream_t s);
 bool chunked_supported(rda_dtype_t dtype, int Dk, int Dv);
+// Scratch the chunked path needs: fixed-length batches pass num_seqs = 0.
+size_t chunked_workspace_bytes(long total_T, int T, int B, int H, int Dv, int num_seqs);
 
 }  // namespace rda

@@ -44,7 +44,9 @@ def test_status_strings_and_version():
 
 
 def test_workspace_query():
-    assert rda.rda_prefill_workspace_bytes(1, 4096, 16, 128, 128, 0) >= 256
+    # the chunked path keeps about 40 KiB of prep results per (chunk, head)
+    assert rda.rda_prefill_workspace_bytes(1, 4096, 16, 128, 128, 0) >= 64 * 16 * 40 * 1024
+    assert rda.rda_prefill_workspace_bytes(1, 4096, 16, 64, 64, 0) >= 256
     assert rda.rda_prefill_workspace_bytes(1, 100, 16, 128, 128, 64) >= 256 + 64 * 4
     assert rda.rda_prefill_workspace_bytes(1, 100, 16, 96, 128, 0) == 0
     assert rda.rda_prefill_workspace_bytes(-1, 100, 16, 128, 128, 0) == 0
@@ -57,7 +59,7 @@ A256 = 0x20000
 
 def _chunked(**kw):
     args = dict(q=A16, k=A16, v=A16, la=A16, be=A16, wg=None, s0=None, sf=None, out=A16,
-                dtype=1, B=1, T=64, H=2, Dk=128, Dv=128, scale=1.0, ws=A256, wsb=256, stream=None)
+                dtype=1, B=1, T=64, H=2, Dk=128, Dv=128, scale=1.0, ws=A256, wsb=1 << 40, stream=None)
     args.update(kw)
     return rda.lib.rda_prefill_chunked(*[args[k] for k in ["q", "k", "v", "la", "be", "wg", "s0", "sf",
                                                            "out", "dtype", "B", "T", "H", "Dk", "Dv",
@@ -86,7 +88,7 @@ def test_chunked_rejects_bad_arguments():
 def _varlen(**kw):
     args = dict(q=A16, k=A16, v=A16, la=A16, be=A16, wg=None, cu=A16, cuh=None, N=2, total=100,
                 s0=None, sf=None, out=A16, dtype=1, H=2, Dk=128, Dv=128, scale=1.0, ws=A256,
-                wsb=1024, stream=None)
+                wsb=1 << 40, stream=None)
     args.update(kw)
     return rda.lib.rda_prefill_varlen(*[args[k] for k in ["q", "k", "v", "la", "be", "wg", "cu", "cuh",
                                                           "N", "total", "s0", "sf", "out", "dtype",
@@ -99,6 +101,7 @@ def test_varlen_rejects_bad_arguments():
     assert _varlen(N=-1) == INVALID
     assert _varlen(Dk=32) == UNSUPPORTED
     assert _varlen(wsb=256) == WORKSPACE          # schedule needs room beyond the error word
+    assert _varlen(dtype=0, Dk=64, wsb=256) == WORKSPACE
     bad = (ctypes.c_int32 * 3)(0, 60, 50)         # total mismatch
     assert _varlen(cuh=ctypes.cast(bad, ctypes.c_void_p)) == INVALID
     dec = (ctypes.c_int32 * 3)(0, 60, 40)         # decreasing
