@@ -105,16 +105,6 @@ __device__ __forceinline__ uint32_t pack_bf16(float a, float b) {
 __device__ __forceinline__ uint4 pack8(const float *x) {
     return make_uint4(pack_bf16(x[0], x[1]), pack_bf16(x[2], x[3]), pack_bf16(x[4], x[5]), pack_bf16(x[6], x[7]));
 }
-__device__ __forceinline__ void unpack8(uint4 u, float *x) {
-    const uint32_t w[4] = {u.x, u.y, u.z, u.w};
-#pragma unroll
-    for (int i = 0; i < 4; ++i) {
-        __nv_bfloat162 hh = *reinterpret_cast<const __nv_bfloat162 *>(&w[i]);
-        float2 f = __bfloat1622float2(hh);
-        x[2 * i] = f.x;
-        x[2 * i + 1] = f.y;
-    }
-}
 
 // ---------------------------------------------------------------------------
 // UT transform.
@@ -531,26 +521,79 @@ prep_kernel(const __grid_constant__ PrepMaps maps, const PrefillArgs a) {
 
 // ---------------------------------------------------------------------------
 // Kernel 2: scan.  One CTA per (sequence, head, value slice of width NV).
+//
+// The chunk-to-chunk dependency is S -> U = U' - W S -> dS = K^T U~ -> S,
+// two small dependent products per chunk (64x128 by 128xNV, then 128x64 by
+// 64xNV).  On tcgen05 each such instruction costs about 90 cycles of pipe
+// time whatever its size plus a commit round trip, so this latency-bound
+// chain runs on register-fragment tensor-core MMAs (mma.sync m16n8k16,
+// bf16 in, fp32 accumulate), operands loaded from shared memory with
+// ldmatrix:
+//   warps 0..3  scan: carry the fp32 state as accumulator fragments (warp w
+//               owns key rows 32w..32w+31), compute U, U~ and the update;
+//   warps 4..7  output: O = scale (e^g Q S + P U) for the chunk, concurrently
+//               with the next chunk's scan (double-buffered S and U);
+//   warp 8      producer: Q, K tiles by TMA and the prep images (W, P, U', g)
+//               by bulk copies into a 3-stage ring.
 // ---------------------------------------------------------------------------
-constexpr int kScanThreads = 192;     // warp 0 loads, warp 1 MMA, warps 2..5 compute
-constexpr uint32_t kScanTmemCols = 256;
-// per-stage shared memory (bytes): Q 16K | K 16K | W 16K | P 8K | U' <= 8K | g 256
-constexpr uint32_t SS_Q = 0, SS_K = 16384, SS_W = 32768, SS_P = 49152, SS_U = 57344, SS_G = 65536;
-constexpr uint32_t SS_STAGE = 66560;                  // 65 KiB (multiple of 1024)
-constexpr uint32_t SC_S = 2 * SS_STAGE;               // state [128 x NV] bf16 MN-major (<= 16K)
-constexpr uint32_t SC_U = SC_S + 16384;               // U  [64 x NV] (<= 8K)
-constexpr uint32_t SC_UT = SC_U + 8192;               // U~ [64 x NV]
-constexpr uint32_t SC_BAR = SC_UT + 8192;
-constexpr int kScanBars = 8;
-constexpr uint32_t SC_TMEMPTR = SC_BAR + kScanBars * 8;
-constexpr uint32_t SC_FLAGS = SC_TMEMPTR + 4;
-constexpr uint32_t kScanSmem = SC_FLAGS + 4 + 1024;
-constexpr uint32_t ST_U = 0, ST_O1 = 64, ST_O2 = 128, ST_DS = 192;   // TMEM columns (NV <= 64)
-enum ScanBar { SB_FULL0 = 0, SB_FULL1, SB_EMPTY0, SB_EMPTY1, SB_UDONE, SB_DSDONE, SB_SREADY, SB_UREADY };
+constexpr int kScanThreads = 288;
+constexpr int kScanStages = 3;
+// per-stage shared memory (bytes)
+constexpr uint32_t SS_Q = 0, SS_K = 16384, SS_W = 32768, SS_P = 49152, SS_U = 57344, SS_G = 61440;
+constexpr uint32_t SS_STAGE = 62464;                         // multiple of 1024
+constexpr uint32_t SC_SS = kScanStages * SS_STAGE;           // 2 x state  [128][RS] bf16
+constexpr uint32_t SC_US = SC_SS + 2 * 128 * 80;             // 2 x U      [64][RS]
+constexpr uint32_t SC_UT = SC_US + 2 * 64 * 80;              // U~         [64][RS]
+constexpr uint32_t SC_BAR = SC_UT + 64 * 80;
+enum ScanBar { SB_FULL = 0, SB_EMPTY = 3, SB_SREADY = 6, SB_UREADY = 8, SB_ODONE = 10, kScanBars = 12 };
+constexpr uint32_t SC_FLAGS = SC_BAR + kScanBars * 8;
+constexpr uint32_t kScanSmem = SC_FLAGS + 16 + 1024;
 
 struct ScanMaps {
     CUtensorMap q, k;
 };
+
+__device__ __forceinline__ void ldsm_x4(uint32_t addr, uint32_t *r) {
+    asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0,%1,%2,%3}, [%4];"
+                 : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3])
+                 : "r"(addr));
+}
+__device__ __forceinline__ void ldsm_x4_t(uint32_t addr, uint32_t *r) {
+    asm volatile("ldmatrix.sync.aligned.m8n8.x4.trans.shared.b16 {%0,%1,%2,%3}, [%4];"
+                 : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3])
+                 : "r"(addr));
+}
+// D += A(16x16, row) * B(16x8, col): bf16 inputs, fp32 accumulate.
+__device__ __forceinline__ void mma16816(float *d, const uint32_t *a, uint32_t b0, uint32_t b1) {
+    asm volatile(
+        "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
+        "{%0,%1,%2,%3};"
+        : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+        : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
+}
+// ldmatrix row address for the 16x16 tile at (row0, col0) of a bf16 K-major
+// SW128 image (64-column halves of `halfbytes`, 128-byte rows).  Lane i
+// addresses row (i&7) + 8((i>>3)&1), column block (i>>4).
+__device__ __forceinline__ uint32_t a_addr_sw128(uint32_t base, int row0, int col0, int lane, uint32_t halfbytes) {
+    const int row = row0 + (lane & 7) + ((lane >> 3) & 1) * 8;
+    const int col = col0 + 8 * (lane >> 4);
+    return base + (col >> 6) * halfbytes + swz(row, (col & 63) >> 3, 128);
+}
+// ldmatrix.trans address giving the A fragment of the transpose of a
+// K-major SW128 image: element (m, k) of the fragment is image[k][m].
+__device__ __forceinline__ uint32_t at_addr_sw128(uint32_t base, int m0, int k0, int lane, uint32_t halfbytes) {
+    const int mi = lane >> 3;
+    const int row = k0 + (lane & 7) + 8 * (mi >> 1);     // image row = k
+    const int col = m0 + 8 * (mi & 1);                   // image column = m
+    return base + (col >> 6) * halfbytes + swz(row, (col & 63) >> 3, 128);
+}
+// ldmatrix.trans address for the two B fragments (n 0..7 and 8..15 from n0)
+// of a row-major [k][n] bf16 buffer with row stride rs bytes.
+__device__ __forceinline__ uint32_t b_addr_rm(uint32_t base, int k0, int n0, int lane, uint32_t rs) {
+    const int row = k0 + (lane & 7) + ((lane >> 3) & 1) * 8;
+    const int col = n0 + 8 * (lane >> 4);
+    return base + row * rs + col * 2;
+}
 
 template <int NV>
 __global__ void __launch_bounds__(kScanThreads, 1)
@@ -558,13 +601,13 @@ scan_kernel(const __grid_constant__ ScanMaps maps, const PrefillArgs a) {
     extern __shared__ uint8_t smem_raw[];
     uint8_t *sm = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     uint64_t *bars = reinterpret_cast<uint64_t *>(sm + SC_BAR);
-    uint32_t *tmem_ptr = reinterpret_cast<uint32_t *>(sm + SC_TMEMPTR);
     volatile int *abort_flag = reinterpret_cast<volatile int *>(sm + SC_FLAGS);
-    constexpr uint32_t VROW = NV * 2;
-    constexpr uint32_t VSW = NV == 64 ? kSw128 : (NV == 32 ? kSw64 : kSw32);
-    constexpr uint32_t VBYTES = 64 * VROW;
+    constexpr int NT = NV / 8;                  // n-tiles of 8 columns
+    constexpr uint32_t RS = NV * 2 + 16;        // padded row stride of the S / U buffers
+    constexpr uint32_t UBYTES = 64 * NV * 2;    // U' slice bytes
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int g = lane >> 2, tg = lane & 3;
     const int slice = blockIdx.x, h = blockIdx.y;
     const int n = a.order ? a.order[blockIdx.z] : (int)blockIdx.z;
     long t0, len, gc0;
@@ -580,12 +623,17 @@ scan_kernel(const __grid_constant__ ScanMaps maps, const PrefillArgs a) {
     const int nchunks = (int)((len + kC - 1) / kC);
     const int j0 = slice * NV;
     const int H = a.H, Dv = a.Dv;
-    const size_t cb = a.chunk_bytes;
 
     if (threadIdx.x == 0) {
-        // a stage is free again once its MMAs are done (commit) and the
-        // compute warps have read its g and U' (arrive): two arrivals
-        for (int i = 0; i < kScanBars; ++i) mbar_init(&bars[i], (i == SB_EMPTY0 || i == SB_EMPTY1) ? 2 : 1);
+        for (int i = 0; i < kScanStages; ++i) {
+            mbar_init(&bars[SB_FULL + i], 1);
+            mbar_init(&bars[SB_EMPTY + i], 256);
+        }
+        for (int i = 0; i < 2; ++i) {
+            mbar_init(&bars[SB_SREADY + i], 1);
+            mbar_init(&bars[SB_UREADY + i], 1);
+            mbar_init(&bars[SB_ODONE + i], 128);
+        }
         *abort_flag = 0;
         fence_mbar_init();
         if (nchunks > 0) {
@@ -593,24 +641,21 @@ scan_kernel(const __grid_constant__ ScanMaps maps, const PrefillArgs a) {
             prefetch_tensormap(&maps.k);
         }
     }
-    if (warp == 1) {
-        tmem_alloc(tmem_ptr, kScanTmemCols);
-        tmem_relinquish();
-    }
-    tc_fence_before();
     __syncthreads();
-    tc_fence_after();
-    const uint32_t tmem = *tmem_ptr;
+    const uint32_t smb = smem_u32(sm);
 
-    if (warp == 0) {
+    if (warp == 8) {
+        // ------------------------------------------------------------ producer
         if (lane == 0) {
             for (int c = 0; c < nchunks; ++c) {
-                const int st = c & 1;
-                if (c >= 2 && !wait_bar(&bars[SB_EMPTY0 + st], ((c >> 1) - 1) & 1, abort_flag, a.err)) break;
-                uint64_t *full = &bars[SB_FULL0 + st];
+                const int st = c % kScanStages;
+                if (c >= kScanStages &&
+                    !wait_bar(&bars[SB_EMPTY + st], (c / kScanStages - 1) & 1, abort_flag, a.err))
+                    break;
+                uint64_t *full = &bars[SB_FULL + st];
                 uint8_t *stg = sm + st * SS_STAGE;
-                const uint8_t *img = a.workspace_chunks + ((size_t)(gc0 + c) * H + h) * cb;
-                mbar_arrive_expect_tx(full, 16384 * 3 + 8192 + VBYTES + 256);
+                const uint8_t *img = a.workspace_chunks + ((size_t)(gc0 + c) * H + h) * a.chunk_bytes;
+                mbar_arrive_expect_tx(full, 16384 * 3 + 8192 + UBYTES + 256);
                 const int r0 = (int)(t0 + (long)c * kC);
                 tma_load_3d(stg + SS_Q, &maps.q, full, 0, h, r0);
                 tma_load_3d(stg + SS_Q + 8192, &maps.q, full, 64, h, r0);
@@ -618,175 +663,208 @@ scan_kernel(const __grid_constant__ ScanMaps maps, const PrefillArgs a) {
                 tma_load_3d(stg + SS_K + 8192, &maps.k, full, 64, h, r0);
                 bulk_load(stg + SS_W, img + kImgW, 16384, full);
                 bulk_load(stg + SS_P, img + kImgP, 8192, full);
-                bulk_load(stg + SS_U, img + kImgU + (size_t)slice * VBYTES, VBYTES, full);
+                bulk_load(stg + SS_U, img + kImgU + (size_t)slice * UBYTES, UBYTES, full);
                 bulk_load(stg + SS_G, img + kImgU + 64 * Dv * 2, 256, full);
             }
         }
-    } else if (warp == 1) {
-        if (lane == 0) {
-            const uint32_t base = smem_u32(sm);
-            const uint32_t ss = smem_u32(sm + SC_S), uu = smem_u32(sm + SC_U), ut = smem_u32(sm + SC_UT);
-            constexpr uint32_t ID_NEG = idesc_bf16(64, NV, 0, 1, 1);
-            constexpr uint32_t ID_O = idesc_bf16(64, NV, 0, 1);
-            constexpr uint32_t ID_DS = idesc_bf16(128, NV, 1, 1);
-            for (int c = 0; c < nchunks; ++c) {
-                const int st = c & 1;
-                const uint32_t ph = c & 1;
-                const uint32_t stg = base + st * SS_STAGE;
-                if (!wait_bar(&bars[SB_FULL0 + st], (c >> 1) & 1, abort_flag, a.err)) break;
-                if (!wait_bar(&bars[SB_SREADY], ph, abort_flag, a.err)) break;
-                tc_fence_after();
-                // U = -W S (U' is added by the compute warps) ; O1 = Q S
+    } else if (warp < 4) {
+        // ------------------------------------------------------------ scan warps
+        const int w = warp;
+        const int tid = threadIdx.x;
+        // S fragments: rows d = 32w + 16mt + g (+8), columns 8nt + 2tg (+1)
+        float S[2][NT][4];
+        const size_t sb = ((size_t)n * H + h) * kDK * Dv + j0;
 #pragma unroll
-                for (int kk = 0; kk < 8; ++kk) {
-                    const uint64_t bs = smem_desc(ss + kk * 16 * VROW, 128 * VROW, 8 * VROW, VSW);
-                    const uint32_t off = (kk >> 2) * 8192 + (kk & 3) * 32;
-                    mma_bf16(tmem + ST_U, smem_desc(stg + SS_W + off, 16, 1024, kSw128), bs, ID_NEG, kk > 0);
-                    mma_bf16(tmem + ST_O1, smem_desc(stg + SS_Q + off, 16, 1024, kSw128), bs, ID_O, kk > 0);
+        for (int mt = 0; mt < 2; ++mt)
+#pragma unroll
+            for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+                for (int hh = 0; hh < 2; ++hh) {
+                    const int d = 32 * w + 16 * mt + g + 8 * hh, j = 8 * nt + 2 * tg;
+                    float2 x = make_float2(0.f, 0.f);
+                    if (a.s0) x = *reinterpret_cast<const float2 *>(a.s0 + sb + (size_t)d * Dv + j);
+                    S[mt][nt][2 * hh] = x.x;
+                    S[mt][nt][2 * hh + 1] = x.y;
                 }
-                mma_commit(&bars[SB_UDONE]);
-                if (!wait_bar(&bars[SB_UREADY], ph, abort_flag, a.err)) break;
-                tc_fence_after();
-                // dS = K^T U~ (A = K tile, MN-major) ; O2 = P U
-#pragma unroll
-                for (int kk = 0; kk < 4; ++kk) {
-                    mma_bf16(tmem + ST_DS, smem_desc(stg + SS_K + kk * 2048, 8192, 1024, kSw128),
-                             smem_desc(ut + kk * 16 * VROW, VBYTES, 8 * VROW, VSW), ID_DS, kk > 0);
-                    mma_bf16(tmem + ST_O2, smem_desc(stg + SS_P + kk * 32, 16, 1024, kSw128),
-                             smem_desc(uu + kk * 16 * VROW, VBYTES, 8 * VROW, VSW), ID_O, kk > 0);
-                }
-                mma_commit(&bars[SB_DSDONE]);
-                mma_commit(&bars[SB_EMPTY0 + st]);
-            }
-        }
-    } else {
-        const int cw = threadIdx.x - 64;
-        const int q4 = warp & 3;
-        const int r = 32 * q4 + lane;
-        const bool lo = lane < 16;
-        const int m = 16 * q4 + lane;
-        const uint32_t tq = tmem + ((uint32_t)(32 * q4) << 16);
-        const size_t sbase = ((size_t)n * H + h) * kDK * Dv + (size_t)r * Dv + j0;
-        __nv_bfloat16 *out = static_cast<__nv_bfloat16 *>(a.out);
-
-        float S[NV];
-#pragma unroll
-        for (int j = 0; j < NV; j += 4) {
-            float4 x = make_float4(0.f, 0.f, 0.f, 0.f);
-            if (a.s0) x = *reinterpret_cast<const float4 *>(a.s0 + sbase + j);
-            S[j] = x.x; S[j + 1] = x.y; S[j + 2] = x.z; S[j + 3] = x.w;
-        }
         for (int c = 0; c < nchunks; ++c) {
-            const int st = c & 1;
-            const uint32_t ph = c & 1;
-            const int lenc = (int)min((long)kC, len - (long)c * kC);
-            const uint8_t *stg = sm + st * SS_STAGE;
-            const float *g_s = reinterpret_cast<const float *>(stg + SS_G);
-            // state -> bf16 MN-major operand
-#pragma unroll
-            for (int cc = 0; cc < NV / 8; ++cc)
-                *reinterpret_cast<uint4 *>(sm + SC_S + swz(r, cc, VROW)) = pack8(S + 8 * cc);
-            fence_proxy_async_smem();
-            named_bar_sync(1, 128);
-            if (cw == 0) {
-                mbar_arrive(&bars[SB_SREADY]);
-                // the stage's loads landed before the MMA warp used it; wait for
-                // them here too, since g and U' are read directly below
-                if (!wait_bar(&bars[SB_FULL0 + st], (c >> 1) & 1, abort_flag, a.err) ||
-                    !wait_bar(&bars[SB_UDONE], ph, abort_flag, a.err))
-                    *abort_flag = 1;
+            const int st = c % kScanStages, buf = c & 1;
+            const uint32_t stg = smb + st * SS_STAGE;
+            const float *g_s = reinterpret_cast<const float *>(sm + st * SS_STAGE + SS_G);
+            if (tid == 0) {
+                bool ok = wait_bar(&bars[SB_FULL + st], (c / kScanStages) & 1, abort_flag, a.err);
+                if (ok && c >= 2) ok = wait_bar(&bars[SB_ODONE + buf], ((c >> 1) - 1) & 1, abort_flag, a.err);
+                if (!ok) *abort_flag = 1;
             }
             named_bar_sync(1, 128);
             if (*abort_flag) break;
-            tc_fence_after();
+            // ---- S -> bf16 row-major [d][j]
+            const uint32_t ssb = smb + SC_SS + buf * (128 * 80);
+#pragma unroll
+            for (int mt = 0; mt < 2; ++mt)
+#pragma unroll
+                for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+                    for (int hh = 0; hh < 2; ++hh) {
+                        const int d = 32 * w + 16 * mt + g + 8 * hh, j = 8 * nt + 2 * tg;
+                        *reinterpret_cast<uint32_t *>(sm + SC_SS + buf * (128 * 80) + d * RS + j * 2) =
+                            pack_bf16(S[mt][nt][2 * hh], S[mt][nt][2 * hh + 1]);
+                    }
+            named_bar_sync(1, 128);
+            if (tid == 0) mbar_arrive(&bars[SB_SREADY + buf]);
+            // ---- U = U' - W S for rows t = 16w .. 16w+15
+            float acc[NT][4];
+#pragma unroll
+            for (int nt = 0; nt < NT; ++nt) acc[nt][0] = acc[nt][1] = acc[nt][2] = acc[nt][3] = 0.f;
+#pragma unroll
+            for (int ks = 0; ks < 8; ++ks) {
+                uint32_t af[4];
+                ldsm_x4(a_addr_sw128(stg + SS_W, 16 * w, 16 * ks, lane, 8192), af);
+#pragma unroll
+                for (int n2 = 0; n2 < NV / 16; ++n2) {
+                    uint32_t bf[4];
+                    ldsm_x4_t(b_addr_rm(ssb, 16 * ks, 16 * n2, lane, RS), bf);
+                    mma16816(acc[2 * n2], af, bf[0], bf[1]);
+                    mma16816(acc[2 * n2 + 1], af, bf[2], bf[3]);
+                }
+            }
             const float gC = g_s[63];
-            // U = U' - W S ; U~ = e^{g_C - g} U
-            {
-                float x[NV];
+            const int ta = 16 * w + g, tb = ta + 8;
+            const float da = __expf(gC - g_s[ta]), db = __expf(gC - g_s[tb]);
+            const uint8_t *up = sm + st * SS_STAGE + SS_U;
 #pragma unroll
-                for (int cc = 0; cc < NV / 16; ++cc) tmem_ld16(tq + ST_U + 16 * cc, x + 16 * cc);
-                tmem_wait_ld();
-                if (lo) {
-                    const uint8_t *urow = stg + SS_U + m * VROW;
-#pragma unroll
-                    for (int cc = 0; cc < NV / 8; ++cc) {
-                        float u[8];
-                        unpack8(*reinterpret_cast<const uint4 *>(urow + 16 * cc), u);
-#pragma unroll
-                        for (int e = 0; e < 8; ++e) x[8 * cc + e] += u[e];
-                    }
-                    const float dec = __expf(gC - g_s[m]);
-#pragma unroll
-                    for (int cc = 0; cc < NV / 8; ++cc) {
-                        *reinterpret_cast<uint4 *>(sm + SC_U + swz(m, cc, VROW)) = pack8(x + 8 * cc);
-                        float y[8];
-#pragma unroll
-                        for (int e = 0; e < 8; ++e) y[e] = x[8 * cc + e] * dec;
-                        *reinterpret_cast<uint4 *>(sm + SC_UT + swz(m, cc, VROW)) = pack8(y);
-                    }
-                }
-            }
-            fence_proxy_async_smem();
-            tc_fence_before();
-            named_bar_sync(1, 128);
-            if (cw == 0) {
-                mbar_arrive(&bars[SB_UREADY]);
-                if (!wait_bar(&bars[SB_DSDONE], ph, abort_flag, a.err)) *abort_flag = 1;
+            for (int nt = 0; nt < NT; ++nt) {
+                const int j = 8 * nt + 2 * tg;
+                const __nv_bfloat162 ua = *reinterpret_cast<const __nv_bfloat162 *>(up + (ta * NV + j) * 2);
+                const __nv_bfloat162 ub = *reinterpret_cast<const __nv_bfloat162 *>(up + (tb * NV + j) * 2);
+                const float2 fa = __bfloat1622float2(ua), fb = __bfloat1622float2(ub);
+                const float u0 = fa.x - acc[nt][0], u1 = fa.y - acc[nt][1];
+                const float u2 = fb.x - acc[nt][2], u3 = fb.y - acc[nt][3];
+                uint8_t *usb = sm + SC_US + buf * (64 * 80);
+                *reinterpret_cast<uint32_t *>(usb + ta * RS + j * 2) = pack_bf16(u0, u1);
+                *reinterpret_cast<uint32_t *>(usb + tb * RS + j * 2) = pack_bf16(u2, u3);
+                *reinterpret_cast<uint32_t *>(sm + SC_UT + ta * RS + j * 2) = pack_bf16(u0 * da, u1 * da);
+                *reinterpret_cast<uint32_t *>(sm + SC_UT + tb * RS + j * 2) = pack_bf16(u2 * db, u3 * db);
             }
             named_bar_sync(1, 128);
-            if (*abort_flag) break;
-            tc_fence_after();
-            // S <- e^{g_C} S + K^T U~
-            {
-                const float eC = __expf(gC);
-                float x[NV];
+            if (tid == 0) mbar_arrive(&bars[SB_UREADY + buf]);
+            // ---- S <- e^{g_C} S + K^T U~ for rows d = 32w .. 32w+31
+            float ds[2][NT][4];
 #pragma unroll
-                for (int cc = 0; cc < NV / 16; ++cc) tmem_ld16(tq + ST_DS + 16 * cc, x + 16 * cc);
-                tmem_wait_ld();
+            for (int mt = 0; mt < 2; ++mt)
 #pragma unroll
-                for (int j = 0; j < NV; ++j) S[j] = fmaf(eC, S[j], x[j]);
-            }
-            // O = scale (e^{g} Q S + P U)
-            {
-                float o1[NV], o2[NV];
+                for (int nt = 0; nt < NT; ++nt) ds[mt][nt][0] = ds[mt][nt][1] = ds[mt][nt][2] = ds[mt][nt][3] = 0.f;
 #pragma unroll
-                for (int cc = 0; cc < NV / 16; ++cc) {
-                    tmem_ld16(tq + ST_O1 + 16 * cc, o1 + 16 * cc);
-                    tmem_ld16(tq + ST_O2 + 16 * cc, o2 + 16 * cc);
-                }
-                tmem_wait_ld();
-                if (lo && m < lenc) {
-                    const float eg = __expf(g_s[m]) * a.scale;
-                    const float sc = a.scale;
-                    __nv_bfloat16 *orow = out + ((size_t)(t0 + (long)c * kC + m) * H + h) * Dv + j0;
+            for (int ks = 0; ks < 4; ++ks) {
+                uint32_t bf[NV / 16][4];
 #pragma unroll
-                    for (int cc = 0; cc < NV / 8; ++cc) {
-                        float y[8];
+                for (int n2 = 0; n2 < NV / 16; ++n2)
+                    ldsm_x4_t(b_addr_rm(smb + SC_UT, 16 * ks, 16 * n2, lane, RS), bf[n2]);
 #pragma unroll
-                        for (int e = 0; e < 8; ++e) y[e] = fmaf(eg, o1[8 * cc + e], sc * o2[8 * cc + e]);
-                        *reinterpret_cast<uint4 *>(orow + 8 * cc) = pack8(y);
+                for (int mt = 0; mt < 2; ++mt) {
+                    uint32_t af[4];
+                    ldsm_x4_t(at_addr_sw128(stg + SS_K, 32 * w + 16 * mt, 16 * ks, lane, 8192), af);
+#pragma unroll
+                    for (int n2 = 0; n2 < NV / 16; ++n2) {
+                        mma16816(ds[mt][2 * n2], af, bf[n2][0], bf[n2][1]);
+                        mma16816(ds[mt][2 * n2 + 1], af, bf[n2][2], bf[n2][3]);
                     }
                 }
             }
-            tc_fence_before();
-            named_bar_sync(1, 128);
-            if (cw == 0) mbar_arrive(&bars[SB_EMPTY0 + st]);
+            const float eC = __expf(gC);
+#pragma unroll
+            for (int mt = 0; mt < 2; ++mt)
+#pragma unroll
+                for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+                    for (int i = 0; i < 4; ++i) S[mt][nt][i] = fmaf(eC, S[mt][nt][i], ds[mt][nt][i]);
+            mbar_arrive(&bars[SB_EMPTY + st]);
         }
         if (a.sf && !*abort_flag) {
 #pragma unroll
-            for (int j = 0; j < NV; j += 4)
-                *reinterpret_cast<float4 *>(a.sf + sbase + j) = make_float4(S[j], S[j + 1], S[j + 2], S[j + 3]);
+            for (int mt = 0; mt < 2; ++mt)
+#pragma unroll
+                for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+                    for (int hh = 0; hh < 2; ++hh) {
+                        const int d = 32 * w + 16 * mt + g + 8 * hh, j = 8 * nt + 2 * tg;
+                        *reinterpret_cast<float2 *>(a.sf + sb + (size_t)d * Dv + j) =
+                            make_float2(S[mt][nt][2 * hh], S[mt][nt][2 * hh + 1]);
+                    }
         }
-    }
-
-    tc_fence_before();
-    __syncthreads();
-    if (warp == 1) {
-        tc_fence_after();
-        tmem_dealloc(tmem, kScanTmemCols);
+    } else {
+        // ------------------------------------------------------------ output warps
+        const int w = warp - 4;
+        const int tid = threadIdx.x - 128;
+        __nv_bfloat16 *out = static_cast<__nv_bfloat16 *>(a.out);
+        for (int c = 0; c < nchunks; ++c) {
+            const int st = c % kScanStages, buf = c & 1;
+            const uint32_t stg = smb + st * SS_STAGE;
+            const float *g_s = reinterpret_cast<const float *>(sm + st * SS_STAGE + SS_G);
+            const int lenc = (int)min((long)kC, len - (long)c * kC);
+            if (tid == 0) {
+                bool ok = wait_bar(&bars[SB_FULL + st], (c / kScanStages) & 1, abort_flag, a.err);
+                if (ok) ok = wait_bar(&bars[SB_SREADY + buf], (c >> 1) & 1, abort_flag, a.err);
+                if (!ok) *abort_flag = 1;
+            }
+            named_bar_sync(2, 128);
+            if (*abort_flag) break;
+            // O1 = Q S for rows t = 16w .. 16w+15
+            const uint32_t ssb = smb + SC_SS + buf * (128 * 80);
+            float o1[NT][4], o2[NT][4];
+#pragma unroll
+            for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+                for (int i = 0; i < 4; ++i) o1[nt][i] = o2[nt][i] = 0.f;
+#pragma unroll
+            for (int ks = 0; ks < 8; ++ks) {
+                uint32_t af[4];
+                ldsm_x4(a_addr_sw128(stg + SS_Q, 16 * w, 16 * ks, lane, 8192), af);
+#pragma unroll
+                for (int n2 = 0; n2 < NV / 16; ++n2) {
+                    uint32_t bf[4];
+                    ldsm_x4_t(b_addr_rm(ssb, 16 * ks, 16 * n2, lane, RS), bf);
+                    mma16816(o1[2 * n2], af, bf[0], bf[1]);
+                    mma16816(o1[2 * n2 + 1], af, bf[2], bf[3]);
+                }
+            }
+            if (tid == 0 && !wait_bar(&bars[SB_UREADY + buf], (c >> 1) & 1, abort_flag, a.err)) *abort_flag = 1;
+            named_bar_sync(2, 128);
+            if (*abort_flag) break;
+            // O2 = P U
+            const uint32_t usb = smb + SC_US + buf * (64 * 80);
+#pragma unroll
+            for (int ks = 0; ks < 4; ++ks) {
+                uint32_t af[4];
+                ldsm_x4(a_addr_sw128(stg + SS_P, 16 * w, 16 * ks, lane, 8192), af);
+#pragma unroll
+                for (int n2 = 0; n2 < NV / 16; ++n2) {
+                    uint32_t bf[4];
+                    ldsm_x4_t(b_addr_rm(usb, 16 * ks, 16 * n2, lane, RS), bf);
+                    mma16816(o2[2 * n2], af, bf[0], bf[1]);
+                    mma16816(o2[2 * n2 + 1], af, bf[2], bf[3]);
+                }
+            }
+            const int ta = 16 * w + g, tb = ta + 8;
+            const float ea = __expf(g_s[ta]) * a.scale, eb = __expf(g_s[tb]) * a.scale;
+            const float sc = a.scale;
+            const long rowa = t0 + (long)c * kC + ta, rowb = rowa + 8;
+#pragma unroll
+            for (int nt = 0; nt < NT; ++nt) {
+                const int j = j0 + 8 * nt + 2 * tg;
+                if (ta < lenc)
+                    *reinterpret_cast<uint32_t *>(out + ((size_t)rowa * H + h) * Dv + j) =
+                        pack_bf16(fmaf(ea, o1[nt][0], sc * o2[nt][0]), fmaf(ea, o1[nt][1], sc * o2[nt][1]));
+                if (tb < lenc)
+                    *reinterpret_cast<uint32_t *>(out + ((size_t)rowb * H + h) * Dv + j) =
+                        pack_bf16(fmaf(eb, o1[nt][2], sc * o2[nt][2]), fmaf(eb, o1[nt][3], sc * o2[nt][3]));
+            }
+            mbar_arrive(&bars[SB_ODONE + buf]);
+            mbar_arrive(&bars[SB_EMPTY + st]);
+        }
     }
 }
 
+// ---------------------------------------------------------------------------
 // Exclusive prefix sum of ceil(len_n / 64) over packed sequences (one CTA).
 __global__ void __launch_bounds__(1024) chunk_base_kernel(const int32_t *cu_seqlens, int num_seqs,
                                                           int32_t *chunk_base) {
@@ -860,11 +938,9 @@ cudaError_t set_smem(K kernel, uint32_t bytes) {
 }
 
 int choose_nv(long units, int Dv) {
-    // The scan is latency-bound per chunk, so narrow slices cost little and
-    // give more CTAs; widen them once the SMs are covered.
-    if (units * (Dv / 64) >= 2 * 148) return 64;
-    if (units * (Dv / 32) >= 148) return 32;
-    return 16;
+    // The scan is latency-bound per chunk: narrow slices give more CTAs at
+    // little extra cost; widen them once the SMs are covered.
+    return units * (Dv / 32) >= 148 ? 32 : 16;
 }
 
 template <int NV>
@@ -935,11 +1011,7 @@ cudaError_t launch_chunked(const PrefillArgs &a0, void *scratch, cudaStream_t s)
     }
     if (a.total_T == 0) chunks_grid = 0;
     const long units = (long)a.num_seqs * a.H;
-    switch (choose_nv(units, a.Dv)) {
-        case 64: return launch_nv<64>(a, chunks_grid, s);
-        case 32: return launch_nv<32>(a, chunks_grid, s);
-        default: return launch_nv<16>(a, chunks_grid, s);
-    }
+    return choose_nv(units, a.Dv) == 32 ? launch_nv<32>(a, chunks_grid, s) : launch_nv<16>(a, chunks_grid, s);
 }
 
 }  // namespace rda
