@@ -55,11 +55,14 @@ constexpr int kC = 64;            // chunk length
 constexpr int kDK = 128;          // key dimension handled here
 constexpr uint64_t kWaitNs = 4000000000ull;   // bounded waits: 4 s
 
-// Per (chunk, head) prep image in the workspace.
-constexpr uint32_t kImgW = 0;          // W, bf16 K-major SW128 image, 2 halves of 8 KiB
-constexpr uint32_t kImgP = 16384;      // P, bf16 K-major SW128 image, 8 KiB
-constexpr uint32_t kImgU = 24576;      // U', bf16, value slices of width NV, each [64][NV]
-                                       // (then g: 64 fp32 after 64*Dv*2 bytes)
+// Per (chunk, head) image in the workspace (bytes).
+constexpr uint32_t kImgW = 0;          // -W, bf16 K-major SW128, 2 halves of 8 KiB (64 rows x 64 cols)
+constexpr uint32_t kImgQ = 16384;      // diag(e^g) Q, same layout
+constexpr uint32_t kImgP = 32768;      // P, bf16 K-major SW128, 8 KiB
+constexpr uint32_t kImgS = 40960;      // state entering the chunk, bf16 MN-major SW128:
+                                       // atoms of 64 value columns, [128 key rows x 128 B] each
+constexpr uint32_t kImgU = 73728;      // U', bf16, value slices of width NV, each [64][NV];
+                                       // then e^{g_t} and e^{g_C - g_t}: 2 x 64 fp32
 
 __device__ __forceinline__ uint64_t globaltimer() {
     uint64_t t;
@@ -224,8 +227,8 @@ constexpr uint32_t PS_P = 49152;       // P image (8 KiB)
 constexpr uint32_t PS_AF = 57344;      // A fp32 [64][kLd]
 constexpr uint32_t PS_TF = PS_AF + 64 * kLd * 4;
 constexpr uint32_t PS_XS = PS_TF + 64 * kLd * 4;     // 4 x 16x8 fp32
-constexpr uint32_t PS_G = PS_XS + 4 * 128 * 4;       // g, beta, beta*gamma, e^g, e^{ref-g}: 5 x 64 fp32
-constexpr uint32_t PS_BAR = PS_G + 5 * 64 * 4;
+constexpr uint32_t PS_G = PS_XS + 4 * 128 * 4;       // g, beta, beta*gamma, e^{ref-g}, e^g, e^{g_C-g}: 6 x 64 fp32
+constexpr uint32_t PS_BAR = PS_G + 6 * 64 * 4;
 constexpr uint32_t PS_TMEMPTR = PS_BAR + 4 * 8;
 constexpr uint32_t PS_FLAGS = PS_TMEMPTR + 4;
 constexpr uint32_t kPrepSmem = PS_FLAGS + 4 + 1024;
@@ -291,7 +294,8 @@ prep_kernel(const __grid_constant__ PrepMaps maps, const PrefillArgs a) {
     uint32_t *tmem_ptr = reinterpret_cast<uint32_t *>(sm + PS_TMEMPTR);
     volatile int *abort_flag = reinterpret_cast<volatile int *>(sm + PS_FLAGS);
     float *g_s = reinterpret_cast<float *>(sm + PS_G);
-    float *b_s = g_s + 64, *bg_s = g_s + 128, *eg_s = g_s + 192, *eb_s = g_s + 256;
+    float *b_s = g_s + 64, *bg_s = g_s + 128, *eb_s = g_s + 192;
+    float *eg_s = g_s + 256, *ed_s = g_s + 320;   // stored for the scan: e^g, e^{g_C - g}
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
 
     if (threadIdx.x == 0) {
@@ -388,6 +392,7 @@ prep_kernel(const __grid_constant__ PrepMaps maps, const PrefillArgs a) {
             // (g is non-increasing, so 0 <= ref - g_s <= 80 and the factor stays finite)
             eg_s[r] = __expf(g_s[r]);
             eb_s[r] = __expf(g_s[r & ~15] - g_s[r]);
+            ed_s[r] = __expf(g_s[63] - g_s[r]);
         }
         if (cw == 0 && !wait_bar(&bars[PB_QK], 0, abort_flag, a.err)) *abort_flag = 1;
         named_bar_sync(1, 128);
@@ -429,15 +434,39 @@ prep_kernel(const __grid_constant__ PrepMaps maps, const PrefillArgs a) {
                     *reinterpret_cast<float4 *>(Af + t * kLd + 4 * c4) = make_float4(y[0], y[1], y[2], y[3]);
                 }
             }
+            // diag(e^g) Q, in place over Q (Q was read only by the first MMA): row t = cw/2,
+            // 64 of its 128 columns per thread
+            {
+                const int tq2 = cw >> 1, half = cw & 1;
+                const float e = eg_s[tq2];
+                uint8_t *row = sm + PS_QK + half * 16384;
+#pragma unroll
+                for (int cc = 0; cc < 8; ++cc) {
+                    uint4 *pq = reinterpret_cast<uint4 *>(row + swz(tq2, cc, 128));
+                    uint4 u = *pq;
+                    uint32_t wv[4] = {u.x, u.y, u.z, u.w};
+#pragma unroll
+                    for (int i = 0; i < 4; ++i) {
+                        float2 f = __bfloat1622float2(*reinterpret_cast<__nv_bfloat162 *>(&wv[i]));
+                        wv[i] = pack_bf16(f.x * e, f.y * e);
+                    }
+                    *pq = make_uint4(wv[0], wv[1], wv[2], wv[3]);
+                }
+            }
         }
         fence_proxy_async_smem();
         named_bar_sync(1, 128);
         if (!*abort_flag) {
             if (cw == 0) {
                 bulk_store(img + kImgP, sm + PS_P, 8192);
+                bulk_store(img + kImgQ, sm + PS_QK, 8192);
+                bulk_store(img + kImgQ + 8192, sm + PS_QK + 16384, 8192);
                 bulk_commit();
             }
             ut_solve(Af, Tf, Xs, cw);
+            // T diag(..) images overwrite diag(e^g) Q: its store must have read it
+            if (cw == 0) bulk_wait_reads();
+            named_bar_sync(1, 128);
             // T diag(beta e^g) and T diag(beta gamma) as bf16 K-major SW128 images
             {
                 const int t = cw >> 1, half = cw & 1;
@@ -468,13 +497,15 @@ prep_kernel(const __grid_constant__ PrepMaps maps, const PrefillArgs a) {
         named_bar_sync(1, 128);
         if (!*abort_flag) {
             tc_fence_after();
-            // W rows -> bf16 K-major SW128 image (2 halves of 64 columns)
+            // -W rows -> bf16 K-major SW128 image (2 halves of 64 columns)
 #pragma unroll
             for (int half = 0; half < 2; ++half) {
                 float x[64];
 #pragma unroll
                 for (int cc = 0; cc < 4; ++cc) tmem_ld16(tq + PT_W + 64 * half + 16 * cc, x + 16 * cc);
                 tmem_wait_ld();
+#pragma unroll
+                for (int i = 0; i < 64; ++i) x[i] = -x[i];
                 if (lo) {
 #pragma unroll
                     for (int cc = 0; cc < 8; ++cc)
@@ -504,10 +535,10 @@ prep_kernel(const __grid_constant__ PrepMaps maps, const PrefillArgs a) {
             if (!*abort_flag) {
                 bulk_store(img + kImgW, sm + PS_WIMG, 16384);
                 bulk_store(img + kImgU, sm + PS_UIMG, 64 * Dv * 2);
-                bulk_store(img + kImgU + 64 * Dv * 2, g_s, 256);
+                bulk_store(img + kImgU + 64 * Dv * 2, eg_s, 512);
                 bulk_commit();
             }
-            bulk_wait_all();
+            bulk_wait_reads();
         }
     }
 
@@ -522,35 +553,33 @@ prep_kernel(const __grid_constant__ PrepMaps maps, const PrefillArgs a) {
 // ---------------------------------------------------------------------------
 // Kernel 2: scan.  One CTA per (sequence, head, value slice of width NV).
 //
-// The chunk-to-chunk dependency is S -> U = U' - W S -> dS = K^T U~ -> S,
+// The chunk-to-chunk dependency is S -> U = U' - W S -> S' = e^{g_C} S + K^T U~,
 // two small dependent products per chunk (64x128 by 128xNV, then 128x64 by
 // 64xNV).  On tcgen05 each such instruction costs about 90 cycles of pipe
-// time whatever its size plus a commit round trip, so this latency-bound
-// chain runs on register-fragment tensor-core MMAs (mma.sync m16n8k16,
-// bf16 in, fp32 accumulate), operands loaded from shared memory with
-// ldmatrix:
-//   warps 0..3  scan: carry the fp32 state as accumulator fragments (warp w
-//               owns key rows 32w..32w+31), compute U, U~ and the update;
-//   warps 4..7  output: O = scale (e^g Q S + P U) for the chunk, concurrently
-//               with the next chunk's scan (double-buffered S and U);
-//   warp 8      producer: Q, K tiles by TMA and the prep images (W, P, U', g)
-//               by bulk copies into a 3-stage ring.
+// time whatever its size, plus a commit round trip, so this latency-bound
+// chain runs on register-fragment tensor-core MMAs (mma.sync m16n8k16, bf16
+// in, fp32 accumulate) with ldmatrix operands.  Everything that does not
+// feed the next state (the outputs) is left to the output kernel, which
+// reads the state entering each chunk from the workspace.
+//   warps 0..3  carry the fp32 state as accumulator fragments (warp w owns
+//               key rows 32w..32w+31) and compute U~ and the update;
+//   warp 4      producer: the K tile by TMA, -W, U' and the decay factors by
+//               bulk copies, into a 4-stage ring.
 // ---------------------------------------------------------------------------
-constexpr int kScanThreads = 288;
-constexpr int kScanStages = 3;
-// per-stage shared memory (bytes)
-constexpr uint32_t SS_Q = 0, SS_K = 16384, SS_W = 32768, SS_P = 49152, SS_U = 57344, SS_G = 61440;
-constexpr uint32_t SS_STAGE = 62464;                         // multiple of 1024
-constexpr uint32_t SC_SS = kScanStages * SS_STAGE;           // 2 x state  [128][RS] bf16
-constexpr uint32_t SC_US = SC_SS + 2 * 128 * 80;             // 2 x U      [64][RS]
-constexpr uint32_t SC_UT = SC_US + 2 * 64 * 80;              // U~         [64][RS]
+constexpr int kScanThreads = 160;
+constexpr int kScanStages = 4;
+// per-stage shared memory (bytes): -W 16K | K 16K | U' <= 4K | decay 512
+constexpr uint32_t SS_W = 0, SS_K = 16384, SS_U = 32768, SS_G = 36864;
+constexpr uint32_t SS_STAGE = 37888;                          // multiple of 1024
+constexpr uint32_t SC_SS = kScanStages * SS_STAGE;            // state  [128][RS] bf16
+constexpr uint32_t SC_UT = SC_SS + 128 * 80;                  // U~     [64][RS]
 constexpr uint32_t SC_BAR = SC_UT + 64 * 80;
-enum ScanBar { SB_FULL = 0, SB_EMPTY = 3, SB_SREADY = 6, SB_UREADY = 8, SB_ODONE = 10, kScanBars = 12 };
+enum ScanBar { SB_FULL = 0, SB_EMPTY = kScanStages, kScanBars = 2 * kScanStages };
 constexpr uint32_t SC_FLAGS = SC_BAR + kScanBars * 8;
 constexpr uint32_t kScanSmem = SC_FLAGS + 16 + 1024;
 
 struct ScanMaps {
-    CUtensorMap q, k;
+    CUtensorMap k;
 };
 
 __device__ __forceinline__ void ldsm_x4(uint32_t addr, uint32_t *r) {
@@ -603,7 +632,7 @@ scan_kernel(const __grid_constant__ ScanMaps maps, const PrefillArgs a) {
     uint64_t *bars = reinterpret_cast<uint64_t *>(sm + SC_BAR);
     volatile int *abort_flag = reinterpret_cast<volatile int *>(sm + SC_FLAGS);
     constexpr int NT = NV / 8;                  // n-tiles of 8 columns
-    constexpr uint32_t RS = NV * 2 + 16;        // padded row stride of the S / U buffers
+    constexpr uint32_t RS = NV * 2 + 16;        // padded row stride of the S / U~ buffers
     constexpr uint32_t UBYTES = 64 * NV * 2;    // U' slice bytes
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -627,24 +656,16 @@ scan_kernel(const __grid_constant__ ScanMaps maps, const PrefillArgs a) {
     if (threadIdx.x == 0) {
         for (int i = 0; i < kScanStages; ++i) {
             mbar_init(&bars[SB_FULL + i], 1);
-            mbar_init(&bars[SB_EMPTY + i], 256);
-        }
-        for (int i = 0; i < 2; ++i) {
-            mbar_init(&bars[SB_SREADY + i], 1);
-            mbar_init(&bars[SB_UREADY + i], 1);
-            mbar_init(&bars[SB_ODONE + i], 128);
+            mbar_init(&bars[SB_EMPTY + i], 128);
         }
         *abort_flag = 0;
         fence_mbar_init();
-        if (nchunks > 0) {
-            prefetch_tensormap(&maps.q);
-            prefetch_tensormap(&maps.k);
-        }
+        if (nchunks > 0) prefetch_tensormap(&maps.k);
     }
     __syncthreads();
     const uint32_t smb = smem_u32(sm);
 
-    if (warp == 8) {
+    if (warp == 4) {
         // ------------------------------------------------------------ producer
         if (lane == 0) {
             for (int c = 0; c < nchunks; ++c) {
@@ -655,25 +676,45 @@ scan_kernel(const __grid_constant__ ScanMaps maps, const PrefillArgs a) {
                 uint64_t *full = &bars[SB_FULL + st];
                 uint8_t *stg = sm + st * SS_STAGE;
                 const uint8_t *img = a.workspace_chunks + ((size_t)(gc0 + c) * H + h) * a.chunk_bytes;
-                mbar_arrive_expect_tx(full, 16384 * 3 + 8192 + UBYTES + 256);
+                mbar_arrive_expect_tx(full, 16384 * 2 + UBYTES + 512);
                 const int r0 = (int)(t0 + (long)c * kC);
-                tma_load_3d(stg + SS_Q, &maps.q, full, 0, h, r0);
-                tma_load_3d(stg + SS_Q + 8192, &maps.q, full, 64, h, r0);
                 tma_load_3d(stg + SS_K, &maps.k, full, 0, h, r0);
                 tma_load_3d(stg + SS_K + 8192, &maps.k, full, 64, h, r0);
                 bulk_load(stg + SS_W, img + kImgW, 16384, full);
-                bulk_load(stg + SS_P, img + kImgP, 8192, full);
                 bulk_load(stg + SS_U, img + kImgU + (size_t)slice * UBYTES, UBYTES, full);
-                bulk_load(stg + SS_G, img + kImgU + 64 * Dv * 2, 256, full);
+                bulk_load(stg + SS_G, img + kImgU + 64 * Dv * 2, 512, full);
             }
         }
-    } else if (warp < 4) {
-        // ------------------------------------------------------------ scan warps
-        const int w = warp;
-        const int tid = threadIdx.x;
-        // S fragments: rows d = 32w + 16mt + g (+8), columns 8nt + 2tg (+1)
-        float S[2][NT][4];
-        const size_t sb = ((size_t)n * H + h) * kDK * Dv + j0;
+        return;
+    }
+
+    // ---------------------------------------------------------------- scan warps
+    const int w = warp;
+    const int tid = threadIdx.x;
+    // S fragments: rows d = 32w + 16mt + g (+8), columns 8nt + 2tg (+1)
+    float S[2][NT][4];
+    const size_t sb = ((size_t)n * H + h) * kDK * Dv + j0;
+#pragma unroll
+    for (int mt = 0; mt < 2; ++mt)
+#pragma unroll
+        for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+            for (int hh = 0; hh < 2; ++hh) {
+                const int d = 32 * w + 16 * mt + g + 8 * hh, j = 8 * nt + 2 * tg;
+                float2 x = make_float2(0.f, 0.f);
+                if (a.s0) x = *reinterpret_cast<const float2 *>(a.s0 + sb + (size_t)d * Dv + j);
+                S[mt][nt][2 * hh] = x.x;
+                S[mt][nt][2 * hh + 1] = x.y;
+            }
+    const uint32_t ssb = smb + SC_SS, utb = smb + SC_UT;
+    for (int c = 0; c < nchunks; ++c) {
+        const int st = c % kScanStages;
+        const uint32_t stg = smb + st * SS_STAGE;
+        const float *eg_s = reinterpret_cast<const float *>(sm + st * SS_STAGE + SS_G);
+        const float *ed_s = eg_s + 64;
+        uint8_t *simg = a.workspace_chunks + ((size_t)(gc0 + c) * H + h) * a.chunk_bytes + kImgS;
+        // ---- S -> bf16: row-major [d][j] in shared memory (this warpgroup's
+        //      B operand) and the MN-major SW128 image the output kernel reads
 #pragma unroll
         for (int mt = 0; mt < 2; ++mt)
 #pragma unroll
@@ -681,186 +722,267 @@ scan_kernel(const __grid_constant__ ScanMaps maps, const PrefillArgs a) {
 #pragma unroll
                 for (int hh = 0; hh < 2; ++hh) {
                     const int d = 32 * w + 16 * mt + g + 8 * hh, j = 8 * nt + 2 * tg;
-                    float2 x = make_float2(0.f, 0.f);
-                    if (a.s0) x = *reinterpret_cast<const float2 *>(a.s0 + sb + (size_t)d * Dv + j);
-                    S[mt][nt][2 * hh] = x.x;
-                    S[mt][nt][2 * hh + 1] = x.y;
+                    const uint32_t v = pack_bf16(S[mt][nt][2 * hh], S[mt][nt][2 * hh + 1]);
+                    *reinterpret_cast<uint32_t *>(sm + SC_SS + d * RS + j * 2) = v;
+                    const int jg = j0 + j;
+                    *reinterpret_cast<uint32_t *>(simg + (jg >> 6) * 16384 + swz(d, (jg & 63) >> 3, 128) +
+                                                  (jg & 7) * 2) = v;
                 }
-        for (int c = 0; c < nchunks; ++c) {
-            const int st = c % kScanStages, buf = c & 1;
-            const uint32_t stg = smb + st * SS_STAGE;
-            const float *g_s = reinterpret_cast<const float *>(sm + st * SS_STAGE + SS_G);
-            if (tid == 0) {
-                bool ok = wait_bar(&bars[SB_FULL + st], (c / kScanStages) & 1, abort_flag, a.err);
-                if (ok && c >= 2) ok = wait_bar(&bars[SB_ODONE + buf], ((c >> 1) - 1) & 1, abort_flag, a.err);
-                if (!ok) *abort_flag = 1;
+        if (tid == 0 && !wait_bar(&bars[SB_FULL + st], (c / kScanStages) & 1, abort_flag, a.err)) *abort_flag = 1;
+        named_bar_sync(1, 128);
+        if (*abort_flag) break;
+        // ---- U = U' + (-W) S for rows t = 16w .. 16w+15: accumulators start at U'
+        const int ta = 16 * w + g, tb = ta + 8;
+        const uint8_t *up = sm + st * SS_STAGE + SS_U;
+        float acc[2][NT][4];
+#pragma unroll
+        for (int nt = 0; nt < NT; ++nt) {
+            const int j = 8 * nt + 2 * tg;
+            const float2 fa = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(up + (ta * NV + j) * 2));
+            const float2 fb = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(up + (tb * NV + j) * 2));
+            acc[0][nt][0] = fa.x; acc[0][nt][1] = fa.y; acc[0][nt][2] = fb.x; acc[0][nt][3] = fb.y;
+            acc[1][nt][0] = acc[1][nt][1] = acc[1][nt][2] = acc[1][nt][3] = 0.f;
+        }
+#pragma unroll
+        for (int ks = 0; ks < 8; ++ks) {
+            uint32_t af[4];
+            ldsm_x4(a_addr_sw128(stg + SS_W, 16 * w, 16 * ks, lane, 8192), af);
+#pragma unroll
+            for (int n2 = 0; n2 < NV / 16; ++n2) {
+                uint32_t bf[4];
+                ldsm_x4_t(b_addr_rm(ssb, 16 * ks, 16 * n2, lane, RS), bf);
+                mma16816(acc[ks & 1][2 * n2], af, bf[0], bf[1]);
+                mma16816(acc[ks & 1][2 * n2 + 1], af, bf[2], bf[3]);
             }
-            named_bar_sync(1, 128);
-            if (*abort_flag) break;
-            // ---- S -> bf16 row-major [d][j]
-            const uint32_t ssb = smb + SC_SS + buf * (128 * 80);
+        }
+        // ---- U~ = e^{g_C - g_t} U -> bf16 row-major [t][j]
+        const float da = ed_s[ta], db = ed_s[tb];
+#pragma unroll
+        for (int nt = 0; nt < NT; ++nt) {
+            const int j = 8 * nt + 2 * tg;
+            *reinterpret_cast<uint32_t *>(sm + SC_UT + ta * RS + j * 2) =
+                pack_bf16((acc[0][nt][0] + acc[1][nt][0]) * da, (acc[0][nt][1] + acc[1][nt][1]) * da);
+            *reinterpret_cast<uint32_t *>(sm + SC_UT + tb * RS + j * 2) =
+                pack_bf16((acc[0][nt][2] + acc[1][nt][2]) * db, (acc[0][nt][3] + acc[1][nt][3]) * db);
+        }
+        named_bar_sync(1, 128);
+        // ---- S <- e^{g_C} S + K^T U~ for rows d = 32w .. 32w+31
+        float ds[2][2][NT][4];
+#pragma unroll
+        for (int p2 = 0; p2 < 2; ++p2)
 #pragma unroll
             for (int mt = 0; mt < 2; ++mt)
 #pragma unroll
                 for (int nt = 0; nt < NT; ++nt)
+                    ds[p2][mt][nt][0] = ds[p2][mt][nt][1] = ds[p2][mt][nt][2] = ds[p2][mt][nt][3] = 0.f;
 #pragma unroll
-                    for (int hh = 0; hh < 2; ++hh) {
-                        const int d = 32 * w + 16 * mt + g + 8 * hh, j = 8 * nt + 2 * tg;
-                        *reinterpret_cast<uint32_t *>(sm + SC_SS + buf * (128 * 80) + d * RS + j * 2) =
-                            pack_bf16(S[mt][nt][2 * hh], S[mt][nt][2 * hh + 1]);
-                    }
-            named_bar_sync(1, 128);
-            if (tid == 0) mbar_arrive(&bars[SB_SREADY + buf]);
-            // ---- U = U' - W S for rows t = 16w .. 16w+15
-            float acc[NT][4];
+        for (int ks = 0; ks < 4; ++ks) {
+            uint32_t bf[NV / 16][4];
 #pragma unroll
-            for (int nt = 0; nt < NT; ++nt) acc[nt][0] = acc[nt][1] = acc[nt][2] = acc[nt][3] = 0.f;
+            for (int n2 = 0; n2 < NV / 16; ++n2) ldsm_x4_t(b_addr_rm(utb, 16 * ks, 16 * n2, lane, RS), bf[n2]);
 #pragma unroll
-            for (int ks = 0; ks < 8; ++ks) {
+            for (int mt = 0; mt < 2; ++mt) {
                 uint32_t af[4];
-                ldsm_x4(a_addr_sw128(stg + SS_W, 16 * w, 16 * ks, lane, 8192), af);
+                ldsm_x4_t(at_addr_sw128(stg + SS_K, 32 * w + 16 * mt, 16 * ks, lane, 8192), af);
 #pragma unroll
                 for (int n2 = 0; n2 < NV / 16; ++n2) {
-                    uint32_t bf[4];
-                    ldsm_x4_t(b_addr_rm(ssb, 16 * ks, 16 * n2, lane, RS), bf);
-                    mma16816(acc[2 * n2], af, bf[0], bf[1]);
-                    mma16816(acc[2 * n2 + 1], af, bf[2], bf[3]);
+                    mma16816(ds[ks & 1][mt][2 * n2], af, bf[n2][0], bf[n2][1]);
+                    mma16816(ds[ks & 1][mt][2 * n2 + 1], af, bf[n2][2], bf[n2][3]);
                 }
             }
-            const float gC = g_s[63];
-            const int ta = 16 * w + g, tb = ta + 8;
-            const float da = __expf(gC - g_s[ta]), db = __expf(gC - g_s[tb]);
-            const uint8_t *up = sm + st * SS_STAGE + SS_U;
-#pragma unroll
-            for (int nt = 0; nt < NT; ++nt) {
-                const int j = 8 * nt + 2 * tg;
-                const __nv_bfloat162 ua = *reinterpret_cast<const __nv_bfloat162 *>(up + (ta * NV + j) * 2);
-                const __nv_bfloat162 ub = *reinterpret_cast<const __nv_bfloat162 *>(up + (tb * NV + j) * 2);
-                const float2 fa = __bfloat1622float2(ua), fb = __bfloat1622float2(ub);
-                const float u0 = fa.x - acc[nt][0], u1 = fa.y - acc[nt][1];
-                const float u2 = fb.x - acc[nt][2], u3 = fb.y - acc[nt][3];
-                uint8_t *usb = sm + SC_US + buf * (64 * 80);
-                *reinterpret_cast<uint32_t *>(usb + ta * RS + j * 2) = pack_bf16(u0, u1);
-                *reinterpret_cast<uint32_t *>(usb + tb * RS + j * 2) = pack_bf16(u2, u3);
-                *reinterpret_cast<uint32_t *>(sm + SC_UT + ta * RS + j * 2) = pack_bf16(u0 * da, u1 * da);
-                *reinterpret_cast<uint32_t *>(sm + SC_UT + tb * RS + j * 2) = pack_bf16(u2 * db, u3 * db);
-            }
-            named_bar_sync(1, 128);
-            if (tid == 0) mbar_arrive(&bars[SB_UREADY + buf]);
-            // ---- S <- e^{g_C} S + K^T U~ for rows d = 32w .. 32w+31
-            float ds[2][NT][4];
-#pragma unroll
-            for (int mt = 0; mt < 2; ++mt)
-#pragma unroll
-                for (int nt = 0; nt < NT; ++nt) ds[mt][nt][0] = ds[mt][nt][1] = ds[mt][nt][2] = ds[mt][nt][3] = 0.f;
-#pragma unroll
-            for (int ks = 0; ks < 4; ++ks) {
-                uint32_t bf[NV / 16][4];
-#pragma unroll
-                for (int n2 = 0; n2 < NV / 16; ++n2)
-                    ldsm_x4_t(b_addr_rm(smb + SC_UT, 16 * ks, 16 * n2, lane, RS), bf[n2]);
-#pragma unroll
-                for (int mt = 0; mt < 2; ++mt) {
-                    uint32_t af[4];
-                    ldsm_x4_t(at_addr_sw128(stg + SS_K, 32 * w + 16 * mt, 16 * ks, lane, 8192), af);
-#pragma unroll
-                    for (int n2 = 0; n2 < NV / 16; ++n2) {
-                        mma16816(ds[mt][2 * n2], af, bf[n2][0], bf[n2][1]);
-                        mma16816(ds[mt][2 * n2 + 1], af, bf[n2][2], bf[n2][3]);
-                    }
-                }
-            }
-            const float eC = __expf(gC);
-#pragma unroll
-            for (int mt = 0; mt < 2; ++mt)
-#pragma unroll
-                for (int nt = 0; nt < NT; ++nt)
-#pragma unroll
-                    for (int i = 0; i < 4; ++i) S[mt][nt][i] = fmaf(eC, S[mt][nt][i], ds[mt][nt][i]);
-            mbar_arrive(&bars[SB_EMPTY + st]);
         }
-        if (a.sf && !*abort_flag) {
+        const float eC = eg_s[63];                    // e^{g_C}
 #pragma unroll
-            for (int mt = 0; mt < 2; ++mt)
-#pragma unroll
-                for (int nt = 0; nt < NT; ++nt)
-#pragma unroll
-                    for (int hh = 0; hh < 2; ++hh) {
-                        const int d = 32 * w + 16 * mt + g + 8 * hh, j = 8 * nt + 2 * tg;
-                        *reinterpret_cast<float2 *>(a.sf + sb + (size_t)d * Dv + j) =
-                            make_float2(S[mt][nt][2 * hh], S[mt][nt][2 * hh + 1]);
-                    }
-        }
-    } else {
-        // ------------------------------------------------------------ output warps
-        const int w = warp - 4;
-        const int tid = threadIdx.x - 128;
-        __nv_bfloat16 *out = static_cast<__nv_bfloat16 *>(a.out);
-        for (int c = 0; c < nchunks; ++c) {
-            const int st = c % kScanStages, buf = c & 1;
-            const uint32_t stg = smb + st * SS_STAGE;
-            const float *g_s = reinterpret_cast<const float *>(sm + st * SS_STAGE + SS_G);
-            const int lenc = (int)min((long)kC, len - (long)c * kC);
-            if (tid == 0) {
-                bool ok = wait_bar(&bars[SB_FULL + st], (c / kScanStages) & 1, abort_flag, a.err);
-                if (ok) ok = wait_bar(&bars[SB_SREADY + buf], (c >> 1) & 1, abort_flag, a.err);
-                if (!ok) *abort_flag = 1;
-            }
-            named_bar_sync(2, 128);
-            if (*abort_flag) break;
-            // O1 = Q S for rows t = 16w .. 16w+15
-            const uint32_t ssb = smb + SC_SS + buf * (128 * 80);
-            float o1[NT][4], o2[NT][4];
+        for (int mt = 0; mt < 2; ++mt)
 #pragma unroll
             for (int nt = 0; nt < NT; ++nt)
 #pragma unroll
-                for (int i = 0; i < 4; ++i) o1[nt][i] = o2[nt][i] = 0.f;
+                for (int i = 0; i < 4; ++i)
+                    S[mt][nt][i] = fmaf(eC, S[mt][nt][i], ds[0][mt][nt][i] + ds[1][mt][nt][i]);
+        mbar_arrive(&bars[SB_EMPTY + st]);
+        // the next chunk rewrites the S and U~ buffers: every warp must be past
+        // its reads of them
+        named_bar_sync(1, 128);
+    }
+    if (a.sf && !*abort_flag) {
 #pragma unroll
-            for (int ks = 0; ks < 8; ++ks) {
-                uint32_t af[4];
-                ldsm_x4(a_addr_sw128(stg + SS_Q, 16 * w, 16 * ks, lane, 8192), af);
+        for (int mt = 0; mt < 2; ++mt)
 #pragma unroll
-                for (int n2 = 0; n2 < NV / 16; ++n2) {
-                    uint32_t bf[4];
-                    ldsm_x4_t(b_addr_rm(ssb, 16 * ks, 16 * n2, lane, RS), bf);
-                    mma16816(o1[2 * n2], af, bf[0], bf[1]);
-                    mma16816(o1[2 * n2 + 1], af, bf[2], bf[3]);
+            for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+                for (int hh = 0; hh < 2; ++hh) {
+                    const int d = 32 * w + 16 * mt + g + 8 * hh, j = 8 * nt + 2 * tg;
+                    *reinterpret_cast<float2 *>(a.sf + sb + (size_t)d * Dv + j) =
+                        make_float2(S[mt][nt][2 * hh], S[mt][nt][2 * hh + 1]);
                 }
-            }
-            if (tid == 0 && !wait_bar(&bars[SB_UREADY + buf], (c >> 1) & 1, abort_flag, a.err)) *abort_flag = 1;
-            named_bar_sync(2, 128);
-            if (*abort_flag) break;
-            // O2 = P U
-            const uint32_t usb = smb + SC_US + buf * (64 * 80);
-#pragma unroll
-            for (int ks = 0; ks < 4; ++ks) {
-                uint32_t af[4];
-                ldsm_x4(a_addr_sw128(stg + SS_P, 16 * w, 16 * ks, lane, 8192), af);
-#pragma unroll
-                for (int n2 = 0; n2 < NV / 16; ++n2) {
-                    uint32_t bf[4];
-                    ldsm_x4_t(b_addr_rm(usb, 16 * ks, 16 * n2, lane, RS), bf);
-                    mma16816(o2[2 * n2], af, bf[0], bf[1]);
-                    mma16816(o2[2 * n2 + 1], af, bf[2], bf[3]);
-                }
-            }
-            const int ta = 16 * w + g, tb = ta + 8;
-            const float ea = __expf(g_s[ta]) * a.scale, eb = __expf(g_s[tb]) * a.scale;
-            const float sc = a.scale;
-            const long rowa = t0 + (long)c * kC + ta, rowb = rowa + 8;
-#pragma unroll
-            for (int nt = 0; nt < NT; ++nt) {
-                const int j = j0 + 8 * nt + 2 * tg;
-                if (ta < lenc)
-                    *reinterpret_cast<uint32_t *>(out + ((size_t)rowa * H + h) * Dv + j) =
-                        pack_bf16(fmaf(ea, o1[nt][0], sc * o2[nt][0]), fmaf(ea, o1[nt][1], sc * o2[nt][1]));
-                if (tb < lenc)
-                    *reinterpret_cast<uint32_t *>(out + ((size_t)rowb * H + h) * Dv + j) =
-                        pack_bf16(fmaf(eb, o1[nt][2], sc * o2[nt][2]), fmaf(eb, o1[nt][3], sc * o2[nt][3]));
-            }
-            mbar_arrive(&bars[SB_ODONE + buf]);
-            mbar_arrive(&bars[SB_EMPTY + st]);
+    }
+}
+
+// ---------------------------------------------------------------------------
+// Kernel 3: outputs.  One CTA per (global chunk, head), all value columns.
+//
+//   D[0:64]    = (-W) S_c          -> U = U' + D[0:64]
+//   D[64:128]  = diag(e^g) Q S_c
+//   D         += [0; P] U          -> D[64:128] = O / scale
+// Both products have M = 128 and N = Dv, the shapes tcgen05 runs well.
+// ---------------------------------------------------------------------------
+constexpr int kOutThreads = 192;      // warp 0 loads, warp 1 MMA, warps 2..5 compute
+constexpr uint32_t kOutTmemCols = 128;
+constexpr uint32_t OS_A = 0;          // [-W ; diag(e^g) Q]: half h at h*16384 (rows 0..63 -W, 64..127 Q~)
+constexpr uint32_t OS_ZP = 32768;     // [0 ; P]: rows 0..63 zero, rows 64..127 P (16 KiB)
+constexpr uint32_t OS_S = 49152;      // S_c image (Dv/64 atoms of 16 KiB)
+constexpr uint32_t OS_U = OS_S;       // U image, bf16 MN-major SW128: atoms [64 rows x 128 B] of 8 KiB,
+                                      // written once the first product has consumed S_c
+constexpr uint32_t OS_UP = 81920;     // U' (64 x Dv bf16, value slices), then the decay factors
+constexpr uint32_t OS_BAR = OS_UP + 16384 + 512;
+constexpr uint32_t OS_TMEMPTR = OS_BAR + 4 * 8;
+constexpr uint32_t OS_FLAGS = OS_TMEMPTR + 4;
+constexpr uint32_t kOutSmem = OS_FLAGS + 4 + 1024;
+enum OutBar { OB_FULL = 0, OB_D1, OB_UREADY, OB_D2 };
+
+template <int NV>
+__global__ void __launch_bounds__(kOutThreads, 2)
+out_kernel(const PrefillArgs a) {
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t *sm = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    ChunkLoc loc;
+    const long gc = blockIdx.x;
+    if (!locate_chunk(a, gc, loc)) return;
+    const int h = blockIdx.y;
+    const int H = a.H, Dv = a.Dv;
+    const int lenc = (int)min((long)kC, loc.len - (long)loc.c * kC);
+    const long row0 = loc.t0 + (long)loc.c * kC;
+    uint64_t *bars = reinterpret_cast<uint64_t *>(sm + OS_BAR);
+    uint32_t *tmem_ptr = reinterpret_cast<uint32_t *>(sm + OS_TMEMPTR);
+    volatile int *abort_flag = reinterpret_cast<volatile int *>(sm + OS_FLAGS);
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const uint8_t *img = a.workspace_chunks + ((size_t)gc * H + h) * a.chunk_bytes;
+
+    if (threadIdx.x == 0) {
+        for (int i = 0; i < 4; ++i) mbar_init(&bars[i], 1);
+        *abort_flag = 0;
+        fence_mbar_init();
+    }
+    if (warp == 1) {
+        tmem_alloc(tmem_ptr, kOutTmemCols);
+        tmem_relinquish();
+    }
+    if (warp >= 2) {
+        // zero rows 0..63 of [0 ; P]
+        for (int i = threadIdx.x - 64; i < 8192 / 16; i += 128)
+            reinterpret_cast<uint4 *>(sm + OS_ZP)[i] = make_uint4(0u, 0u, 0u, 0u);
+        fence_proxy_async_smem();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = *tmem_ptr;
+
+    if (warp == 0) {
+        if (lane == 0) {
+            uint64_t *full = &bars[OB_FULL];
+            const uint32_t sbytes = (uint32_t)(Dv / 64) * 16384;
+            mbar_arrive_expect_tx(full, 32768 + 8192 + sbytes + 64 * Dv * 2 + 512);
+            bulk_load(sm + OS_A, img + kImgW, 8192, full);
+            bulk_load(sm + OS_A + 8192, img + kImgQ, 8192, full);
+            bulk_load(sm + OS_A + 16384, img + kImgW + 8192, 8192, full);
+            bulk_load(sm + OS_A + 24576, img + kImgQ + 8192, 8192, full);
+            bulk_load(sm + OS_ZP + 8192, img + kImgP, 8192, full);
+            bulk_load(sm + OS_S, img + kImgS, sbytes, full);
+            bulk_load(sm + OS_UP, img + kImgU, 64 * Dv * 2 + 512, full);
         }
+    } else if (warp == 1) {
+        if (lane == 0) {
+            const uint32_t aa = smem_u32(sm + OS_A), zp = smem_u32(sm + OS_ZP);
+            const uint32_t ss = smem_u32(sm + OS_S), uu = smem_u32(sm + OS_U);
+            const uint32_t id = Dv == 128 ? idesc_bf16(128, 128, 0, 1) : idesc_bf16(128, 64, 0, 1);
+            bool ok = wait_bar(&bars[OB_FULL], 0, abort_flag, a.err);
+            if (ok) {
+                tc_fence_after();
+#pragma unroll
+                for (int kk = 0; kk < 8; ++kk)
+                    mma_bf16(tmem, smem_desc(aa + (kk >> 2) * 16384 + (kk & 3) * 32, 16, 1024, kSw128),
+                             smem_desc(ss + kk * 2048, 16384, 1024, kSw128), id, kk > 0);
+                mma_commit(&bars[OB_D1]);
+                ok = wait_bar(&bars[OB_UREADY], 0, abort_flag, a.err);
+            }
+            if (ok) {
+                tc_fence_after();
+#pragma unroll
+                for (int kk = 0; kk < 4; ++kk)
+                    mma_bf16(tmem, smem_desc(zp + kk * 32, 16, 1024, kSw128),
+                             smem_desc(uu + kk * 2048, 8192, 1024, kSw128), id, 1);
+                mma_commit(&bars[OB_D2]);
+            }
+        }
+    } else {
+        const int cw = threadIdx.x - 64;
+        const int q4 = warp & 3;
+        const int r = 32 * q4 + lane;            // accumulator row = TMEM lane
+        const uint32_t tq = tmem + ((uint32_t)(32 * q4) << 16);
+        if (cw == 0 && !wait_bar(&bars[OB_D1], 0, abort_flag, a.err)) *abort_flag = 1;
+        named_bar_sync(1, 128);
+        if (!*abort_flag) {
+            tc_fence_after();
+            if (r < 64) {
+                // U row t = U' + (-W S)  -> MN-major SW128 image
+                const int t = r;
+                for (int j16 = 0; j16 < Dv; j16 += 16) {
+                    float x[16];
+                    tmem_ld16(tq + j16, x);
+                    tmem_wait_ld();
+                    const uint8_t *src = sm + OS_UP + (j16 / NV) * (64 * NV * 2) + (t * NV + j16 % NV) * 2;
+                    const uint4 u0 = *reinterpret_cast<const uint4 *>(src);
+                    const uint4 u1 = *reinterpret_cast<const uint4 *>(src + 16);
+                    const uint32_t uw[8] = {u0.x, u0.y, u0.z, u0.w, u1.x, u1.y, u1.z, u1.w};
+#pragma unroll
+                    for (int e = 0; e < 8; ++e) {
+                        const float2 f = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(&uw[e]));
+                        x[2 * e] += f.x;
+                        x[2 * e + 1] += f.y;
+                    }
+#pragma unroll
+                    for (int h8 = 0; h8 < 2; ++h8) {
+                        const int j = j16 + 8 * h8;
+                        *reinterpret_cast<uint4 *>(sm + OS_U + (j >> 6) * 8192 + swz(t, (j & 63) >> 3, 128)) =
+                            pack8(x + 8 * h8);
+                    }
+                }
+            }
+            fence_proxy_async_smem();
+            tc_fence_before();
+        }
+        named_bar_sync(1, 128);
+        if (cw == 0 && !*abort_flag) {
+            mbar_arrive(&bars[OB_UREADY]);
+            if (!wait_bar(&bars[OB_D2], 0, abort_flag, a.err)) *abort_flag = 1;
+        }
+        named_bar_sync(1, 128);
+        if (!*abort_flag) {
+            tc_fence_after();
+            if (r >= 64) {
+                const int t = r - 64;
+                __nv_bfloat16 *orow = static_cast<__nv_bfloat16 *>(a.out) + ((size_t)(row0 + t) * H + h) * Dv;
+                for (int j16 = 0; j16 < Dv; j16 += 16) {
+                    float x[16];
+                    tmem_ld16(tq + j16, x);
+                    tmem_wait_ld();
+                    if (t < lenc) {
+#pragma unroll
+                        for (int e = 0; e < 16; ++e) x[e] *= a.scale;
+                        *reinterpret_cast<uint4 *>(orow + j16) = pack8(x);
+                        *reinterpret_cast<uint4 *>(orow + j16 + 8) = pack8(x + 8);
+                    }
+                }
+            }
+        }
+    }
+
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 1) {
+        tc_fence_after();
+        tmem_dealloc(tmem, kOutTmemCols);
     }
 }
 
@@ -950,6 +1072,7 @@ cudaError_t launch_nv(const PrefillArgs &a, long chunks_grid, cudaStream_t s) {
     std::call_once(once, [] {
         attr = set_smem(prep_kernel<NV>, kPrepSmem);
         if (attr == cudaSuccess) attr = set_smem(scan_kernel<NV>, kScanSmem);
+        if (attr == cudaSuccess) attr = set_smem(out_kernel<NV>, kOutSmem);
     });
     if (attr != cudaSuccess) return attr;
     PrepMaps pm;
@@ -960,7 +1083,6 @@ cudaError_t launch_nv(const PrefillArgs &a, long chunks_grid, cudaStream_t s) {
         if (!make_map(&pm.q, a.q, kDK, a.H, a.total_T, 64) || !make_map(&pm.k, a.k, kDK, a.H, a.total_T, 64) ||
             !make_map(&pm.v, a.v, a.Dv, a.H, a.total_T, 64))
             return cudaErrorInvalidValue;
-        sm.q = pm.q;
         sm.k = pm.k;
     }
     if (chunks_grid > 0) {
@@ -969,10 +1091,13 @@ cudaError_t launch_nv(const PrefillArgs &a, long chunks_grid, cudaStream_t s) {
         if (e != cudaSuccess) return e;
     }
     scan_kernel<NV><<<dim3(a.Dv / NV, a.H, a.num_seqs), kScanThreads, kScanSmem, s>>>(sm, a);
+    cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess || chunks_grid == 0) return e;
+    out_kernel<NV><<<dim3((unsigned)chunks_grid, a.H, 1), kOutThreads, kOutSmem, s>>>(a);
     return cudaGetLastError();
 }
 
-size_t image_bytes(int Dv) { return (size_t)kImgU + 64 * (size_t)Dv * 2 + 256; }
+size_t image_bytes(int Dv) { return (size_t)kImgU + 64 * (size_t)Dv * 2 + 512; }
 
 size_t header_bytes(int num_seqs) {
     size_t b = 4 * (size_t)(num_seqs + 1);

@@ -69,6 +69,8 @@ __device__ __forceinline__ void bulk_store(void *dst, const void *src, uint32_t 
 }
 __device__ __forceinline__ void bulk_commit() { asm volatile("cp.async.bulk.commit_group;" ::: "memory"); }
 __device__ __forceinline__ void bulk_wait_all() { asm volatile("cp.async.bulk.wait_group 0;" ::: "memory"); }
+// waits until every committed bulk store has finished reading shared memory
+__device__ __forceinline__ void bulk_wait_reads() { asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory"); }
 
 // ------------------------------------------------------------------ fences / barriers
 __device__ __forceinline__ void fence_proxy_async_smem() {
