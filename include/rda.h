@@ -89,21 +89,28 @@ const char *rda_version(void);
 
 /*
  * Bytes of device workspace that rda_prefill_chunked (num_seqs = 0) or
- * rda_prefill_varlen (num_seqs = N) needs for these sizes.  Always >= 256
- * (the first 256 bytes hold the device error word).  The workspace must be
- * 256-byte aligned.  Returns 0 for unsupported sizes.
+ * rda_prefill_varlen (num_seqs = N, pass B = 1 and T = total_T) needs for
+ * these sizes, enough for either dtype.  Always >= 256: the first 256 bytes
+ * hold the device error word.  When the chunked tensor-core path can run
+ * (Dk = 128) it also holds that path's per-chunk scratch, about 88.5 KiB per
+ * 64-token chunk and head at Dv = 128 (e.g. 90.6 MB for B=1, T=4096, H=16).
+ * The workspace must be 256-byte aligned; its contents need no
+ * initialisation beyond a cleared error word, and are overwritten by each
+ * call.  Returns 0 for unsupported sizes.
  */
 size_t rda_prefill_workspace_bytes(int B, int T, int H, int Dk, int Dv, int num_seqs);
 
 /*
  * Fixed-length prefill over B sequences of T tokens each.
  *
- * Defined by the gated delta rule above; the chunked form it uses (64-token
- * chunks, a UT transform of each chunk, tensor-core products, a sequential
- * scan of fp32 states across chunks) reaches the same result up to rounding.
- * bf16 inputs take the chunked tensor-core path when Dk = 128; fp32 inputs,
- * and bf16 with Dk = 64, take a token-sequential fp32 path (fp32 inputs are
- * held to fp32 accuracy, which bf16 tensor-core operands cannot give).
+ * Defined by the gated delta rule above; the chunked form it uses reaches the
+ * same result up to rounding: 64-token chunks, a UT transform of each chunk
+ * and its products on the tensor cores (chunk-parallel), a sequential scan of
+ * the fp32 state across chunks, then the outputs (chunk-parallel).  bf16
+ * inputs take this path when Dk = 128; fp32 inputs, and bf16 with Dk = 64,
+ * take a token-sequential fp32 path (fp32 inputs are held to fp32 accuracy,
+ * which bf16 tensor-core operands cannot give).  Several kernels are
+ * enqueued on `stream`, in order.
  *
  *   q, k, v        device, dtype, layouts above, 16-byte aligned
  *   log_alpha      device fp32 [B,T,H]; beta device fp32 [B,T,H]
