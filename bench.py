@@ -117,6 +117,23 @@ class ClockSampler:
                 "samples": len(inside)}
 
 
+def captured_traffic():
+    """DRAM bytes per step from a committed ncu capture, only while the kernel
+    source it was taken on is unchanged (sha256 match); else None."""
+    import hashlib
+    try:
+        with open(os.path.join(ROOT, "profiles", "traffic.json")) as f:
+            rec = json.load(f)
+        src = os.path.join(ROOT, rec["source"])
+        with open(src, "rb") as f:
+            digest = hashlib.sha256(f.read()).hexdigest()
+        if digest != rec["source_sha256"]:
+            return None
+        return float(rec["dram_bytes_per_step"])
+    except Exception:
+        return None
+
+
 def gpu_id_for(device):
     import torch
     try:
@@ -282,7 +299,7 @@ def run_ours(args, rank, world, device):
                    "l2": "flushed between timed steps (256 MiB write)",
                    "parallelism": f"replicas x{world}"},
         "roofline": {"bound": "hbm", "achieved": gbs, "peak": hbm, "unit": "GB/s",
-                     "frac": gbs / hbm, "traffic": None, "peak_source": src,
+                     "frac": gbs / hbm, "traffic": captured_traffic(), "peak_source": src,
                      "algorithmic_bytes_per_launch": alg_bytes,
                      "tensor": {"achieved_tflops": tflops, "peak_tflops": tf,
                                 "frac": tflops / tf, "algorithmic_flops_per_launch": alg_flops}},

@@ -61,7 +61,9 @@ constexpr uint32_t kImgQ = 16384;      // diag(e^g) Q, same layout
 constexpr uint32_t kImgP = 32768;      // P, bf16 K-major SW128, 8 KiB
 constexpr uint32_t kImgS = 40960;      // state entering the chunk, bf16 MN-major SW128:
                                        // atoms of 64 value columns, [128 key rows x 128 B] each
-constexpr uint32_t kImgU = 73728;      // U', bf16, value slices of width NV, each [64][NV];
+constexpr uint32_t kImgV = 73728;      // U = U' - W S_c, bf16 MN-major SW128: atoms of 64 value
+                                       // columns, [64 token rows x 128 B] each (written by the scan)
+constexpr uint32_t kImgU = 90112;      // U', bf16, value slices of width NV, each [64][NV];
                                        // then e^{g_t} and e^{g_C - g_t}: 2 x 64 fp32
 
 __device__ __forceinline__ uint64_t globaltimer() {
@@ -245,35 +247,38 @@ struct PrepMaps {
     CUtensorMap q, k, v;
 };
 
-// Where chunk `gc` (global over all sequences) lives.
+// Which chunk a prep / output CTA handles: `idx` enumerates every chunk of
+// every sequence in order.
 struct ChunkLoc {
     long t0;       // first token of the sequence
     long len;      // sequence length
     int c;         // chunk index within the sequence
+    long gc;       // global chunk index: where its images live in the workspace
 };
 
-__device__ __forceinline__ bool locate_chunk(const PrefillArgs &a, long gc, ChunkLoc &loc) {
+__device__ __forceinline__ bool locate_chunk(const PrefillArgs &a, long idx, ChunkLoc &loc) {
+    loc.gc = idx;
     if (!a.cu_seqlens) {
         const long cps = (a.T + kC - 1) / kC;
         if (cps == 0) return false;
-        const long n = gc / cps;
+        const long n = idx / cps;
         if (n >= a.num_seqs) return false;
         loc.t0 = n * (long)a.T;
         loc.len = a.T;
-        loc.c = (int)(gc - n * cps);
+        loc.c = (int)(idx - n * cps);
         return true;
     }
     const int32_t *cb = a.chunk_base;
-    if (gc >= cb[a.num_seqs]) return false;
-    int lo = 0, hi = a.num_seqs - 1;      // last n with cb[n] <= gc
+    if (idx >= cb[a.num_seqs]) return false;
+    int lo = 0, hi = a.num_seqs - 1;      // last n with cb[n] <= idx
     while (lo < hi) {
         const int mid = (lo + hi + 1) >> 1;
-        if (cb[mid] <= gc) lo = mid;
+        if (cb[mid] <= idx) lo = mid;
         else hi = mid - 1;
     }
     loc.t0 = a.cu_seqlens[lo];
     loc.len = (long)a.cu_seqlens[lo + 1] - loc.t0;
-    loc.c = (int)(gc - cb[lo]);
+    loc.c = (int)(idx - cb[lo]);
     return true;
 }
 
@@ -283,8 +288,8 @@ prep_kernel(const __grid_constant__ PrepMaps maps, const PrefillArgs a) {
     extern __shared__ uint8_t smem_raw[];
     uint8_t *sm = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     ChunkLoc loc;
-    const long gc = blockIdx.x;
-    if (!locate_chunk(a, gc, loc)) return;     // uniform across the CTA
+    if (!locate_chunk(a, blockIdx.x, loc)) return;     // uniform across the CTA
+    const long gc = loc.gc;
     const int h = blockIdx.y;
     const int H = a.H, Dv = a.Dv;
     const int lenc = (int)min((long)kC, loc.len - (long)loc.c * kC);
@@ -558,25 +563,32 @@ prep_kernel(const __grid_constant__ PrepMaps maps, const PrefillArgs a) {
 // 64xNV).  On tcgen05 each such instruction costs about 90 cycles of pipe
 // time whatever its size, plus a commit round trip, so this latency-bound
 // chain runs on register-fragment tensor-core MMAs (mma.sync m16n8k16, bf16
-// in, fp32 accumulate) with ldmatrix operands.  Everything that does not
-// feed the next state (the outputs) is left to the output kernel, which
-// reads the state entering each chunk from the workspace.
-//   warps 0..3  carry the fp32 state as accumulator fragments (warp w owns
-//               key rows 32w..32w+31) and compute U~ and the update;
+// in, fp32 accumulate) with ldmatrix operands.  The outputs are left to the
+// output kernel, which reads the state entering each chunk and U from the
+// workspace.
+//   warps 0..3  warp w owns key rows 32w..32w+31 of the fp32 state (as
+//               accumulator fragments) across the slice's NV value columns;
+//               (splitting the columns over twice the warps doubles the
+//               operand traffic through shared memory and measured slower)
 //   warp 4      producer: the K tile by TMA, -W, U' and the decay factors by
 //               bulk copies, into a 4-stage ring.
 // ---------------------------------------------------------------------------
-constexpr int kScanThreads = 160;
-constexpr int kScanStages = 4;
+constexpr int kScanWarps = 4;
+constexpr int kScanThreads = (kScanWarps + 1) * 32;
+constexpr int kScanStages = 3;
 // per-stage shared memory (bytes): -W 16K | K 16K | U' <= 4K | decay 512
 constexpr uint32_t SS_W = 0, SS_K = 16384, SS_U = 32768, SS_G = 36864;
 constexpr uint32_t SS_STAGE = 37888;                          // multiple of 1024
-constexpr uint32_t SC_SS = kScanStages * SS_STAGE;            // state  [128][RS] bf16
-constexpr uint32_t SC_UT = SC_SS + 128 * 80;                  // U~     [64][RS]
-constexpr uint32_t SC_BAR = SC_UT + 64 * 80;
 enum ScanBar { SB_FULL = 0, SB_EMPTY = kScanStages, kScanBars = 2 * kScanStages };
-constexpr uint32_t SC_FLAGS = SC_BAR + kScanBars * 8;
-constexpr uint32_t kScanSmem = SC_FLAGS + 16 + 1024;
+// then: state [128][RS] bf16, U~ [64][RS], barriers, flags (RS = 2 NV + 16)
+template <int NV> struct ScanSmem {
+    static constexpr uint32_t RS = NV * 2 + 16;
+    static constexpr uint32_t SS = kScanStages * SS_STAGE;
+    static constexpr uint32_t UT = SS + 128 * RS;
+    static constexpr uint32_t BAR = UT + 64 * RS;
+    static constexpr uint32_t FLAGS = BAR + kScanBars * 8;
+    static constexpr uint32_t BYTES = FLAGS + 16 + 1024;
+};
 
 struct ScanMaps {
     CUtensorMap k;
@@ -590,6 +602,11 @@ __device__ __forceinline__ void ldsm_x4(uint32_t addr, uint32_t *r) {
 __device__ __forceinline__ void ldsm_x4_t(uint32_t addr, uint32_t *r) {
     asm volatile("ldmatrix.sync.aligned.m8n8.x4.trans.shared.b16 {%0,%1,%2,%3}, [%4];"
                  : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3])
+                 : "r"(addr));
+}
+__device__ __forceinline__ void ldsm_x2_t(uint32_t addr, uint32_t *r) {
+    asm volatile("ldmatrix.sync.aligned.m8n8.x2.trans.shared.b16 {%0,%1}, [%2];"
+                 : "=r"(r[0]), "=r"(r[1])
                  : "r"(addr));
 }
 // D += A(16x16, row) * B(16x8, col): bf16 inputs, fp32 accumulate.
@@ -616,12 +633,28 @@ __device__ __forceinline__ uint32_t at_addr_sw128(uint32_t base, int m0, int k0,
     const int col = m0 + 8 * (mi & 1);                   // image column = m
     return base + (col >> 6) * halfbytes + swz(row, (col & 63) >> 3, 128);
 }
-// ldmatrix.trans address for the two B fragments (n 0..7 and 8..15 from n0)
-// of a row-major [k][n] bf16 buffer with row stride rs bytes.
+// ldmatrix.trans address for B fragments of a row-major [k][n] bf16 buffer
+// (row stride rs bytes): x4 gives n0..n0+7 and n0+8..n0+15, x2 gives n0..n0+7.
 __device__ __forceinline__ uint32_t b_addr_rm(uint32_t base, int k0, int n0, int lane, uint32_t rs) {
     const int row = k0 + (lane & 7) + ((lane >> 3) & 1) * 8;
     const int col = n0 + 8 * (lane >> 4);
     return base + row * rs + col * 2;
+}
+// B fragments for one warp's NW value columns (8, 16 or 32) at k-tile k0:
+// bf[2nt], bf[2nt+1] feed n-tile nt.
+template <int NW>
+__device__ __forceinline__ void ld_b(uint32_t base, int k0, int n0, int lane, uint32_t rs, uint32_t *bf) {
+    if constexpr (NW == 8) {
+        ldsm_x2_t(b_addr_rm(base, k0, n0, lane & 15, rs), bf);
+    } else {
+#pragma unroll
+        for (int i = 0; i < NW / 16; ++i) ldsm_x4_t(b_addr_rm(base, k0, n0 + 16 * i, lane, rs), bf + 4 * i);
+    }
+}
+// Byte offset of value column j of row `row` in an MN-major SW128 image whose
+// 64-column atoms have `atom_bytes` (rows of 128 B).
+__device__ __forceinline__ uint32_t mn_off(int row, int j, uint32_t atom_bytes) {
+    return (j >> 6) * atom_bytes + swz(row, (j & 63) >> 3, 128) + (j & 7) * 2;
 }
 
 template <int NV>
@@ -629,11 +662,15 @@ __global__ void __launch_bounds__(kScanThreads, 1)
 scan_kernel(const __grid_constant__ ScanMaps maps, const PrefillArgs a) {
     extern __shared__ uint8_t smem_raw[];
     uint8_t *sm = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-    uint64_t *bars = reinterpret_cast<uint64_t *>(sm + SC_BAR);
-    volatile int *abort_flag = reinterpret_cast<volatile int *>(sm + SC_FLAGS);
-    constexpr int NT = NV / 8;                  // n-tiles of 8 columns
+    using L = ScanSmem<NV>;
+    constexpr uint32_t SC_SS = L::SS, SC_UT = L::UT;
+    uint64_t *bars = reinterpret_cast<uint64_t *>(sm + L::BAR);
+    volatile int *abort_flag = reinterpret_cast<volatile int *>(sm + L::FLAGS);
+    constexpr int NW = NV * 4 / kScanWarps;     // value columns per warp
+    constexpr int NT = NW / 8;                  // n-tiles of 8 columns per warp
     constexpr uint32_t RS = NV * 2 + 16;        // padded row stride of the S / U~ buffers
     constexpr uint32_t UBYTES = 64 * NV * 2;    // U' slice bytes
+    constexpr uint32_t NCW = kScanWarps * 32;
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int g = lane >> 2, tg = lane & 3;
@@ -650,13 +687,15 @@ scan_kernel(const __grid_constant__ ScanMaps maps, const PrefillArgs a) {
         gc0 = (long)n * ((a.T + kC - 1) / kC);
     }
     const int nchunks = (int)((len + kC - 1) / kC);
+    const float *s_in = a.s0;
+    float *s_out = a.sf;
     const int j0 = slice * NV;
     const int H = a.H, Dv = a.Dv;
 
     if (threadIdx.x == 0) {
         for (int i = 0; i < kScanStages; ++i) {
             mbar_init(&bars[SB_FULL + i], 1);
-            mbar_init(&bars[SB_EMPTY + i], 128);
+            mbar_init(&bars[SB_EMPTY + i], NCW);
         }
         *abort_flag = 0;
         fence_mbar_init();
@@ -665,7 +704,7 @@ scan_kernel(const __grid_constant__ ScanMaps maps, const PrefillArgs a) {
     __syncthreads();
     const uint32_t smb = smem_u32(sm);
 
-    if (warp == 4) {
+    if (warp == kScanWarps) {
         // ------------------------------------------------------------ producer
         if (lane == 0) {
             for (int c = 0; c < nchunks; ++c) {
@@ -689,9 +728,11 @@ scan_kernel(const __grid_constant__ ScanMaps maps, const PrefillArgs a) {
     }
 
     // ---------------------------------------------------------------- scan warps
-    const int w = warp;
+    const int rg = warp & 3;                    // row group
+    const int c0 = (warp >> 2) * NW;            // first value column (within the slice)
+    static_assert(kScanWarps == 4 || kScanWarps == 8, "warps cover 4 row groups");
     const int tid = threadIdx.x;
-    // S fragments: rows d = 32w + 16mt + g (+8), columns 8nt + 2tg (+1)
+    // S fragments: rows d = 32rg + 16mt + g (+8), columns c0 + 8nt + 2tg (+1)
     float S[2][NT][4];
     const size_t sb = ((size_t)n * H + h) * kDK * Dv + j0;
 #pragma unroll
@@ -700,9 +741,9 @@ scan_kernel(const __grid_constant__ ScanMaps maps, const PrefillArgs a) {
         for (int nt = 0; nt < NT; ++nt)
 #pragma unroll
             for (int hh = 0; hh < 2; ++hh) {
-                const int d = 32 * w + 16 * mt + g + 8 * hh, j = 8 * nt + 2 * tg;
+                const int d = 32 * rg + 16 * mt + g + 8 * hh, j = c0 + 8 * nt + 2 * tg;
                 float2 x = make_float2(0.f, 0.f);
-                if (a.s0) x = *reinterpret_cast<const float2 *>(a.s0 + sb + (size_t)d * Dv + j);
+                if (s_in) x = *reinterpret_cast<const float2 *>(s_in + sb + (size_t)d * Dv + j);
                 S[mt][nt][2 * hh] = x.x;
                 S[mt][nt][2 * hh + 1] = x.y;
             }
@@ -712,32 +753,30 @@ scan_kernel(const __grid_constant__ ScanMaps maps, const PrefillArgs a) {
         const uint32_t stg = smb + st * SS_STAGE;
         const float *eg_s = reinterpret_cast<const float *>(sm + st * SS_STAGE + SS_G);
         const float *ed_s = eg_s + 64;
-        uint8_t *simg = a.workspace_chunks + ((size_t)(gc0 + c) * H + h) * a.chunk_bytes + kImgS;
-        // ---- S -> bf16: row-major [d][j] in shared memory (this warpgroup's
-        //      B operand) and the MN-major SW128 image the output kernel reads
+        uint8_t *cimg = a.workspace_chunks + ((size_t)(gc0 + c) * H + h) * a.chunk_bytes;
+        // ---- S -> bf16: row-major [d][j] in shared memory (the B operand
+        //      below) and the MN-major image the output kernel reads
 #pragma unroll
         for (int mt = 0; mt < 2; ++mt)
 #pragma unroll
             for (int nt = 0; nt < NT; ++nt)
 #pragma unroll
                 for (int hh = 0; hh < 2; ++hh) {
-                    const int d = 32 * w + 16 * mt + g + 8 * hh, j = 8 * nt + 2 * tg;
+                    const int d = 32 * rg + 16 * mt + g + 8 * hh, j = c0 + 8 * nt + 2 * tg;
                     const uint32_t v = pack_bf16(S[mt][nt][2 * hh], S[mt][nt][2 * hh + 1]);
                     *reinterpret_cast<uint32_t *>(sm + SC_SS + d * RS + j * 2) = v;
-                    const int jg = j0 + j;
-                    *reinterpret_cast<uint32_t *>(simg + (jg >> 6) * 16384 + swz(d, (jg & 63) >> 3, 128) +
-                                                  (jg & 7) * 2) = v;
+                    *reinterpret_cast<uint32_t *>(cimg + kImgS + mn_off(d, j0 + j, 16384)) = v;
                 }
         if (tid == 0 && !wait_bar(&bars[SB_FULL + st], (c / kScanStages) & 1, abort_flag, a.err)) *abort_flag = 1;
-        named_bar_sync(1, 128);
+        named_bar_sync(1, NCW);
         if (*abort_flag) break;
-        // ---- U = U' + (-W) S for rows t = 16w .. 16w+15: accumulators start at U'
-        const int ta = 16 * w + g, tb = ta + 8;
+        // ---- U = U' + (-W) S for rows t = 16rg .. 16rg+15 (accumulators start at U')
+        const int ta = 16 * rg + g, tb = ta + 8;
         const uint8_t *up = sm + st * SS_STAGE + SS_U;
         float acc[2][NT][4];
 #pragma unroll
         for (int nt = 0; nt < NT; ++nt) {
-            const int j = 8 * nt + 2 * tg;
+            const int j = c0 + 8 * nt + 2 * tg;
             const float2 fa = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(up + (ta * NV + j) * 2));
             const float2 fb = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(up + (tb * NV + j) * 2));
             acc[0][nt][0] = fa.x; acc[0][nt][1] = fa.y; acc[0][nt][2] = fb.x; acc[0][nt][3] = fb.y;
@@ -745,28 +784,26 @@ scan_kernel(const __grid_constant__ ScanMaps maps, const PrefillArgs a) {
         }
 #pragma unroll
         for (int ks = 0; ks < 8; ++ks) {
-            uint32_t af[4];
-            ldsm_x4(a_addr_sw128(stg + SS_W, 16 * w, 16 * ks, lane, 8192), af);
+            uint32_t af[4], bf[NW / 4 > 4 ? NW / 4 : 4];
+            ldsm_x4(a_addr_sw128(stg + SS_W, 16 * rg, 16 * ks, lane, 8192), af);
+            ld_b<NW>(ssb, 16 * ks, c0, lane, RS, bf);
 #pragma unroll
-            for (int n2 = 0; n2 < NV / 16; ++n2) {
-                uint32_t bf[4];
-                ldsm_x4_t(b_addr_rm(ssb, 16 * ks, 16 * n2, lane, RS), bf);
-                mma16816(acc[ks & 1][2 * n2], af, bf[0], bf[1]);
-                mma16816(acc[ks & 1][2 * n2 + 1], af, bf[2], bf[3]);
-            }
+            for (int nt = 0; nt < NT; ++nt) mma16816(acc[ks & 1][nt], af, bf[2 * nt], bf[2 * nt + 1]);
         }
-        // ---- U~ = e^{g_C - g_t} U -> bf16 row-major [t][j]
+        // ---- U -> image for the output kernel; U~ = e^{g_C - g_t} U -> shared memory
         const float da = ed_s[ta], db = ed_s[tb];
 #pragma unroll
         for (int nt = 0; nt < NT; ++nt) {
-            const int j = 8 * nt + 2 * tg;
-            *reinterpret_cast<uint32_t *>(sm + SC_UT + ta * RS + j * 2) =
-                pack_bf16((acc[0][nt][0] + acc[1][nt][0]) * da, (acc[0][nt][1] + acc[1][nt][1]) * da);
-            *reinterpret_cast<uint32_t *>(sm + SC_UT + tb * RS + j * 2) =
-                pack_bf16((acc[0][nt][2] + acc[1][nt][2]) * db, (acc[0][nt][3] + acc[1][nt][3]) * db);
+            const int j = c0 + 8 * nt + 2 * tg;
+            const float u0 = acc[0][nt][0] + acc[1][nt][0], u1 = acc[0][nt][1] + acc[1][nt][1];
+            const float u2 = acc[0][nt][2] + acc[1][nt][2], u3 = acc[0][nt][3] + acc[1][nt][3];
+            *reinterpret_cast<uint32_t *>(cimg + kImgV + mn_off(ta, j0 + j, 8192)) = pack_bf16(u0, u1);
+            *reinterpret_cast<uint32_t *>(cimg + kImgV + mn_off(tb, j0 + j, 8192)) = pack_bf16(u2, u3);
+            *reinterpret_cast<uint32_t *>(sm + SC_UT + ta * RS + j * 2) = pack_bf16(u0 * da, u1 * da);
+            *reinterpret_cast<uint32_t *>(sm + SC_UT + tb * RS + j * 2) = pack_bf16(u2 * db, u3 * db);
         }
-        named_bar_sync(1, 128);
-        // ---- S <- e^{g_C} S + K^T U~ for rows d = 32w .. 32w+31
+        named_bar_sync(1, NCW);
+        // ---- S <- e^{g_C} S + K^T U~ for rows d = 32rg .. 32rg+31
         float ds[2][2][NT][4];
 #pragma unroll
         for (int p2 = 0; p2 < 2; ++p2)
@@ -777,18 +814,14 @@ scan_kernel(const __grid_constant__ ScanMaps maps, const PrefillArgs a) {
                     ds[p2][mt][nt][0] = ds[p2][mt][nt][1] = ds[p2][mt][nt][2] = ds[p2][mt][nt][3] = 0.f;
 #pragma unroll
         for (int ks = 0; ks < 4; ++ks) {
-            uint32_t bf[NV / 16][4];
-#pragma unroll
-            for (int n2 = 0; n2 < NV / 16; ++n2) ldsm_x4_t(b_addr_rm(utb, 16 * ks, 16 * n2, lane, RS), bf[n2]);
+            uint32_t bf[NW / 4 > 4 ? NW / 4 : 4];
+            ld_b<NW>(utb, 16 * ks, c0, lane, RS, bf);
 #pragma unroll
             for (int mt = 0; mt < 2; ++mt) {
                 uint32_t af[4];
-                ldsm_x4_t(at_addr_sw128(stg + SS_K, 32 * w + 16 * mt, 16 * ks, lane, 8192), af);
+                ldsm_x4_t(at_addr_sw128(stg + SS_K, 32 * rg + 16 * mt, 16 * ks, lane, 8192), af);
 #pragma unroll
-                for (int n2 = 0; n2 < NV / 16; ++n2) {
-                    mma16816(ds[ks & 1][mt][2 * n2], af, bf[n2][0], bf[n2][1]);
-                    mma16816(ds[ks & 1][mt][2 * n2 + 1], af, bf[n2][2], bf[n2][3]);
-                }
+                for (int nt = 0; nt < NT; ++nt) mma16816(ds[ks & 1][mt][nt], af, bf[2 * nt], bf[2 * nt + 1]);
             }
         }
         const float eC = eg_s[63];                    // e^{g_C}
@@ -802,52 +835,47 @@ scan_kernel(const __grid_constant__ ScanMaps maps, const PrefillArgs a) {
         mbar_arrive(&bars[SB_EMPTY + st]);
         // the next chunk rewrites the S and U~ buffers: every warp must be past
         // its reads of them
-        named_bar_sync(1, 128);
+        named_bar_sync(1, NCW);
     }
-    if (a.sf && !*abort_flag) {
+    if (s_out && !*abort_flag) {
 #pragma unroll
         for (int mt = 0; mt < 2; ++mt)
 #pragma unroll
             for (int nt = 0; nt < NT; ++nt)
 #pragma unroll
                 for (int hh = 0; hh < 2; ++hh) {
-                    const int d = 32 * w + 16 * mt + g + 8 * hh, j = 8 * nt + 2 * tg;
-                    *reinterpret_cast<float2 *>(a.sf + sb + (size_t)d * Dv + j) =
+                    const int d = 32 * rg + 16 * mt + g + 8 * hh, j = c0 + 8 * nt + 2 * tg;
+                    *reinterpret_cast<float2 *>(s_out + sb + (size_t)d * Dv + j) =
                         make_float2(S[mt][nt][2 * hh], S[mt][nt][2 * hh + 1]);
                 }
     }
 }
 
 // ---------------------------------------------------------------------------
-// Kernel 3: outputs.  One CTA per (global chunk, head), all value columns.
-//
-//   D[0:64]    = (-W) S_c          -> U = U' + D[0:64]
-//   D[64:128]  = diag(e^g) Q S_c
-//   D         += [0; P] U          -> D[64:128] = O / scale
-// Both products have M = 128 and N = Dv, the shapes tcgen05 runs well.
+// Kernel 3: outputs.  One CTA per (global chunk, head), all value columns:
+//     O = scale [diag(e^g) Q | P] [S_c ; U]        (M = 64, N = Dv, K = 192)
+// one tcgen05 accumulation chain of 12 instructions over images the prep and
+// scan kernels left in the workspace.
 // ---------------------------------------------------------------------------
-constexpr int kOutThreads = 192;      // warp 0 loads, warp 1 MMA, warps 2..5 compute
+constexpr int kOutThreads = 192;      // warp 0 loads, warp 1 MMA, warps 2..5 epilogue
 constexpr uint32_t kOutTmemCols = 128;
-constexpr uint32_t OS_A = 0;          // [-W ; diag(e^g) Q]: half h at h*16384 (rows 0..63 -W, 64..127 Q~)
-constexpr uint32_t OS_ZP = 32768;     // [0 ; P]: rows 0..63 zero, rows 64..127 P (16 KiB)
-constexpr uint32_t OS_S = 49152;      // S_c image (Dv/64 atoms of 16 KiB)
-constexpr uint32_t OS_U = OS_S;       // U image, bf16 MN-major SW128: atoms [64 rows x 128 B] of 8 KiB,
-                                      // written once the first product has consumed S_c
-constexpr uint32_t OS_UP = 81920;     // U' (64 x Dv bf16, value slices), then the decay factors
-constexpr uint32_t OS_BAR = OS_UP + 16384 + 512;
-constexpr uint32_t OS_TMEMPTR = OS_BAR + 4 * 8;
+constexpr uint32_t OS_Q = 0;          // diag(e^g) Q: 2 halves of 8 KiB (K-major SW128)
+constexpr uint32_t OS_P = 16384;      // P (8 KiB)
+constexpr uint32_t OS_S = 24576;      // S_c: Dv/64 atoms of 16 KiB (MN-major SW128)
+constexpr uint32_t OS_V = 57344;      // U:   Dv/64 atoms of 8 KiB  (MN-major SW128)
+constexpr uint32_t OS_BAR = 73728;
+constexpr uint32_t OS_TMEMPTR = OS_BAR + 2 * 8;
 constexpr uint32_t OS_FLAGS = OS_TMEMPTR + 4;
 constexpr uint32_t kOutSmem = OS_FLAGS + 4 + 1024;
-enum OutBar { OB_FULL = 0, OB_D1, OB_UREADY, OB_D2 };
+enum OutBar { OB_FULL = 0, OB_DONE };
 
-template <int NV>
-__global__ void __launch_bounds__(kOutThreads, 2)
+__global__ void __launch_bounds__(kOutThreads, 3)
 out_kernel(const PrefillArgs a) {
     extern __shared__ uint8_t smem_raw[];
     uint8_t *sm = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     ChunkLoc loc;
-    const long gc = blockIdx.x;
-    if (!locate_chunk(a, gc, loc)) return;
+    if (!locate_chunk(a, blockIdx.x, loc)) return;
+    const long gc = loc.gc;
     const int h = blockIdx.y;
     const int H = a.H, Dv = a.Dv;
     const int lenc = (int)min((long)kC, loc.len - (long)loc.c * kC);
@@ -859,19 +887,13 @@ out_kernel(const PrefillArgs a) {
     const uint8_t *img = a.workspace_chunks + ((size_t)gc * H + h) * a.chunk_bytes;
 
     if (threadIdx.x == 0) {
-        for (int i = 0; i < 4; ++i) mbar_init(&bars[i], 1);
+        for (int i = 0; i < 2; ++i) mbar_init(&bars[i], 1);
         *abort_flag = 0;
         fence_mbar_init();
     }
     if (warp == 1) {
         tmem_alloc(tmem_ptr, kOutTmemCols);
         tmem_relinquish();
-    }
-    if (warp >= 2) {
-        // zero rows 0..63 of [0 ; P]
-        for (int i = threadIdx.x - 64; i < 8192 / 16; i += 128)
-            reinterpret_cast<uint4 *>(sm + OS_ZP)[i] = make_uint4(0u, 0u, 0u, 0u);
-        fence_proxy_async_smem();
     }
     tc_fence_before();
     __syncthreads();
@@ -881,98 +903,50 @@ out_kernel(const PrefillArgs a) {
     if (warp == 0) {
         if (lane == 0) {
             uint64_t *full = &bars[OB_FULL];
-            const uint32_t sbytes = (uint32_t)(Dv / 64) * 16384;
-            mbar_arrive_expect_tx(full, 32768 + 8192 + sbytes + 64 * Dv * 2 + 512);
-            bulk_load(sm + OS_A, img + kImgW, 8192, full);
-            bulk_load(sm + OS_A + 8192, img + kImgQ, 8192, full);
-            bulk_load(sm + OS_A + 16384, img + kImgW + 8192, 8192, full);
-            bulk_load(sm + OS_A + 24576, img + kImgQ + 8192, 8192, full);
-            bulk_load(sm + OS_ZP + 8192, img + kImgP, 8192, full);
-            bulk_load(sm + OS_S, img + kImgS, sbytes, full);
-            bulk_load(sm + OS_UP, img + kImgU, 64 * Dv * 2 + 512, full);
+            const uint32_t atoms = (uint32_t)(Dv / 64);
+            mbar_arrive_expect_tx(full, 16384 + 8192 + atoms * (16384 + 8192));
+            bulk_load(sm + OS_Q, img + kImgQ, 16384, full);
+            bulk_load(sm + OS_P, img + kImgP, 8192, full);
+            bulk_load(sm + OS_S, img + kImgS, atoms * 16384, full);
+            bulk_load(sm + OS_V, img + kImgV, atoms * 8192, full);
         }
     } else if (warp == 1) {
         if (lane == 0) {
-            const uint32_t aa = smem_u32(sm + OS_A), zp = smem_u32(sm + OS_ZP);
-            const uint32_t ss = smem_u32(sm + OS_S), uu = smem_u32(sm + OS_U);
-            const uint32_t id = Dv == 128 ? idesc_bf16(128, 128, 0, 1) : idesc_bf16(128, 64, 0, 1);
-            bool ok = wait_bar(&bars[OB_FULL], 0, abort_flag, a.err);
-            if (ok) {
+            const uint32_t qq = smem_u32(sm + OS_Q), pp = smem_u32(sm + OS_P);
+            const uint32_t ss = smem_u32(sm + OS_S), vv = smem_u32(sm + OS_V);
+            const uint32_t id = Dv == 128 ? idesc_bf16(64, 128, 0, 1) : idesc_bf16(64, 64, 0, 1);
+            if (wait_bar(&bars[OB_FULL], 0, abort_flag, a.err)) {
                 tc_fence_after();
 #pragma unroll
                 for (int kk = 0; kk < 8; ++kk)
-                    mma_bf16(tmem, smem_desc(aa + (kk >> 2) * 16384 + (kk & 3) * 32, 16, 1024, kSw128),
+                    mma_bf16(tmem, smem_desc(qq + (kk >> 2) * 8192 + (kk & 3) * 32, 16, 1024, kSw128),
                              smem_desc(ss + kk * 2048, 16384, 1024, kSw128), id, kk > 0);
-                mma_commit(&bars[OB_D1]);
-                ok = wait_bar(&bars[OB_UREADY], 0, abort_flag, a.err);
-            }
-            if (ok) {
-                tc_fence_after();
 #pragma unroll
                 for (int kk = 0; kk < 4; ++kk)
-                    mma_bf16(tmem, smem_desc(zp + kk * 32, 16, 1024, kSw128),
-                             smem_desc(uu + kk * 2048, 8192, 1024, kSw128), id, 1);
-                mma_commit(&bars[OB_D2]);
+                    mma_bf16(tmem, smem_desc(pp + kk * 32, 16, 1024, kSw128),
+                             smem_desc(vv + kk * 2048, 8192, 1024, kSw128), id, 1);
+                mma_commit(&bars[OB_DONE]);
             }
         }
     } else {
         const int cw = threadIdx.x - 64;
         const int q4 = warp & 3;
-        const int r = 32 * q4 + lane;            // accumulator row = TMEM lane
         const uint32_t tq = tmem + ((uint32_t)(32 * q4) << 16);
-        if (cw == 0 && !wait_bar(&bars[OB_D1], 0, abort_flag, a.err)) *abort_flag = 1;
+        const int t = 16 * q4 + lane;            // accumulator row (M = 64 layout), lanes < 16
+        if (cw == 0 && !wait_bar(&bars[OB_DONE], 0, abort_flag, a.err)) *abort_flag = 1;
         named_bar_sync(1, 128);
         if (!*abort_flag) {
             tc_fence_after();
-            if (r < 64) {
-                // U row t = U' + (-W S)  -> MN-major SW128 image
-                const int t = r;
-                for (int j16 = 0; j16 < Dv; j16 += 16) {
-                    float x[16];
-                    tmem_ld16(tq + j16, x);
-                    tmem_wait_ld();
-                    const uint8_t *src = sm + OS_UP + (j16 / NV) * (64 * NV * 2) + (t * NV + j16 % NV) * 2;
-                    const uint4 u0 = *reinterpret_cast<const uint4 *>(src);
-                    const uint4 u1 = *reinterpret_cast<const uint4 *>(src + 16);
-                    const uint32_t uw[8] = {u0.x, u0.y, u0.z, u0.w, u1.x, u1.y, u1.z, u1.w};
+            __nv_bfloat16 *orow = static_cast<__nv_bfloat16 *>(a.out) + ((size_t)(row0 + t) * H + h) * Dv;
+            for (int j16 = 0; j16 < Dv; j16 += 16) {
+                float x[16];
+                tmem_ld16(tq + j16, x);
+                tmem_wait_ld();
+                if (lane < 16 && t < lenc) {
 #pragma unroll
-                    for (int e = 0; e < 8; ++e) {
-                        const float2 f = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(&uw[e]));
-                        x[2 * e] += f.x;
-                        x[2 * e + 1] += f.y;
-                    }
-#pragma unroll
-                    for (int h8 = 0; h8 < 2; ++h8) {
-                        const int j = j16 + 8 * h8;
-                        *reinterpret_cast<uint4 *>(sm + OS_U + (j >> 6) * 8192 + swz(t, (j & 63) >> 3, 128)) =
-                            pack8(x + 8 * h8);
-                    }
-                }
-            }
-            fence_proxy_async_smem();
-            tc_fence_before();
-        }
-        named_bar_sync(1, 128);
-        if (cw == 0 && !*abort_flag) {
-            mbar_arrive(&bars[OB_UREADY]);
-            if (!wait_bar(&bars[OB_D2], 0, abort_flag, a.err)) *abort_flag = 1;
-        }
-        named_bar_sync(1, 128);
-        if (!*abort_flag) {
-            tc_fence_after();
-            if (r >= 64) {
-                const int t = r - 64;
-                __nv_bfloat16 *orow = static_cast<__nv_bfloat16 *>(a.out) + ((size_t)(row0 + t) * H + h) * Dv;
-                for (int j16 = 0; j16 < Dv; j16 += 16) {
-                    float x[16];
-                    tmem_ld16(tq + j16, x);
-                    tmem_wait_ld();
-                    if (t < lenc) {
-#pragma unroll
-                        for (int e = 0; e < 16; ++e) x[e] *= a.scale;
-                        *reinterpret_cast<uint4 *>(orow + j16) = pack8(x);
-                        *reinterpret_cast<uint4 *>(orow + j16 + 8) = pack8(x + 8);
-                    }
+                    for (int e = 0; e < 16; ++e) x[e] *= a.scale;
+                    *reinterpret_cast<uint4 *>(orow + j16) = pack8(x);
+                    *reinterpret_cast<uint4 *>(orow + j16 + 8) = pack8(x + 8);
                 }
             }
         }
@@ -1060,21 +1034,27 @@ cudaError_t set_smem(K kernel, uint32_t bytes) {
 }
 
 int choose_nv(long units, int Dv) {
-    // The scan is latency-bound per chunk: narrow slices give more CTAs at
-    // little extra cost; widen them once the SMs are covered.
+    // The scan is bound by MMA throughput per SM: narrow slices spread a head
+    // over more SMs; widen them once the SMs are covered.
     return units * (Dv / 32) >= 148 ? 32 : 16;
 }
 
 template <int NV>
-cudaError_t launch_nv(const PrefillArgs &a, long chunks_grid, cudaStream_t s) {
+cudaError_t init_attrs() {
     static std::once_flag once;
     static cudaError_t attr = cudaSuccess;
     std::call_once(once, [] {
         attr = set_smem(prep_kernel<NV>, kPrepSmem);
-        if (attr == cudaSuccess) attr = set_smem(scan_kernel<NV>, kScanSmem);
-        if (attr == cudaSuccess) attr = set_smem(out_kernel<NV>, kOutSmem);
+        if (attr == cudaSuccess) attr = set_smem(scan_kernel<NV>, ScanSmem<NV>::BYTES);
+        if (attr == cudaSuccess) attr = set_smem(out_kernel, kOutSmem);
     });
-    if (attr != cudaSuccess) return attr;
+    return attr;
+}
+
+template <int NV>
+cudaError_t launch_nv(const PrefillArgs &a, long chunks_grid, cudaStream_t s) {
+    cudaError_t e = init_attrs<NV>();
+    if (e != cudaSuccess) return e;
     PrepMaps pm;
     ScanMaps sm;
     std::memset(&pm, 0, sizeof(pm));
@@ -1085,15 +1065,16 @@ cudaError_t launch_nv(const PrefillArgs &a, long chunks_grid, cudaStream_t s) {
             return cudaErrorInvalidValue;
         sm.k = pm.k;
     }
+    const dim3 scan_grid(a.Dv / NV, a.H, a.num_seqs);
+    const uint32_t scan_smem = ScanSmem<NV>::BYTES;
+
     if (chunks_grid > 0) {
         prep_kernel<NV><<<dim3((unsigned)chunks_grid, a.H, 1), kPrepThreads, kPrepSmem, s>>>(pm, a);
-        cudaError_t e = cudaGetLastError();
-        if (e != cudaSuccess) return e;
+        if ((e = cudaGetLastError()) != cudaSuccess) return e;
     }
-    scan_kernel<NV><<<dim3(a.Dv / NV, a.H, a.num_seqs), kScanThreads, kScanSmem, s>>>(sm, a);
-    cudaError_t e = cudaGetLastError();
-    if (e != cudaSuccess || chunks_grid == 0) return e;
-    out_kernel<NV><<<dim3((unsigned)chunks_grid, a.H, 1), kOutThreads, kOutSmem, s>>>(a);
+    scan_kernel<NV><<<scan_grid, kScanThreads, scan_smem, s>>>(sm, a);
+    if ((e = cudaGetLastError()) != cudaSuccess || chunks_grid == 0) return e;
+    out_kernel<<<dim3((unsigned)chunks_grid, a.H, 1), kOutThreads, kOutSmem, s>>>(a);
     return cudaGetLastError();
 }
 
@@ -1120,7 +1101,8 @@ size_t chunked_workspace_bytes(long total_T, int T, int B, int H, int Dv, int nu
 cudaError_t launch_chunked(const PrefillArgs &a0, void *scratch, cudaStream_t s) {
     PrefillArgs a = a0;
     uint8_t *ws = static_cast<uint8_t *>(scratch);
-    a.workspace_chunks = ws + header_bytes(a.cu_seqlens ? a.num_seqs : 0);
+    const int nseq_hdr = a.cu_seqlens ? a.num_seqs : 0;
+    a.workspace_chunks = ws + header_bytes(nseq_hdr);
     a.chunk_bytes = image_bytes(a.Dv);
     long chunks_grid;
     if (a.cu_seqlens) {

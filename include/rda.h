@@ -92,8 +92,8 @@ const char *rda_version(void);
  * rda_prefill_varlen (num_seqs = N, pass B = 1 and T = total_T) needs for
  * these sizes, enough for either dtype.  Always >= 256: the first 256 bytes
  * hold the device error word.  When the chunked tensor-core path can run
- * (Dk = 128) it also holds that path's per-chunk scratch, about 88.5 KiB per
- * 64-token chunk and head at Dv = 128 (e.g. 90.6 MB for B=1, T=4096, H=16).
+ * (Dk = 128) it also holds that path's per-chunk scratch, about 104.5 KiB
+ * per 64-token chunk and head at Dv = 128 (e.g. 110 MB for B=1, T=4096, H=16).
  * The workspace must be 256-byte aligned; its contents need no
  * initialisation beyond a cleared error word, and are overwritten by each
  * call.  Returns 0 for unsupported sizes.

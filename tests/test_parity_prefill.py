@@ -127,3 +127,20 @@ def test_in_place_final_state(cuda_device):
     torch.cuda.synchronize()
     assert rel_l2(st.double().cpu().numpy(), rs) < 1e-2
     assert rel_l2(out.double().cpu().numpy(), ro) < 1e-2
+
+
+@pytest.mark.parametrize("Dv", [64, 128])
+def test_bf16_long_odd_chunk_count(cuda_device, Dv):
+    """38 chunks (an odd count) with a ragged tail, B > 1, write gate, and the
+    final state written over the initial one."""
+    import gated_delta_rule_rda_b200 as rda
+    inp = rda_gen.fixed_inputs(2, 64 * 37 + 5, 3, 128, Dv, dtype=torch.bfloat16, seed=40 + Dv, s0=True,
+                               gamma=True)
+    ro, rs = oracle_fixed(inp, scale=0.5)
+    d = inp.to("cuda")
+    st = d.initial_state.clone()
+    out, _ = rda.rda_prefill_chunked(d.q, d.k, d.v, d.log_alpha, d.beta, write_gate=d.gamma,
+                                     initial_state=st, final_state=st, scale=0.5)
+    torch.cuda.synchronize()
+    assert rel_l2(out.double().cpu().numpy(), ro) <= 1e-2
+    assert rel_l2(st.double().cpu().numpy(), rs) <= 1e-2
