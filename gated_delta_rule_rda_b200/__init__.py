@@ -49,6 +49,8 @@ lib.rda_decode_step.argtypes = [_vp] * 8 + [_i] * 5 + [_f, _vp]
 lib.rda_decode_step.restype = _i
 lib.rda_read_device_error.argtypes = [_vp, ctypes.POINTER(_i), _vp]
 lib.rda_read_device_error.restype = _i
+lib.rda_prefill_chunked_noalloc.argtypes = [_vp] * 9 + [_i] * 6 + [_f, _vp]
+lib.rda_prefill_chunked_noalloc.restype = _i
 
 RDA_OK = 0
 RDA_F32 = 0
@@ -207,6 +209,28 @@ def rda_decode_step(q, k, v, log_alpha, beta, state, write_gate=None, scale=1.0,
     return out
 
 
+def rda_prefill_chunked_noalloc(q, k, v, log_alpha, beta, write_gate=None, initial_state=None,
+                                scale=1.0, out=None, final_state=None, stream=None):
+    """rda_prefill_chunked without a workspace: for callers that cannot give
+    the library scratch memory.  Uses the library's fixed 64 MiB device array
+    (see include/rda.h); larger problems raise RdaError (RDA_ERR_WORKSPACE)."""
+    B, T, H, Dk = q.shape
+    Dv = v.shape[-1]
+    _need_cuda(q, k, v, log_alpha, beta, write_gate, initial_state, out, final_state)
+    _need_f32(log_alpha, beta, write_gate, initial_state, final_state)
+    dt = _dtype_code(q)
+    if out is None:
+        out = torch.empty((B, T, H, Dv), dtype=q.dtype, device=q.device)
+    if final_state is None:
+        final_state = torch.empty((B, H, Dk, Dv), dtype=torch.float32, device=q.device)
+    code = lib.rda_prefill_chunked_noalloc(_ptr(q), _ptr(k), _ptr(v), _ptr(log_alpha), _ptr(beta),
+                                           _ptr(write_gate), _ptr(initial_state), _ptr(final_state),
+                                           _ptr(out), dt, B, T, H, Dk, Dv, float(scale),
+                                           _stream(stream))
+    _check(code, "rda_prefill_chunked_noalloc")
+    return out, final_state
+
+
 def rda_read_device_error(workspace, stream=None) -> int:
     code = _i(0)
     _check(lib.rda_read_device_error(_ptr(workspace), ctypes.byref(code), _stream(stream)),
@@ -215,5 +239,6 @@ def rda_read_device_error(workspace, stream=None) -> int:
 
 
 __all__ = ["rda_prefill_chunked", "rda_prefill_varlen", "rda_decode_step",
+           "rda_prefill_chunked_noalloc",
            "rda_read_device_error", "rda_prefill_workspace_bytes", "new_workspace", "version",
            "RdaError", "lib", "LIB_PATH"]

@@ -174,6 +174,36 @@ rda_status_t rda_decode_step(const void *q, const void *k, const void *v,
                              int B, int H, int Dk, int Dv, float scale, void *stream);
 
 /*
+ * Fixed-length prefill that allocates nothing and takes no workspace.
+ *
+ * The pages describe no such call; it exists for callers that cannot give the
+ * library scratch memory: host programs that own all device memory themselves
+ * (an inference server that sizes its memory pool once at start-up and allows
+ * no cudaMalloc afterwards, a plug-in whose host framework passes tensors but
+ * offers no way to ask for scratch).  Arguments, layouts, results and errors
+ * are those of rda_prefill_chunked; it calls no cudaMalloc, cudaFree or other
+ * allocating routine.
+ *
+ * Its scratch is a fixed 64 MiB array in device memory that every GPU loading
+ * this library holds until the process exits.  Problems whose
+ * rda_prefill_workspace_bytes(B,T,H,Dk,Dv,0) exceeds 64 MiB are rejected with
+ * RDA_ERR_WORKSPACE before anything is enqueued (at Dv = 128 the limit is
+ * about 600 chunk-head pairs, e.g. B = 1, T = 2048, H = 16).  The first call on
+ * a device looks up the array's device address; make that first call before
+ * any stream capture.  All calls on a device share the array, which keeps the
+ * last call's contents: calls whose work overlaps on the GPU (unordered
+ * streams) race on it.  Each call clears the array's device error word before
+ * launching; a device-side timeout is not reported back through this call.
+ */
+rda_status_t rda_prefill_chunked_noalloc(const void *q, const void *k, const void *v,
+                                         const float *log_alpha, const float *beta,
+                                         const float *write_gate,
+                                         const float *initial_state, float *final_state,
+                                         void *out, rda_dtype_t dtype,
+                                         int B, int T, int H, int Dk, int Dv, float scale,
+                                         void *stream);
+
+/*
  * Waits for `stream`, then reads and clears the device error word at the start
  * of `workspace`.  Writes RDA_OK or the recorded code to *code.  Returns
  * RDA_ERR_CUDA if the copy fails.
