@@ -270,6 +270,10 @@ def run_ours(args, rank, world, device):
                "tokens_per_s": Bd * world / (dms * 1e-3)}
         del din, st
 
+    extra = {}
+    if args.all:
+        extra = other_workloads(device, stream, rank, world)
+
     clocks = None
     if sampler:
         sampler.stop()
@@ -308,7 +312,61 @@ def run_ours(args, rank, world, device):
         "gpu_launches": args.steps,
         "clocks": clocks,
         "decode": dec,
+        **extra,
     }
+
+
+def other_workloads(device, stream, rank, world, reps=5):
+    """Long-context and packed (varlen) prefill: event-timed, L2 flushed between
+    repetitions (both inputs are larger than L2 anyway)."""
+    import torch
+    import gated_delta_rule_rda_b200 as rda
+    import rda_gen
+    res = {}
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device=device)
+
+    def timed(fn):
+        for _ in range(2):
+            fn()
+        ts = []
+        for _ in range(reps):
+            flush.zero_()
+            s, e = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            s.record(stream)
+            fn()
+            e.record(stream)
+            ts.append((s, e))
+        torch.cuda.synchronize()
+        return sorted(a.elapsed_time(b) for a, b in ts)[len(ts) // 2]
+
+    inp = rda_gen.workload("long_prefill_b1_t32768_h16_d128").to(device)
+    B, T, H, Dk = inp.q.shape
+    ws = rda.new_workspace(rda.rda_prefill_workspace_bytes(B, T, H, Dk, Dk, 0), device)
+    out = torch.empty_like(inp.v)
+    sf = torch.empty((B, H, Dk, Dk), device=device)
+    ms = timed(lambda: rda.rda_prefill_chunked(inp.q, inp.k, inp.v, inp.log_alpha, inp.beta,
+                                               out=out, final_state=sf, workspace=ws))
+    nbytes = B * T * H * prefill_bytes_per_token_head() + B * state_bytes(H, Dk, Dk)
+    res["long_prefill"] = {"workload": "long_prefill_b1_t32768_h16_d128", "ms": ms,
+                           "tokens_per_s": world * B * T / (ms * 1e-3),
+                           "hbm_frac": nbytes / (ms * 1e-3) / 1e9 / load_peaks()[0]}
+    del inp, ws, out, sf
+    vin = rda_gen.workload("varlen_64seqs_128to8192_h16_d128")
+    d = vin.to(device)
+    total, H, Dk = vin.q.shape
+    N = vin.cu_seqlens.numel() - 1
+    ws = rda.new_workspace(rda.rda_prefill_workspace_bytes(1, total, H, Dk, Dk, N), device)
+    out = torch.empty_like(d.v)
+    sf = torch.empty((N, H, Dk, Dk), device=device)
+    ms = timed(lambda: rda.rda_prefill_varlen(d.q, d.k, d.v, d.log_alpha, d.beta, d.cu_seqlens,
+                                              initial_states=d.initial_states, out=out,
+                                              final_states=sf, cu_seqlens_host=vin.cu_seqlens,
+                                              workspace=ws))
+    nbytes = total * H * prefill_bytes_per_token_head() + 2 * N * state_bytes(H, Dk, Dk)
+    res["varlen_prefill"] = {"workload": "varlen_64seqs_128to8192_h16_d128", "tokens": total,
+                             "ms": ms, "tokens_per_s": world * total / (ms * 1e-3),
+                             "hbm_frac": nbytes / (ms * 1e-3) / 1e9 / load_peaks()[0]}
+    return res
 
 
 # ------------------------------------------------------------------ oracle timing
@@ -389,6 +447,8 @@ def main():
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--no-decode", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--all", action="store_true",
+                    help="also time the long-context and packed (varlen) prefill workloads")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")

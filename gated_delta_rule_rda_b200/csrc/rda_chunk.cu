@@ -575,7 +575,7 @@ prep_kernel(const __grid_constant__ PrepMaps maps, const PrefillArgs a) {
 // ---------------------------------------------------------------------------
 constexpr int kScanWarps = 4;
 constexpr int kScanThreads = (kScanWarps + 1) * 32;
-constexpr int kScanStages = 3;
+constexpr int kScanStages = 4;
 // per-stage shared memory (bytes): -W 16K | K 16K | U' <= 4K | decay 512
 constexpr uint32_t SS_W = 0, SS_K = 16384, SS_U = 32768, SS_G = 36864;
 constexpr uint32_t SS_STAGE = 37888;                          // multiple of 1024
@@ -782,13 +782,22 @@ scan_kernel(const __grid_constant__ ScanMaps maps, const PrefillArgs a) {
             acc[0][nt][0] = fa.x; acc[0][nt][1] = fa.y; acc[0][nt][2] = fb.x; acc[0][nt][3] = fb.y;
             acc[1][nt][0] = acc[1][nt][1] = acc[1][nt][2] = acc[1][nt][3] = 0.f;
         }
+        // operands of a group of k-steps are loaded before its MMAs are issued, so
+        // the shared-memory latency is paid once per group
+        constexpr int KGU = NW >= 32 ? 4 : 8;
 #pragma unroll
-        for (int ks = 0; ks < 8; ++ks) {
-            uint32_t af[4], bf[NW / 4 > 4 ? NW / 4 : 4];
-            ldsm_x4(a_addr_sw128(stg + SS_W, 16 * rg, 16 * ks, lane, 8192), af);
-            ld_b<NW>(ssb, 16 * ks, c0, lane, RS, bf);
+        for (int k0 = 0; k0 < 8; k0 += KGU) {
+            uint32_t af[KGU][4], bf[KGU][NW / 4 > 4 ? NW / 4 : 4];
 #pragma unroll
-            for (int nt = 0; nt < NT; ++nt) mma16816(acc[ks & 1][nt], af, bf[2 * nt], bf[2 * nt + 1]);
+            for (int kk = 0; kk < KGU; ++kk) {
+                ldsm_x4(a_addr_sw128(stg + SS_W, 16 * rg, 16 * (k0 + kk), lane, 8192), af[kk]);
+                ld_b<NW>(ssb, 16 * (k0 + kk), c0, lane, RS, bf[kk]);
+            }
+#pragma unroll
+            for (int kk = 0; kk < KGU; ++kk)
+#pragma unroll
+                for (int nt = 0; nt < NT; ++nt)
+                    mma16816(acc[kk & 1][nt], af[kk], bf[kk][2 * nt], bf[kk][2 * nt + 1]);
         }
         // ---- U -> image for the output kernel; U~ = e^{g_C - g_t} U -> shared memory
         const float da = ed_s[ta], db = ed_s[tb];
@@ -812,17 +821,24 @@ scan_kernel(const __grid_constant__ ScanMaps maps, const PrefillArgs a) {
 #pragma unroll
                 for (int nt = 0; nt < NT; ++nt)
                     ds[p2][mt][nt][0] = ds[p2][mt][nt][1] = ds[p2][mt][nt][2] = ds[p2][mt][nt][3] = 0.f;
+        constexpr int KGD = NW >= 32 ? 2 : 4;
 #pragma unroll
-        for (int ks = 0; ks < 4; ++ks) {
-            uint32_t bf[NW / 4 > 4 ? NW / 4 : 4];
-            ld_b<NW>(utb, 16 * ks, c0, lane, RS, bf);
+        for (int k0 = 0; k0 < 4; k0 += KGD) {
+            uint32_t af[KGD][2][4], bf[KGD][NW / 4 > 4 ? NW / 4 : 4];
 #pragma unroll
-            for (int mt = 0; mt < 2; ++mt) {
-                uint32_t af[4];
-                ldsm_x4_t(at_addr_sw128(stg + SS_K, 32 * rg + 16 * mt, 16 * ks, lane, 8192), af);
+            for (int kk = 0; kk < KGD; ++kk) {
+                ld_b<NW>(utb, 16 * (k0 + kk), c0, lane, RS, bf[kk]);
 #pragma unroll
-                for (int nt = 0; nt < NT; ++nt) mma16816(ds[ks & 1][mt][nt], af, bf[2 * nt], bf[2 * nt + 1]);
+                for (int mt = 0; mt < 2; ++mt)
+                    ldsm_x4_t(at_addr_sw128(stg + SS_K, 32 * rg + 16 * mt, 16 * (k0 + kk), lane, 8192), af[kk][mt]);
             }
+#pragma unroll
+            for (int kk = 0; kk < KGD; ++kk)
+#pragma unroll
+                for (int mt = 0; mt < 2; ++mt)
+#pragma unroll
+                    for (int nt = 0; nt < NT; ++nt)
+                        mma16816(ds[kk & 1][mt][nt], af[kk][mt], bf[kk][2 * nt], bf[kk][2 * nt + 1]);
         }
         const float eC = eg_s[63];                    // e^{g_C}
 #pragma unroll
@@ -833,9 +849,10 @@ scan_kernel(const __grid_constant__ ScanMaps maps, const PrefillArgs a) {
                 for (int i = 0; i < 4; ++i)
                     S[mt][nt][i] = fmaf(eC, S[mt][nt][i], ds[0][mt][nt][i] + ds[1][mt][nt][i]);
         mbar_arrive(&bars[SB_EMPTY + st]);
-        // the next chunk rewrites the S and U~ buffers: every warp must be past
-        // its reads of them
-        named_bar_sync(1, NCW);
+        // No barrier here: the next chunk writes the state buffer after every
+        // warp passed this chunk's second barrier (its reads of the state are
+        // done), and U~ after the next first barrier (every warp is past this
+        // chunk's update).
     }
     if (s_out && !*abort_flag) {
 #pragma unroll
