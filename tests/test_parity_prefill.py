@@ -144,3 +144,12 @@ def test_bf16_long_odd_chunk_count(cuda_device, Dv):
     torch.cuda.synchronize()
     assert rel_l2(out.double().cpu().numpy(), ro) <= 1e-2
     assert rel_l2(st.double().cpu().numpy(), rs) <= 1e-2
+
+
+@pytest.mark.parametrize("B,H", [(2, 12), (3, 13)])
+def test_bf16_many_heads(cuda_device, B, H):
+    """Many (sequence, head) pairs: the scan runs more CTAs than there are SMs,
+    with value slices of 16 columns (B=2, H=12) and of 32 columns (B=3, H=13)."""
+    inp = rda_gen.fixed_inputs(B, 130, H, 128, 128, dtype=torch.bfloat16, seed=B * 100 + H, s0=True,
+                               gamma=True)
+    _check(inp, scale=0.75)
