@@ -366,6 +366,40 @@ def other_workloads(device, stream, rank, world, reps=5):
     res["varlen_prefill"] = {"workload": "varlen_64seqs_128to8192_h16_d128", "tokens": total,
                              "ms": ms, "tokens_per_s": world * total / (ms * 1e-3),
                              "hbm_frac": nbytes / (ms * 1e-3) / 1e9 / load_peaks()[0]}
+    del d, vin, ws, out, sf
+
+    # mini shape (H = 40) prefill, same kernels
+    inp = rda_gen.workload("mini_prefill_b1_t4096_h40_d128").to(device)
+    B, T, H, Dk = inp.q.shape
+    ws = rda.new_workspace(rda.rda_prefill_workspace_bytes(B, T, H, Dk, Dk, 0), device)
+    out = torch.empty_like(inp.v)
+    sf = torch.empty((B, H, Dk, Dk), device=device)
+    ms = timed(lambda: rda.rda_prefill_chunked(inp.q, inp.k, inp.v, inp.log_alpha, inp.beta,
+                                               initial_state=inp.initial_state, out=out,
+                                               final_state=sf, workspace=ws))
+    nbytes = B * T * H * prefill_bytes_per_token_head() + 2 * B * state_bytes(H, Dk, Dk)
+    res["mini_prefill"] = {"workload": "mini_prefill_b1_t4096_h40_d128", "ms": ms,
+                           "tokens_per_s": world * B * T / (ms * 1e-3),
+                           "hbm_frac": nbytes / (ms * 1e-3) / 1e9 / load_peaks()[0]}
+    del inp, ws, out, sf
+
+    # multi-token decode: the decode workload's 128 tokens as 16 calls of 8
+    din = rda_gen.workload("decode_b256_h16_d128_128steps")
+    blocks = [[x[t0:t0 + 8].transpose(0, 1).contiguous().to(device)
+               for x in (din.q, din.k, din.v, din.log_alpha, din.beta)] for t0 in range(0, 128, 8)]
+    st = din.state.to(device)
+    Bd, H, Dk, Dv = st.shape
+    dout = torch.empty((Bd, 8, H, Dv), dtype=din.q.dtype, device=device)
+
+    def tok_rep():
+        for q, k, v, la, be in blocks:
+            rda.rda_decode_tokens(q, k, v, la, be, st, out=dout)
+    ms = timed(tok_rep) / len(blocks)
+    bytes_call = Bd * H * (2 * state_bytes(1, Dk, Dv) + 8 * prefill_bytes_per_token_head())
+    gbs = bytes_call / (ms * 1e-3) / 1e9
+    res["decode_tokens"] = {"workload": "decode_b256_h16_d128_128steps, 8 tokens per call",
+                            "ms_per_call": ms, "tokens_per_s": world * Bd * 8 / (ms * 1e-3),
+                            "state_gbs": world * gbs, "hbm_frac": gbs / load_peaks()[0]}
     return res
 
 

@@ -47,6 +47,8 @@ lib.rda_prefill_varlen.argtypes = [_vp] * 8 + [_i, _i, _vp, _vp, _vp, _i, _i, _i
 lib.rda_prefill_varlen.restype = _i
 lib.rda_decode_step.argtypes = [_vp] * 8 + [_i] * 5 + [_f, _vp]
 lib.rda_decode_step.restype = _i
+lib.rda_decode_tokens.argtypes = [_vp] * 8 + [_i] * 6 + [_f, _vp]
+lib.rda_decode_tokens.restype = _i
 lib.rda_read_device_error.argtypes = [_vp, ctypes.POINTER(_i), _vp]
 lib.rda_read_device_error.restype = _i
 lib.rda_prefill_chunked_noalloc.argtypes = [_vp] * 9 + [_i] * 6 + [_f, _vp]
@@ -209,6 +211,25 @@ def rda_decode_step(q, k, v, log_alpha, beta, state, write_gate=None, scale=1.0,
     return out
 
 
+def rda_decode_tokens(q, k, v, log_alpha, beta, state, write_gate=None, scale=1.0, out=None,
+                      stream=None):
+    """T (<= 8) decode steps in one pass over the state.  q, k ``[B,T,H,Dk]``;
+    v ``[B,T,H,Dv]``; gates fp32 ``[B,T,H]``; state fp32 ``[B,H,Dk,Dv]`` updated
+    in place.  Returns ``out [B,T,H,Dv]``."""
+    B, T, H, Dk = q.shape
+    Dv = v.shape[-1]
+    _need_cuda(q, k, v, log_alpha, beta, state, write_gate, out)
+    _need_f32(log_alpha, beta, state, write_gate)
+    dt = _dtype_code(q)
+    if out is None:
+        out = torch.empty((B, T, H, Dv), dtype=q.dtype, device=q.device)
+    code = lib.rda_decode_tokens(_ptr(q), _ptr(k), _ptr(v), _ptr(log_alpha), _ptr(beta),
+                                 _ptr(write_gate), _ptr(state), _ptr(out), dt, B, T, H, Dk, Dv,
+                                 float(scale), _stream(stream))
+    _check(code, "rda_decode_tokens")
+    return out
+
+
 def rda_prefill_chunked_noalloc(q, k, v, log_alpha, beta, write_gate=None, initial_state=None,
                                 scale=1.0, out=None, final_state=None, stream=None):
     """rda_prefill_chunked without a workspace: for callers that cannot give
@@ -238,7 +259,7 @@ def rda_read_device_error(workspace, stream=None) -> int:
     return int(code.value)
 
 
-__all__ = ["rda_prefill_chunked", "rda_prefill_varlen", "rda_decode_step",
+__all__ = ["rda_prefill_chunked", "rda_prefill_varlen", "rda_decode_step", "rda_decode_tokens",
            "rda_prefill_chunked_noalloc",
            "rda_read_device_error", "rda_prefill_workspace_bytes", "new_workspace", "version",
            "RdaError", "lib", "LIB_PATH"]

@@ -202,6 +202,32 @@ rda_status_t rda_decode_step(const void *q, const void *k, const void *v,
     return launch_decode(a, dtype, static_cast<cudaStream_t>(stream)) == cudaSuccess ? RDA_OK : RDA_ERR_CUDA;
 }
 
+rda_status_t rda_decode_tokens(const void *q, const void *k, const void *v,
+                               const float *log_alpha, const float *beta,
+                               const float *write_gate,
+                               float *state, void *out, rda_dtype_t dtype,
+                               int B, int T, int H, int Dk, int Dv, float scale, void *stream) {
+    if (dtype != RDA_F32 && dtype != RDA_BF16) return RDA_ERR_UNSUPPORTED;
+    if (B < 0 || H <= 0 || T < 0) return RDA_ERR_INVALID_ARG;
+    if (T > kMaxDecodeTokens) return RDA_ERR_UNSUPPORTED;
+    if (!dims_ok(Dk, Dv)) return RDA_ERR_UNSUPPORTED;
+    if ((long long)B * H * Dk * Dv >= (1LL << 31) || (long long)B * T * H * (Dk > Dv ? Dk : Dv) >= (1LL << 31))
+        return RDA_ERR_INVALID_ARG;
+    if (B == 0 || T == 0) return RDA_OK;
+    rda_status_t st = check_io_ptrs(q, k, v, log_alpha, beta, out);
+    if (st != RDA_OK) return st;
+    if (!state) return RDA_ERR_INVALID_ARG;
+    if (!aligned(state, 16)) return RDA_ERR_MISALIGNED;
+    if (write_gate && !aligned(write_gate, 4)) return RDA_ERR_MISALIGNED;
+    DecodeArgs a{};
+    a.q = q; a.k = k; a.v = v;
+    a.log_alpha = log_alpha; a.beta = beta; a.gamma = write_gate;
+    a.state = state; a.out = out;
+    a.B = B; a.T = T; a.H = H; a.Dk = Dk; a.Dv = Dv; a.scale = scale;
+    return launch_decode_tokens(a, dtype, static_cast<cudaStream_t>(stream)) == cudaSuccess ? RDA_OK
+                                                                                              : RDA_ERR_CUDA;
+}
+
 rda_status_t rda_read_device_error(void *workspace, int *code, void *stream) {
     if (!workspace || !code) return RDA_ERR_INVALID_ARG;
     cudaStream_t s = static_cast<cudaStream_t>(stream);

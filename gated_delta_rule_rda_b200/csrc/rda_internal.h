@@ -44,10 +44,15 @@ struct DecodeArgs {
     void *out;
     int B, H, Dk, Dv;
     float scale;
+    int T;                       // tokens per sequence (multi-token decode only)
 };
+
+// Most tokens one multi-token decode call takes per sequence.
+constexpr int kMaxDecodeTokens = 8;
 
 cudaError_t launch_recurrent(const PrefillArgs &a, rda_dtype_t dtype, cudaStream_t s);
 cudaError_t launch_decode(const DecodeArgs &a, rda_dtype_t dtype, cudaStream_t s);
+cudaError_t launch_decode_tokens(const DecodeArgs &a, rda_dtype_t dtype, cudaStream_t s);
 // Chunked tensor-core prefill (bf16, Dk = 128, Dv in {64, 128}).  `scratch`
 // points at chunked_workspace_bytes() bytes of device memory (256-aligned).
 cudaError_t launch_chunked(const PrefillArgs &a, void *scratch, cudaStream_t s);

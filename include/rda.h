@@ -174,6 +174,29 @@ rda_status_t rda_decode_step(const void *q, const void *k, const void *v,
                              int B, int H, int Dk, int Dv, float scale, void *stream);
 
 /*
+ * Multi-token decode: T new tokens per sequence (1 <= T <= 8), state updated in
+ * place, with the result of T successive rda_decode_step calls (equivalently,
+ * a T-token prefill from the state).  For speculative decoding: the model card
+ * "KRAFTON/Raon-1-nano-gguf" (section "Model: KRAFTON/Raon-1-nano-gguf") runs
+ * multi-token prediction with draft tokens per step, and the blog post on
+ * Raon-1 mini (section "Bạn có thể chạy gì trong tuần này") quotes a draft model
+ * at block size 8.  The state is read and written once whatever T is: after t
+ * tokens every row of the state is a combination of its old value and the new
+ * keys, so the kernel needs only the old state's products with the T keys and
+ * queries, and the tokens' Gram values.
+ *
+ *   q, k   device, dtype, [B,T,H,Dk];  v, out device, dtype, [B,T,H,Dv]
+ *   log_alpha, beta  device fp32 [B,T,H];  write_gate device fp32 [B,T,H] or NULL
+ *   state  device fp32 [B,H,Dk,Dv], read and overwritten, 16-byte aligned
+ * Returns RDA_ERR_UNSUPPORTED for T > 8; T = 0 (or B = 0) does nothing.
+ */
+rda_status_t rda_decode_tokens(const void *q, const void *k, const void *v,
+                               const float *log_alpha, const float *beta,
+                               const float *write_gate,
+                               float *state, void *out, rda_dtype_t dtype,
+                               int B, int T, int H, int Dk, int Dv, float scale, void *stream);
+
+/*
  * Fixed-length prefill that allocates nothing and takes no workspace.
  *
  * The pages describe no such call; it exists for callers that cannot give the

@@ -187,7 +187,7 @@ def decode_inputs(B=256, H=16, Dk=128, Dv=128, steps=128, dtype=torch.bfloat16, 
                         dict(B=B, H=H, Dk=Dk, Dv=Dv, steps=steps, dtype=dtype, seed=seed))
 
 
-# The five measured workloads.  Seeds are the workload numbers.
+# The measured workloads.  Seeds are the workload numbers (the mini shape, H = 40, is 6).
 WORKLOADS = {
     "fp32_parity_b1_t256_h2_d64": dict(kind="fixed", B=1, T=256, H=2, Dk=64, Dv=64,
                                        dtype=torch.float32, seed=1, s0=False, decay="softplus"),
@@ -197,6 +197,9 @@ WORKLOADS = {
     "long_prefill_b1_t32768_h16_d128": dict(kind="fixed", B=1, T=32768, H=16, Dk=128, Dv=128,
                                             dtype=torch.bfloat16, seed=3, s0=False,
                                             decay="uniform"),
+    "mini_prefill_b1_t4096_h40_d128": dict(kind="fixed", B=1, T=4096, H=40, Dk=128, Dv=128,
+                                           dtype=torch.bfloat16, seed=6, s0=True,
+                                           decay="softplus"),
     "decode_b256_h16_d128_128steps": dict(kind="decode", B=256, H=16, Dk=128, Dv=128,
                                           steps=128, dtype=torch.bfloat16, seed=4),
     "varlen_64seqs_128to8192_h16_d128": dict(kind="varlen", num_seqs=64, min_len=128,

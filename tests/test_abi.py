@@ -23,7 +23,7 @@ def _declared_functions():
 
 def test_header_declares_the_entry_points():
     names = _declared_functions()
-    for want in ["rda_prefill_chunked", "rda_prefill_varlen", "rda_decode_step",
+    for want in ["rda_prefill_chunked", "rda_prefill_varlen", "rda_decode_step", "rda_decode_tokens",
                  "rda_prefill_workspace_bytes", "rda_read_device_error", "rda_status_string",
                  "rda_version"]:
         assert want in names
@@ -138,3 +138,24 @@ def test_python_binding_refuses_cpu_tensors():
     q = torch.zeros(1, 4, 1, 64)
     with pytest.raises(ValueError, match="CUDA"):
         rda.rda_prefill_chunked(q, q, q, torch.zeros(1, 4, 1), torch.zeros(1, 4, 1))
+
+
+def _tokens(**kw):
+    args = dict(q=A16, k=A16, v=A16, la=A16, be=A16, wg=None, st=A16, out=A16, dtype=1, B=4, T=4, H=2,
+                Dk=128, Dv=128, scale=1.0, stream=None)
+    args.update(kw)
+    return rda.lib.rda_decode_tokens(*[args[k] for k in ["q", "k", "v", "la", "be", "wg", "st", "out",
+                                                         "dtype", "B", "T", "H", "Dk", "Dv", "scale",
+                                                         "stream"]])
+
+
+def test_decode_tokens_rejects_bad_arguments():
+    assert _tokens(T=9) == UNSUPPORTED              # at most 8 tokens per call
+    assert _tokens(T=-1) == INVALID
+    assert _tokens(st=None) == INVALID
+    assert _tokens(st=A16 + 4) == MISALIGNED
+    assert _tokens(q=A16 + 2) == MISALIGNED
+    assert _tokens(Dk=96) == UNSUPPORTED
+    assert _tokens(dtype=3) == UNSUPPORTED
+    assert _tokens(T=0) == OK                       # nothing to do, nothing launched
+    assert _tokens(B=0) == OK

@@ -153,3 +153,9 @@ def test_bf16_many_heads(cuda_device, B, H):
     inp = rda_gen.fixed_inputs(B, 130, H, 128, 128, dtype=torch.bfloat16, seed=B * 100 + H, s0=True,
                                gamma=True)
     _check(inp, scale=0.75)
+
+
+def test_mini_shape_workload_sampled_heads(cuda_device):
+    """bf16, B=1, T=4096, H=40 (the mini model's head count), D=128: the GPU runs
+    all heads; the oracle checks three of them."""
+    _check(rda_gen.workload("mini_prefill_b1_t4096_h40_d128"), heads=[0, 21, 39])
