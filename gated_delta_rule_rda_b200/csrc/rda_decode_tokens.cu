@@ -86,19 +86,20 @@ decode_tokens_kernel(DecodeArgs a) {
         if (lane == 0) (which ? kq_s : kk_s)[i][t] = acc;
     }
 
-    // partial products of the old state with every new key and query
+    // partial products of the old state with every new key and query (paired
+    // fp32 FMAs: two value columns per instruction)
     for (int t = 0; t < T; ++t) {
-        float4 pa = make_float4(0.f, 0.f, 0.f, 0.f), pb = pa;
+        float2 pa0 = make_float2(0.f, 0.f), pa1 = pa0, pb0 = pa0, pb1 = pa0;
 #pragma unroll
         for (int r = 0; r < R; ++r) {
             const float kr = k_s[t][rg + RG * r], qr = q_s[t][rg + RG * r];
-            pa.x = fmaf(S[r].x, kr, pa.x); pa.y = fmaf(S[r].y, kr, pa.y);
-            pa.z = fmaf(S[r].z, kr, pa.z); pa.w = fmaf(S[r].w, kr, pa.w);
-            pb.x = fmaf(S[r].x, qr, pb.x); pb.y = fmaf(S[r].y, qr, pb.y);
-            pb.z = fmaf(S[r].z, qr, pb.z); pb.w = fmaf(S[r].w, qr, pb.w);
+            const float2 k2 = make_float2(kr, kr), q2 = make_float2(qr, qr);
+            const float2 s0 = make_float2(S[r].x, S[r].y), s1 = make_float2(S[r].z, S[r].w);
+            pa0 = __ffma2_rn(s0, k2, pa0); pa1 = __ffma2_rn(s1, k2, pa1);
+            pb0 = __ffma2_rn(s0, q2, pb0); pb1 = __ffma2_rn(s1, q2, pb1);
         }
-        red[(0 * T + t) * RG * TPR + rg * TPR + col4] = pa;
-        red[(1 * T + t) * RG * TPR + rg * TPR + col4] = pb;
+        red[(0 * T + t) * RG * TPR + rg * TPR + col4] = make_float4(pa0.x, pa0.y, pa1.x, pa1.y);
+        red[(1 * T + t) * RG * TPR + rg * TPR + col4] = make_float4(pb0.x, pb0.y, pb1.x, pb1.y);
     }
     __syncthreads();
 
@@ -156,16 +157,16 @@ decode_tokens_kernel(DecodeArgs a) {
 #pragma unroll
     for (int r = 0; r < R; ++r) {
         const int d = rg + RG * r;
-        float4 s = make_float4(c * S[r].x, c * S[r].y, c * S[r].z, c * S[r].w);
-#pragma unroll
+        float2 s0 = make_float2(c * S[r].x, c * S[r].y), s1 = make_float2(c * S[r].z, c * S[r].w);
 #pragma unroll
         for (int i = 0; i < kMaxT; ++i) {
             if (i >= T) break;
             const float kd = k_s[i][d];
-            s.x = fmaf(w4[i].x, kd, s.x); s.y = fmaf(w4[i].y, kd, s.y);
-            s.z = fmaf(w4[i].z, kd, s.z); s.w = fmaf(w4[i].w, kd, s.w);
+            const float2 k2 = make_float2(kd, kd);
+            s0 = __ffma2_rn(make_float2(w4[i].x, w4[i].y), k2, s0);
+            s1 = __ffma2_rn(make_float2(w4[i].z, w4[i].w), k2, s1);
         }
-        __stcs(reinterpret_cast<float4 *>(st + (size_t)d * DV) + col4, s);
+        __stcs(reinterpret_cast<float4 *>(st + (size_t)d * DV) + col4, make_float4(s0.x, s0.y, s1.x, s1.y));
     }
 }
 
