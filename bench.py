@@ -383,23 +383,27 @@ def other_workloads(device, stream, rank, world, reps=5):
                            "hbm_frac": nbytes / (ms * 1e-3) / 1e9 / load_peaks()[0]}
     del inp, ws, out, sf
 
-    # multi-token decode: the decode workload's 128 tokens as 16 calls of 8
+    # multi-token decode: the decode workload's first 128 tokens as calls of T tokens
     din = rda_gen.workload("decode_b256_h16_d128_128steps")
-    blocks = [[x[t0:t0 + 8].transpose(0, 1).contiguous().to(device)
-               for x in (din.q, din.k, din.v, din.log_alpha, din.beta)] for t0 in range(0, 128, 8)]
     st = din.state.to(device)
     Bd, H, Dk, Dv = st.shape
-    dout = torch.empty((Bd, 8, H, Dv), dtype=din.q.dtype, device=device)
+    res["decode_tokens"] = {}
+    for T in (1, 2, 4, 8):
+        blocks = [[x[t0:t0 + T].transpose(0, 1).contiguous().to(device)
+                   for x in (din.q, din.k, din.v, din.log_alpha, din.beta)] for t0 in range(0, 128, T)]
+        dout = torch.empty((Bd, T, H, Dv), dtype=din.q.dtype, device=device)
 
-    def tok_rep():
-        for q, k, v, la, be in blocks:
-            rda.rda_decode_tokens(q, k, v, la, be, st, out=dout)
-    ms = timed(tok_rep) / len(blocks)
-    bytes_call = Bd * H * (2 * state_bytes(1, Dk, Dv) + 8 * prefill_bytes_per_token_head())
-    gbs = bytes_call / (ms * 1e-3) / 1e9
-    res["decode_tokens"] = {"workload": "decode_b256_h16_d128_128steps, 8 tokens per call",
-                            "ms_per_call": ms, "tokens_per_s": world * Bd * 8 / (ms * 1e-3),
-                            "state_gbs": world * gbs, "hbm_frac": gbs / load_peaks()[0]}
+        def tok_rep():
+            for q, k, v, la, be in blocks:
+                rda.rda_decode_tokens(q, k, v, la, be, st, out=dout)
+        ms = timed(tok_rep) / len(blocks)
+        bytes_call = Bd * H * (2 * state_bytes(1, Dk, Dv) + T * prefill_bytes_per_token_head())
+        gbs = bytes_call / (ms * 1e-3) / 1e9
+        res["decode_tokens"][f"T{T}"] = {
+            "workload": f"decode_b256_h16_d128_128steps, {T} tokens per call", "ms_per_call": ms,
+            "tokens_per_s": world * Bd * T / (ms * 1e-3), "state_gbs": world * gbs,
+            "hbm_frac": gbs / load_peaks()[0]}
+        del blocks
     return res
 
 
