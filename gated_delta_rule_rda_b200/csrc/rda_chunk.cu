@@ -17,20 +17,27 @@
 //
 // which equals the token-by-token rule exactly in real arithmetic.
 //
-// Two kernels, both on the caller's stream:
+// Four kernels on the caller's stream (one of them forked onto a side stream):
 //
 //  1. prep (chunk-parallel; one CTA per (chunk, head) over every chunk of
-//     every sequence at once).  Computes everything that does not depend on
-//     the state: g, [Q;K] K^T on the tensor cores, P and A, the UT transform
-//     (diagonal 16x16 blocks by forward substitution, off-diagonal blocks by
-//     tf32 mma.sync), then W and U' on the tensor cores.  Writes W and P as
-//     ready-to-use swizzled MMA operand images, U' and g, into the caller's
-//     workspace (40.25 KiB per chunk and head at Dv = 128).
-//
+//     every sequence at once): what the state scan needs from a chunk.  g,
+//     K K^T on the tensor cores, A, the UT transform (diagonal 16x16 blocks by
+//     forward substitution, off-diagonal blocks by tf32 mma.sync), then W and
+//     U' on the tensor cores.  Writes -W as a ready-to-use swizzled operand
+//     image, U' in value slices and the decay factors.
 //  2. scan (sequential over the chunks of one (sequence, head, value slice)).
-//     Carries the fp32 state in registers; per chunk issues -W S and Q S, then
-//     K^T U~ and P U on the tensor cores and updates the state.  Value columns
-//     are independent under the rule, so slicing is exact.
+//     Carries the fp32 state in registers; per chunk U = U' - W S, then
+//     S <- e^{g_C} S + K^T diag(e^{g_C - g}) U on register-fragment MMAs.
+//     Value columns are independent under the rule, so slicing is exact.
+//     Writes the state entering each chunk and U as operand images.
+//  3. output operands (chunk-parallel): P and diag(e^g) Q.  Independent of
+//     1 and 2, so it runs on a side stream alongside them.
+//  4. outputs (chunk-parallel): O = scale [diag(e^g) Q | P] [S_c ; U], one
+//     tcgen05 accumulation chain.
+//
+// The prep is split from the output operands so that each chunk-parallel
+// kernel fits several CTAs per SM: the prep needs 72 KiB of shared memory and
+// 128 TMEM columns (three per SM), the output operands 43 KiB and 64 columns.
 //
 // Operands: bf16 in shared memory, fp32 accumulators in TMEM (tcgen05.mma),
 // Q/K/V tiles by TMA, workspace images by bulk copies.  Every wait is
@@ -92,6 +99,14 @@ __device__ __noinline__ bool wait_bar_slow(uint64_t *bar, uint32_t parity, volat
 __device__ __forceinline__ bool wait_bar(uint64_t *bar, uint32_t parity, volatile int *abort_flag, int32_t *err) {
     if (mbar_try_wait(bar, parity)) return true;
     return wait_bar_slow(bar, parity, abort_flag, err);
+}
+
+// Bounded wait that ignores the abort flag: used only to let copies or MMAs
+// already in flight land before a CTA that gave up exits.
+__device__ __noinline__ void drain_bar(uint64_t *bar, uint32_t parity) {
+    const uint64_t t0 = globaltimer();
+    while (!mbar_try_wait(bar, parity))
+        if (globaltimer() - t0 > kWaitNs) return;
 }
 
 // Byte offset of 16-byte chunk `c` of row `row` in a tile whose rows are
@@ -218,36 +233,35 @@ __device__ __forceinline__ void ut_solve(const float *Af, float *Tf, float *Xs, 
 }
 
 // ---------------------------------------------------------------------------
-// Kernel 1: prep.  One CTA per (global chunk, head).
+// Kernel 1: prep.  One CTA per (global chunk, head): everything the scan
+// needs from a chunk -- g, A from K K^T, the UT transform T, then W and U'.
 // ---------------------------------------------------------------------------
 constexpr int kPrepThreads = 192;     // warp 0 TMA, warp 1 MMA, warps 2..5 compute
-constexpr uint32_t kPrepTmemCols = 256;
+constexpr uint32_t kPrepTmemCols = 128;
 // shared memory (bytes from a 1024-aligned base)
-constexpr uint32_t PS_QK = 0;          // [Q;K]: half h at h*16384: rows 0..63 Q, 64..127 K
-constexpr uint32_t PS_V = 32768;       // V [64 x 128]: 2 halves of 8 KiB (SW128)
-constexpr uint32_t PS_P = 49152;       // P image (8 KiB)
-constexpr uint32_t PS_AF = 57344;      // A fp32 [64][kLd]
-constexpr uint32_t PS_TF = PS_AF + 64 * kLd * 4;
+constexpr uint32_t PS_K = 0;           // K [64 x 128]: halves of 8 KiB (SW128)
+constexpr uint32_t PS_V = 16384;       // V [64 x Dv]: halves of 8 KiB (SW128); later U' staging
+constexpr uint32_t PS_AF = 32768;      // A fp32 [64][kLd]; later the T images
+constexpr uint32_t PS_TF = PS_AF + 64 * kLd * 4;     // T fp32 [64][kLd]; later -W staging
 constexpr uint32_t PS_XS = PS_TF + 64 * kLd * 4;     // 4 x 16x8 fp32
 constexpr uint32_t PS_G = PS_XS + 4 * 128 * 4;       // g, beta, beta*gamma, e^{ref-g}, e^g, e^{g_C-g}: 6 x 64 fp32
 constexpr uint32_t PS_BAR = PS_G + 6 * 64 * 4;
-constexpr uint32_t PS_TMEMPTR = PS_BAR + 4 * 8;
+constexpr uint32_t PS_TMEMPTR = PS_BAR + 8 * 8;
 constexpr uint32_t PS_FLAGS = PS_TMEMPTR + 4;
 constexpr uint32_t kPrepSmem = PS_FLAGS + 4 + 1024;
-// regions reused once their first contents are consumed
-constexpr uint32_t PS_TBG = PS_QK + 0;        // over Q half 0 (Q is read only by the first MMA)
-constexpr uint32_t PS_TB = PS_QK + 16384;     // over Q half 1
-constexpr uint32_t PS_WIMG = PS_V;            // W image over V (after W and U' are done)
-constexpr uint32_t PS_UIMG = PS_AF;           // U' staging over A (after the solve)
-// TMEM columns
-constexpr uint32_t PT_QK = 0, PT_U = 0, PT_W = 128;
-enum PrepBar { PB_FULL = 0, PB_QK, PB_TREADY, PB_WU };
+constexpr uint32_t PS_TBG = PS_AF;            // T diag(beta e^g), over A (after the solve)
+constexpr uint32_t PS_TB = PS_AF + 8192;      // T diag(beta gamma)
+constexpr uint32_t PS_WIMG = PS_TF;           // -W image, over T (after the W MMA)
+constexpr uint32_t PS_UIMG = PS_V;            // U' slices, over V (after the U' MMA)
+// TMEM columns: K K^T, then W, then U' (one at a time)
+constexpr uint32_t PT_KK = 0, PT_W = 0, PT_U = 0;
+enum PrepBar { PB_FULL = 0, PB_KK, PB_TREADY, PB_W, PB_WFREE, PB_U, PB_DRAIN, kPrepBars };
 
 struct PrepMaps {
     CUtensorMap q, k, v;
 };
 
-// Which chunk a prep / output CTA handles: `idx` enumerates every chunk of
+// Which chunk a chunk-parallel CTA handles: `idx` enumerates every chunk of
 // every sequence in order.
 struct ChunkLoc {
     long t0;       // first token of the sequence
@@ -282,8 +296,65 @@ __device__ __forceinline__ bool locate_chunk(const PrefillArgs &a, long idx, Chu
     return true;
 }
 
+// Gates of one chunk, by the 128 compute threads (r = 0..127): g = cumsum of
+// log alpha (masked past the end), beta, beta*gamma and the decay factors.
+// Ends with a barrier of the compute threads.
+__device__ __forceinline__ void chunk_gates(const PrefillArgs &a, long row0, int lenc, int h, int r, int lane,
+                                            float *g_s) {
+    float *b_s = g_s + 64, *bg_s = g_s + 128, *eb_s = g_s + 192, *eg_s = g_s + 256, *ed_s = g_s + 320;
+    if (r < 64) {
+        const bool valid = r < lenc;
+        const size_t row = (size_t)(row0 + r) * a.H + h;
+        float la = valid ? a.log_alpha[row] : 0.f;
+        const float be = valid ? a.beta[row] : 0.f;
+        const float ga = (valid && a.gamma) ? a.gamma[row] : 1.f;
+#pragma unroll
+        for (int off = 1; off < 32; off <<= 1) {
+            const float y = __shfl_up_sync(0xffffffffu, la, off);
+            if (lane >= off) la += y;
+        }
+        g_s[r] = la;
+        b_s[r] = be;
+        bg_s[r] = be * ga;
+    }
+    named_bar_sync(1, 128);
+    if (r >= 32 && r < 64) g_s[r] += g_s[31];
+    named_bar_sync(1, 128);
+    if (r < 64) {
+        // e^{g_s}, and e^{ref - g_s} with ref = g at the first token of s's 16-block
+        // (g is non-increasing, so 0 <= ref - g_s <= 80 and the factor stays finite)
+        eg_s[r] = __expf(g_s[r]);
+        eb_s[r] = __expf(g_s[r & ~15] - g_s[r]);
+        ed_s[r] = __expf(g_s[63] - g_s[r]);
+    }
+    named_bar_sync(1, 128);
+}
+
+// Row t of a decayed, masked 64x64 Gram matrix from an M=64 TMEM accumulator
+// (lane quarter of this warp, this thread's row): y[s] = w * X[t][s] e^{g_t - g_s}
+// for s < t (strict) or s <= t, in pieces of 16 columns handed to `emit`.
+template <bool STRICT, typename F>
+__device__ __forceinline__ void gram_row(uint32_t taddr, int t, float w, const float *g_s, F emit) {
+    const float *eb_s = g_s + 192;
+    const float gt = g_s[t & 63];
+#pragma unroll
+    for (int b = 0; b < 4; ++b) {
+        float x[16];
+        tmem_ld16(taddr + 16 * b, x);
+        tmem_wait_ld();
+        // e^{g_t - g_s} = e^{g_t - ref(s)} e^{ref(s) - g_s}, both factors bounded
+        const float ea = (16 * b <= t) ? w * __expf(gt - g_s[16 * b]) : 0.f;
+#pragma unroll
+        for (int e = 0; e < 16; ++e) {
+            const int s = 16 * b + e;
+            x[e] = (STRICT ? s < t : s <= t) ? x[e] * ea * eb_s[s] : 0.f;
+        }
+        emit(b, x);
+    }
+}
+
 template <int NV>
-__global__ void __launch_bounds__(kPrepThreads, 2)
+__global__ void __launch_bounds__(kPrepThreads, 3)
 prep_kernel(const __grid_constant__ PrepMaps maps, const PrefillArgs a) {
     extern __shared__ uint8_t smem_raw[];
     uint8_t *sm = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -299,12 +370,11 @@ prep_kernel(const __grid_constant__ PrepMaps maps, const PrefillArgs a) {
     uint32_t *tmem_ptr = reinterpret_cast<uint32_t *>(sm + PS_TMEMPTR);
     volatile int *abort_flag = reinterpret_cast<volatile int *>(sm + PS_FLAGS);
     float *g_s = reinterpret_cast<float *>(sm + PS_G);
-    float *b_s = g_s + 64, *bg_s = g_s + 128, *eb_s = g_s + 192;
-    float *eg_s = g_s + 256, *ed_s = g_s + 320;   // stored for the scan: e^g, e^{g_C - g}
+    const float *b_s = g_s + 64, *bg_s = g_s + 128, *eg_s = g_s + 256;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
 
     if (threadIdx.x == 0) {
-        for (int i = 0; i < 4; ++i) mbar_init(&bars[i], 1);
+        for (int i = 0; i < kPrepBars; ++i) mbar_init(&bars[i], 1);
         *abort_flag = 0;
         fence_mbar_init();
     }
@@ -321,46 +391,52 @@ prep_kernel(const __grid_constant__ PrepMaps maps, const PrefillArgs a) {
     if (warp == 0) {
         if (lane == 0) {
             uint64_t *full = &bars[PB_FULL];
-            mbar_arrive_expect_tx(full, 32768 + 64 * Dv * 2);
+            mbar_arrive_expect_tx(full, 16384 + 64 * Dv * 2);
             const int r0 = (int)row0;
-            tma_load_3d(sm + PS_QK + 0, &maps.q, full, 0, h, r0);
-            tma_load_3d(sm + PS_QK + 8192, &maps.k, full, 0, h, r0);
-            tma_load_3d(sm + PS_QK + 16384, &maps.q, full, 64, h, r0);
-            tma_load_3d(sm + PS_QK + 24576, &maps.k, full, 64, h, r0);
+            tma_load_3d(sm + PS_K, &maps.k, full, 0, h, r0);
+            tma_load_3d(sm + PS_K + 8192, &maps.k, full, 64, h, r0);
             tma_load_3d(sm + PS_V, &maps.v, full, 0, h, r0);
             if (Dv == 128) tma_load_3d(sm + PS_V + 8192, &maps.v, full, 64, h, r0);
+            drain_bar(full, 0);      // the CTA may not exit with the copies in flight
         }
     } else if (warp == 1) {
         if (lane == 0) {
-            const uint32_t qk = smem_u32(sm + PS_QK), vv = smem_u32(sm + PS_V);
+            const uint32_t kk_ = smem_u32(sm + PS_K), vv = smem_u32(sm + PS_V);
             const uint32_t tbg = smem_u32(sm + PS_TBG), tb = smem_u32(sm + PS_TB);
-            constexpr uint32_t ID_QK = idesc_bf16(128, 64, 0, 0);
+            constexpr uint32_t ID_KK = idesc_bf16(64, 64, 0, 0);
             constexpr uint32_t ID_W = idesc_bf16(64, 128, 0, 1);
             const uint32_t ID_U = Dv == 128 ? idesc_bf16(64, 128, 0, 1) : idesc_bf16(64, 64, 0, 1);
             bool ok = wait_bar(&bars[PB_FULL], 0, abort_flag, a.err);
             if (ok) {
                 tc_fence_after();
 #pragma unroll
-                for (int kk = 0; kk < 8; ++kk) {
-                    const uint32_t off = (kk >> 2) * 16384 + (kk & 3) * 32;
-                    mma_bf16(tmem + PT_QK, smem_desc(qk + off, 16, 1024, kSw128),
-                             smem_desc(qk + off + 8192, 16, 1024, kSw128), ID_QK, kk > 0);
+                for (int kk = 0; kk < 8; ++kk) {     // K K^T: A = B = the K tile (K-major)
+                    const uint32_t off = (kk >> 2) * 8192 + (kk & 3) * 32;
+                    mma_bf16(tmem + PT_KK, smem_desc(kk_ + off, 16, 1024, kSw128),
+                             smem_desc(kk_ + off, 16, 1024, kSw128), ID_KK, kk > 0);
                 }
-                mma_commit(&bars[PB_QK]);
+                mma_commit(&bars[PB_KK]);
                 ok = wait_bar(&bars[PB_TREADY], 0, abort_flag, a.err);
             }
             if (ok) {
                 tc_fence_after();
 #pragma unroll
-                for (int kk = 0; kk < 4; ++kk) {
-                    // W = T diag(beta e^g) K ; U' = T diag(beta gamma) V  (B operands MN-major)
+                for (int kk = 0; kk < 4; ++kk)       // W = T diag(beta e^g) K  (B = K, MN-major)
                     mma_bf16(tmem + PT_W, smem_desc(tbg + kk * 32, 16, 1024, kSw128),
-                             smem_desc(qk + 8192 + kk * 2048, 16384, 1024, kSw128), ID_W, kk > 0);
+                             smem_desc(kk_ + kk * 2048, 8192, 1024, kSw128), ID_W, kk > 0);
+                mma_commit(&bars[PB_W]);
+                ok = wait_bar(&bars[PB_WFREE], 0, abort_flag, a.err);
+            }
+            if (ok) {
+                tc_fence_after();
+#pragma unroll
+                for (int kk = 0; kk < 4; ++kk)       // U' = T diag(beta gamma) V  (B = V, MN-major)
                     mma_bf16(tmem + PT_U, smem_desc(tb + kk * 32, 16, 1024, kSw128),
                              smem_desc(vv + kk * 2048, 8192, 1024, kSw128), ID_U, kk > 0);
-                }
-                mma_commit(&bars[PB_WU]);
+                mma_commit(&bars[PB_U]);
             }
+            mma_commit(&bars[PB_DRAIN]);      // every MMA issued has completed before TMEM is freed
+            drain_bar(&bars[PB_DRAIN], 0);
         }
     } else {
         const int cw = threadIdx.x - 64;
@@ -373,122 +449,70 @@ prep_kernel(const __grid_constant__ PrepMaps maps, const PrefillArgs a) {
         float *Tf = reinterpret_cast<float *>(sm + PS_TF);
         float *Xs = reinterpret_cast<float *>(sm + PS_XS);
 
-        // ---- gates: g = cumsum(log alpha) (masked past the end), beta, beta*gamma
-        if (r < 64) {
-            const bool valid = r < lenc;
-            const size_t row = (size_t)(row0 + r) * H + h;
-            float la = valid ? a.log_alpha[row] : 0.f;
-            const float be = valid ? a.beta[row] : 0.f;
-            const float ga = (valid && a.gamma) ? a.gamma[row] : 1.f;
-#pragma unroll
-            for (int off = 1; off < 32; off <<= 1) {
-                const float y = __shfl_up_sync(0xffffffffu, la, off);
-                if (lane >= off) la += y;
-            }
-            g_s[r] = la;
-            b_s[r] = be;
-            bg_s[r] = be * ga;
-        }
-        named_bar_sync(1, 128);
-        if (r >= 32 && r < 64) g_s[r] += g_s[31];
-        named_bar_sync(1, 128);
-        if (r < 64) {
-            // e^{g_s}, and e^{ref - g_s} with ref = g at the first token of s's 16-block
-            // (g is non-increasing, so 0 <= ref - g_s <= 80 and the factor stays finite)
-            eg_s[r] = __expf(g_s[r]);
-            eb_s[r] = __expf(g_s[r & ~15] - g_s[r]);
-            ed_s[r] = __expf(g_s[63] - g_s[r]);
-        }
-        if (cw == 0 && !wait_bar(&bars[PB_QK], 0, abort_flag, a.err)) *abort_flag = 1;
+        chunk_gates(a, row0, lenc, h, r, lane, g_s);
+        if (cw == 0 && !wait_bar(&bars[PB_KK], 0, abort_flag, a.err)) *abort_flag = 1;
         named_bar_sync(1, 128);
         if (!*abort_flag) {
             tc_fence_after();
-            float x[64];
+            // A row m: beta_m (K K^T)[m][s] e^{g_m - g_s}, s < m  (all four warps load: the
+            // TMEM load is warp-wide; lanes >= 16 hold no row and store nothing)
+            gram_row<true>(tq + PT_KK, m, b_s[m & 63], g_s, [&](int b, const float *x) {
+                if (lo) {
 #pragma unroll
-            for (int cc = 0; cc < 4; ++cc) tmem_ld16(tq + PT_QK + 16 * cc, x + 16 * cc);
-            tmem_wait_ld();
-            const int t = r & 63;
-            const float gt = g_s[t];
-            // e^{g_t - g_s} = e^{g_t - ref(s)} e^{ref(s) - g_s}, both factors bounded
-            float ea[4];
-#pragma unroll
-            for (int b = 0; b < 4; ++b) ea[b] = (16 * b <= t) ? __expf(gt - g_s[16 * b]) : 0.f;
-            if (r < 64) {
-                // P row t: (Q K^T)[t][s] e^{g_t - g_s}, s <= t  -> bf16 K-major SW128 image
-#pragma unroll
-                for (int cc = 0; cc < 8; ++cc) {
-                    float y[8];
-#pragma unroll
-                    for (int e = 0; e < 8; ++e) {
-                        const int s = 8 * cc + e;
-                        y[e] = (s <= t) ? x[s] * ea[s >> 4] * eb_s[s] : 0.f;
-                    }
-                    *reinterpret_cast<uint4 *>(sm + PS_P + swz(t, cc, 128)) = pack8(y);
+                    for (int c4 = 0; c4 < 4; ++c4)
+                        *reinterpret_cast<float4 *>(Af + m * kLd + 16 * b + 4 * c4) =
+                            make_float4(x[4 * c4], x[4 * c4 + 1], x[4 * c4 + 2], x[4 * c4 + 3]);
                 }
-            } else {
-                // A row t: beta_t (K K^T)[t][s] e^{g_t - g_s}, s < t
-                const float bt = b_s[t];
-#pragma unroll
-                for (int c4 = 0; c4 < 16; ++c4) {
-                    float y[4];
-#pragma unroll
-                    for (int e = 0; e < 4; ++e) {
-                        const int s = 4 * c4 + e;
-                        y[e] = (s < t) ? bt * x[s] * ea[s >> 4] * eb_s[s] : 0.f;
-                    }
-                    *reinterpret_cast<float4 *>(Af + t * kLd + 4 * c4) = make_float4(y[0], y[1], y[2], y[3]);
-                }
-            }
-            // diag(e^g) Q, in place over Q (Q was read only by the first MMA): row t = cw/2,
-            // 64 of its 128 columns per thread
-            {
-                const int tq2 = cw >> 1, half = cw & 1;
-                const float e = eg_s[tq2];
-                uint8_t *row = sm + PS_QK + half * 16384;
-#pragma unroll
-                for (int cc = 0; cc < 8; ++cc) {
-                    uint4 *pq = reinterpret_cast<uint4 *>(row + swz(tq2, cc, 128));
-                    uint4 u = *pq;
-                    uint32_t wv[4] = {u.x, u.y, u.z, u.w};
-#pragma unroll
-                    for (int i = 0; i < 4; ++i) {
-                        float2 f = __bfloat1622float2(*reinterpret_cast<__nv_bfloat162 *>(&wv[i]));
-                        wv[i] = pack_bf16(f.x * e, f.y * e);
-                    }
-                    *pq = make_uint4(wv[0], wv[1], wv[2], wv[3]);
-                }
-            }
+            });
+            tc_fence_before();
         }
-        fence_proxy_async_smem();
         named_bar_sync(1, 128);
         if (!*abort_flag) {
-            if (cw == 0) {
-                bulk_store(img + kImgP, sm + PS_P, 8192);
-                bulk_store(img + kImgQ, sm + PS_QK, 8192);
-                bulk_store(img + kImgQ + 8192, sm + PS_QK + 16384, 8192);
-                bulk_commit();
+            ut_solve(Af, Tf, Xs, cw);      // ends with a barrier: A is dead from here
+            // T diag(beta e^g) and T diag(beta gamma) as bf16 K-major SW128 images, over A
+            const int t = cw >> 1, half = cw & 1;
+#pragma unroll
+            for (int cc = 0; cc < 4; ++cc) {
+                const int s0 = 32 * half + 8 * cc;
+                const float4 t0 = *reinterpret_cast<const float4 *>(Tf + t * kLd + s0);
+                const float4 t1 = *reinterpret_cast<const float4 *>(Tf + t * kLd + s0 + 4);
+                const float tv[8] = {t0.x, t0.y, t0.z, t0.w, t1.x, t1.y, t1.z, t1.w};
+                float y1[8], y2[8];
+#pragma unroll
+                for (int e = 0; e < 8; ++e) {
+                    y1[e] = tv[e] * b_s[s0 + e] * eg_s[s0 + e];
+                    y2[e] = tv[e] * bg_s[s0 + e];
+                }
+                *reinterpret_cast<uint4 *>(sm + PS_TBG + swz(t, 4 * half + cc, 128)) = pack8(y1);
+                *reinterpret_cast<uint4 *>(sm + PS_TB + swz(t, 4 * half + cc, 128)) = pack8(y2);
             }
-            ut_solve(Af, Tf, Xs, cw);
-            // T diag(..) images overwrite diag(e^g) Q: its store must have read it
-            if (cw == 0) bulk_wait_reads();
-            named_bar_sync(1, 128);
-            // T diag(beta e^g) and T diag(beta gamma) as bf16 K-major SW128 images
-            {
-                const int t = cw >> 1, half = cw & 1;
+            fence_proxy_async_smem();
+        }
+        named_bar_sync(1, 128);
+        if (cw == 0 && !*abort_flag) {
+            mbar_arrive(&bars[PB_TREADY]);
+            if (!wait_bar(&bars[PB_W], 0, abort_flag, a.err)) *abort_flag = 1;
+        }
+        named_bar_sync(1, 128);
+        if (!*abort_flag) {
+            tc_fence_after();
+            // -W rows -> bf16 K-major SW128 image (2 halves of 64 columns), over T
 #pragma unroll
-                for (int cc = 0; cc < 4; ++cc) {
-                    const int s0 = 32 * half + 8 * cc;
-                    const float4 t0 = *reinterpret_cast<const float4 *>(Tf + t * kLd + s0);
-                    const float4 t1 = *reinterpret_cast<const float4 *>(Tf + t * kLd + s0 + 4);
-                    const float tv[8] = {t0.x, t0.y, t0.z, t0.w, t1.x, t1.y, t1.z, t1.w};
-                    float y1[8], y2[8];
+            for (int half = 0; half < 2; ++half) {
 #pragma unroll
-                    for (int e = 0; e < 8; ++e) {
-                        y1[e] = tv[e] * b_s[s0 + e] * eg_s[s0 + e];
-                        y2[e] = tv[e] * bg_s[s0 + e];
+                for (int p = 0; p < 2; ++p) {
+                    float x[32];
+                    tmem_ld16(tq + PT_W + 64 * half + 32 * p, x);
+                    tmem_ld16(tq + PT_W + 64 * half + 32 * p + 16, x + 16);
+                    tmem_wait_ld();
+                    if (lo) {
+#pragma unroll
+                        for (int i = 0; i < 32; ++i) x[i] = -x[i];
+#pragma unroll
+                        for (int cc = 0; cc < 4; ++cc)
+                            *reinterpret_cast<uint4 *>(sm + PS_WIMG + half * 8192 + swz(m, 4 * p + cc, 128)) =
+                                pack8(x + 8 * cc);
                     }
-                    *reinterpret_cast<uint4 *>(sm + PS_TBG + swz(t, 4 * half + cc, 128)) = pack8(y1);
-                    *reinterpret_cast<uint4 *>(sm + PS_TB + swz(t, 4 * half + cc, 128)) = pack8(y2);
                 }
             }
             fence_proxy_async_smem();
@@ -496,40 +520,30 @@ prep_kernel(const __grid_constant__ PrepMaps maps, const PrefillArgs a) {
         }
         named_bar_sync(1, 128);
         if (cw == 0 && !*abort_flag) {
-            mbar_arrive(&bars[PB_TREADY]);
-            if (!wait_bar(&bars[PB_WU], 0, abort_flag, a.err)) *abort_flag = 1;
+            mbar_arrive(&bars[PB_WFREE]);
+            bulk_store(img + kImgW, sm + PS_WIMG, 16384);
+            bulk_commit();
+            if (!wait_bar(&bars[PB_U], 0, abort_flag, a.err)) *abort_flag = 1;
         }
         named_bar_sync(1, 128);
         if (!*abort_flag) {
             tc_fence_after();
-            // -W rows -> bf16 K-major SW128 image (2 halves of 64 columns)
-#pragma unroll
-            for (int half = 0; half < 2; ++half) {
-                float x[64];
-#pragma unroll
-                for (int cc = 0; cc < 4; ++cc) tmem_ld16(tq + PT_W + 64 * half + 16 * cc, x + 16 * cc);
-                tmem_wait_ld();
-#pragma unroll
-                for (int i = 0; i < 64; ++i) x[i] = -x[i];
-                if (lo) {
-#pragma unroll
-                    for (int cc = 0; cc < 8; ++cc)
-                        *reinterpret_cast<uint4 *>(sm + PS_WIMG + half * 8192 + swz(m, cc, 128)) = pack8(x + 8 * cc);
-                }
-            }
             // U' rows -> bf16, value slices of width NV: slice s at s*64*NV*2, row m at m*NV*2
             for (int half = 0; half < Dv / 64; ++half) {
-                float x[64];
 #pragma unroll
-                for (int cc = 0; cc < 4; ++cc) tmem_ld16(tq + PT_U + 64 * half + 16 * cc, x + 16 * cc);
-                tmem_wait_ld();
-                if (lo) {
+                for (int p = 0; p < 2; ++p) {
+                    float x[32];
+                    tmem_ld16(tq + PT_U + 64 * half + 32 * p, x);
+                    tmem_ld16(tq + PT_U + 64 * half + 32 * p + 16, x + 16);
+                    tmem_wait_ld();
+                    if (lo) {
 #pragma unroll
-                    for (int cc = 0; cc < 8; ++cc) {
-                        const int col = 64 * half + 8 * cc;
-                        const int sl = col / NV, cin = col % NV;
-                        *reinterpret_cast<uint4 *>(sm + PS_UIMG + sl * (64 * NV * 2) + m * (NV * 2) + cin * 2) =
-                            pack8(x + 8 * cc);
+                        for (int cc = 0; cc < 4; ++cc) {
+                            const int col = 64 * half + 32 * p + 8 * cc;
+                            const int sl = col / NV, cin = col % NV;
+                            *reinterpret_cast<uint4 *>(sm + PS_UIMG + sl * (64 * NV * 2) + m * (NV * 2) + cin * 2) =
+                                pack8(x + 8 * cc);
+                        }
                     }
                 }
             }
@@ -538,9 +552,8 @@ prep_kernel(const __grid_constant__ PrepMaps maps, const PrefillArgs a) {
         named_bar_sync(1, 128);
         if (cw == 0) {
             if (!*abort_flag) {
-                bulk_store(img + kImgW, sm + PS_WIMG, 16384);
                 bulk_store(img + kImgU, sm + PS_UIMG, 64 * Dv * 2);
-                bulk_store(img + kImgU + 64 * Dv * 2, eg_s, 512);
+                bulk_store(img + kImgU + 64 * Dv * 2, eg_s, 512);     // e^g, e^{g_C - g}
                 bulk_commit();
             }
             bulk_wait_reads();
@@ -552,6 +565,141 @@ prep_kernel(const __grid_constant__ PrepMaps maps, const PrefillArgs a) {
     if (warp == 1) {
         tc_fence_after();
         tmem_dealloc(tmem, kPrepTmemCols);
+    }
+}
+
+// ---------------------------------------------------------------------------
+// Kernel 1b: output operands.  One CTA per (global chunk, head): P = (Q K^T) o
+// Gamma (causal, diagonal kept) and diag(e^g) Q, the chunk-local half of the
+// output product, as the output kernel's shared-memory images.
+// ---------------------------------------------------------------------------
+constexpr int kQkThreads = 192;       // warp 0 TMA, warp 1 MMA, warps 2..5 compute
+constexpr uint32_t kQkTmemCols = 64;
+constexpr uint32_t QS_Q = 0;          // Q [64 x 128]: halves of 8 KiB (SW128), scaled in place
+constexpr uint32_t QS_K = 16384;      // K [64 x 128]
+constexpr uint32_t QS_P = 32768;      // P image (8 KiB)
+constexpr uint32_t QS_G = 40960;      // gates (6 x 64 fp32)
+constexpr uint32_t QS_BAR = QS_G + 6 * 64 * 4;
+constexpr uint32_t QS_TMEMPTR = QS_BAR + 4 * 8;
+constexpr uint32_t QS_FLAGS = QS_TMEMPTR + 4;
+constexpr uint32_t kQkSmem = QS_FLAGS + 4 + 1024;
+enum QkBar { QB_FULL = 0, QB_QK, QB_DRAIN, kQkBars };
+
+__global__ void __launch_bounds__(kQkThreads, 4)
+qk_kernel(const __grid_constant__ PrepMaps maps, const PrefillArgs a) {
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t *sm = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    ChunkLoc loc;
+    if (!locate_chunk(a, blockIdx.x, loc)) return;
+    const long gc = loc.gc;
+    const int h = blockIdx.y;
+    const int H = a.H;
+    const int lenc = (int)min((long)kC, loc.len - (long)loc.c * kC);
+    const long row0 = loc.t0 + (long)loc.c * kC;
+    uint64_t *bars = reinterpret_cast<uint64_t *>(sm + QS_BAR);
+    uint32_t *tmem_ptr = reinterpret_cast<uint32_t *>(sm + QS_TMEMPTR);
+    volatile int *abort_flag = reinterpret_cast<volatile int *>(sm + QS_FLAGS);
+    float *g_s = reinterpret_cast<float *>(sm + QS_G);
+    const float *eg_s = g_s + 256;
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+
+    if (threadIdx.x == 0) {
+        for (int i = 0; i < kQkBars; ++i) mbar_init(&bars[i], 1);
+        *abort_flag = 0;
+        fence_mbar_init();
+    }
+    if (warp == 1) {
+        tmem_alloc(tmem_ptr, kQkTmemCols);
+        tmem_relinquish();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = *tmem_ptr;
+    uint8_t *img = a.workspace_chunks + ((size_t)gc * H + h) * a.chunk_bytes;
+
+    if (warp == 0) {
+        if (lane == 0) {
+            uint64_t *full = &bars[QB_FULL];
+            mbar_arrive_expect_tx(full, 32768);
+            const int r0 = (int)row0;
+            tma_load_3d(sm + QS_Q, &maps.q, full, 0, h, r0);
+            tma_load_3d(sm + QS_Q + 8192, &maps.q, full, 64, h, r0);
+            tma_load_3d(sm + QS_K, &maps.k, full, 0, h, r0);
+            tma_load_3d(sm + QS_K + 8192, &maps.k, full, 64, h, r0);
+            drain_bar(full, 0);
+        }
+    } else if (warp == 1) {
+        if (lane == 0) {
+            const uint32_t qq = smem_u32(sm + QS_Q), kk_ = smem_u32(sm + QS_K);
+            constexpr uint32_t ID_QK = idesc_bf16(64, 64, 0, 0);
+            if (wait_bar(&bars[QB_FULL], 0, abort_flag, a.err)) {
+                tc_fence_after();
+#pragma unroll
+                for (int kk = 0; kk < 8; ++kk) {
+                    const uint32_t off = (kk >> 2) * 8192 + (kk & 3) * 32;
+                    mma_bf16(tmem, smem_desc(qq + off, 16, 1024, kSw128), smem_desc(kk_ + off, 16, 1024, kSw128),
+                             ID_QK, kk > 0);
+                }
+                mma_commit(&bars[QB_QK]);
+            }
+            mma_commit(&bars[QB_DRAIN]);
+            drain_bar(&bars[QB_DRAIN], 0);
+        }
+    } else {
+        const int cw = threadIdx.x - 64;
+        const int q4 = warp & 3;
+        const int r = 32 * q4 + lane;
+        const bool lo = lane < 16;
+        const int m = 16 * q4 + lane;
+        const uint32_t tq = tmem + ((uint32_t)(32 * q4) << 16);
+        chunk_gates(a, row0, lenc, h, r, lane, g_s);
+        if (cw == 0 && !wait_bar(&bars[QB_QK], 0, abort_flag, a.err)) *abort_flag = 1;
+        named_bar_sync(1, 128);
+        if (!*abort_flag) {
+            tc_fence_after();
+            // P row m: (Q K^T)[m][s] e^{g_m - g_s}, s <= m  -> bf16 K-major SW128 image
+            gram_row<false>(tq, m, 1.f, g_s, [&](int b, const float *x) {
+                if (lo) {
+                    *reinterpret_cast<uint4 *>(sm + QS_P + swz(m, 2 * b, 128)) = pack8(x);
+                    *reinterpret_cast<uint4 *>(sm + QS_P + swz(m, 2 * b + 1, 128)) = pack8(x + 8);
+                }
+            });
+            // diag(e^g) Q in place (Q was read only by the MMA): row cw/2, 64 columns per thread
+            const int t = cw >> 1, half = cw & 1;
+            const float e = eg_s[t];
+            uint8_t *row = sm + QS_Q + half * 8192;
+#pragma unroll
+            for (int cc = 0; cc < 8; ++cc) {
+                uint4 *pq = reinterpret_cast<uint4 *>(row + swz(t, cc, 128));
+                uint4 u = *pq;
+                uint32_t wv[4] = {u.x, u.y, u.z, u.w};
+#pragma unroll
+                for (int i = 0; i < 4; ++i) {
+                    float2 f = __bfloat1622float2(*reinterpret_cast<__nv_bfloat162 *>(&wv[i]));
+                    wv[i] = pack_bf16(f.x * e, f.y * e);
+                }
+                *pq = make_uint4(wv[0], wv[1], wv[2], wv[3]);
+            }
+            tc_fence_before();
+        }
+        fence_proxy_async_smem();
+        named_bar_sync(1, 128);
+        if (cw == 0) {
+            if (!*abort_flag) {
+                bulk_store(img + kImgP, sm + QS_P, 8192);
+                bulk_store(img + kImgQ, sm + QS_Q, 16384);
+                bulk_commit();
+            }
+            bulk_wait_reads();
+        }
+    }
+
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 1) {
+        tc_fence_after();
+        tmem_dealloc(tmem, kQkTmemCols);
     }
 }
 
@@ -1062,10 +1210,43 @@ cudaError_t init_attrs() {
     static cudaError_t attr = cudaSuccess;
     std::call_once(once, [] {
         attr = set_smem(prep_kernel<NV>, kPrepSmem);
+        if (attr == cudaSuccess) attr = set_smem(qk_kernel, kQkSmem);
         if (attr == cudaSuccess) attr = set_smem(scan_kernel<NV>, ScanSmem<NV>::BYTES);
         if (attr == cudaSuccess) attr = set_smem(out_kernel, kOutSmem);
     });
     return attr;
+}
+
+// The output-operand kernel depends only on the inputs, so it runs on a side
+// stream next to the prep and the state scan (which leaves SMs and shared
+// memory idle), forked from and joined back to the caller's stream with
+// events.  One side stream and event pair per device, created on first use;
+// a mutex keeps the record / wait pairs of concurrent callers apart.
+struct SideStream {
+    cudaStream_t stream = nullptr;
+    cudaEvent_t fork = nullptr, join = nullptr;
+    bool ready = false;
+};
+std::mutex g_side_mu;
+SideStream g_side[64];
+
+cudaError_t side_stream(SideStream **out) {
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return e;
+    if (dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
+    SideStream &ss = g_side[dev];
+    if (!ss.ready) {
+        int least = 0, greatest = 0;
+        if ((e = cudaDeviceGetStreamPriorityRange(&least, &greatest)) != cudaSuccess) return e;
+        if (!ss.stream && (e = cudaStreamCreateWithPriority(&ss.stream, cudaStreamNonBlocking, least)) != cudaSuccess)
+            return e;
+        if (!ss.fork && (e = cudaEventCreateWithFlags(&ss.fork, cudaEventDisableTiming)) != cudaSuccess) return e;
+        if (!ss.join && (e = cudaEventCreateWithFlags(&ss.join, cudaEventDisableTiming)) != cudaSuccess) return e;
+        ss.ready = true;
+    }
+    *out = &ss;
+    return cudaSuccess;
 }
 
 template <int NV>
@@ -1084,14 +1265,26 @@ cudaError_t launch_nv(const PrefillArgs &a, long chunks_grid, cudaStream_t s) {
     }
     const dim3 scan_grid(a.Dv / NV, a.H, a.num_seqs);
     const uint32_t scan_smem = ScanSmem<NV>::BYTES;
+    const dim3 chunk_grid((unsigned)chunks_grid, a.H, 1);
 
+    std::lock_guard<std::mutex> lk(g_side_mu);
+    SideStream *ss = nullptr;
     if (chunks_grid > 0) {
-        prep_kernel<NV><<<dim3((unsigned)chunks_grid, a.H, 1), kPrepThreads, kPrepSmem, s>>>(pm, a);
+        if ((e = side_stream(&ss)) != cudaSuccess) return e;
+        // fork: the output operands wait for everything already on the caller's stream
+        // (a previous call's output kernel may still read the same workspace)
+        if ((e = cudaEventRecord(ss->fork, s)) != cudaSuccess) return e;
+        if ((e = cudaStreamWaitEvent(ss->stream, ss->fork, 0)) != cudaSuccess) return e;
+        qk_kernel<<<chunk_grid, kQkThreads, kQkSmem, ss->stream>>>(pm, a);
+        if ((e = cudaGetLastError()) != cudaSuccess) return e;
+        if ((e = cudaEventRecord(ss->join, ss->stream)) != cudaSuccess) return e;
+        prep_kernel<NV><<<chunk_grid, kPrepThreads, kPrepSmem, s>>>(pm, a);
         if ((e = cudaGetLastError()) != cudaSuccess) return e;
     }
     scan_kernel<NV><<<scan_grid, kScanThreads, scan_smem, s>>>(sm, a);
     if ((e = cudaGetLastError()) != cudaSuccess || chunks_grid == 0) return e;
-    out_kernel<<<dim3((unsigned)chunks_grid, a.H, 1), kOutThreads, kOutSmem, s>>>(a);
+    if ((e = cudaStreamWaitEvent(s, ss->join, 0)) != cudaSuccess) return e;      // join
+    out_kernel<<<chunk_grid, kOutThreads, kOutSmem, s>>>(a);
     return cudaGetLastError();
 }
 
