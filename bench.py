@@ -6,7 +6,8 @@ Dk=Dv=128, 64-token chunks, nonzero fp32 initial state, final state returned)
 with its inputs resident in HBM; L2 is flushed (a 256 MiB write) between
 timed steps and each step is timed alone with CUDA events on the launching
 stream.  ``e2e`` times the same call with host (pinned) inputs and outputs,
-copies included.  ``decode`` times 128 consecutive decode steps over
+copies included, as a two-slot pipeline (one step's copies overlap the next
+step's compute and copies; every step moves all of its own bytes).  ``decode`` times 128 consecutive decode steps over
 B=256 sequences (state 256 MiB, larger than L2).
 
 Multi-GPU (torchrun): the path does not shard within one problem; every rank
@@ -29,6 +30,9 @@ sys.path.insert(0, ROOT)
 
 METRIC = "RDA prefill tokens/s (H=16,D=128) and decode state GB/s on 1 B200 vs roofline"
 WORKLOAD = "nano_prefill_b1_t4096_h16_d128"
+# kernels one fixed-length bf16 prefill call enqueues (prep, output operands,
+# state scan, outputs)
+LAUNCHES_PER_PREFILL = 4
 CHUNK = 64
 
 
@@ -197,33 +201,53 @@ def run_ours(args, rank, world, device):
         ms_per_step = float(t.item())
     assert rda.rda_read_device_error(ws) == 0, "device error word set during the benchmark"
 
-    # ---- e2e: host (pinned) inputs and outputs, copies inside the timed region
+    # ---- e2e: host (pinned) inputs and outputs, copies inside the timed region.
+    # Two pipeline slots on two streams, each with its own device buffers and
+    # workspace: step i copies its inputs in, runs the prefill and copies the
+    # output and final state back on slot i % 2, so one step's copies overlap
+    # the neighbouring step's (PCIe is full duplex).  Every step still moves all
+    # of its own bytes both ways.
     host_in = [t.pin_memory() for t in (inp.q, inp.k, inp.v, inp.log_alpha, inp.beta, inp.initial_state)]
-    dev_in = [torch.empty_like(t, device=device) for t in host_in]
-    host_out = torch.empty((B, T, H, Dv), dtype=inp.q.dtype).pin_memory()
-    host_sf = torch.empty((B, H, Dk, Dv), dtype=torch.float32).pin_memory()
     h2d = sum(t.numel() * t.element_size() for t in host_in)
-    d2h = host_out.numel() * host_out.element_size() + host_sf.numel() * host_sf.element_size()
+    slots = []
+    for _ in range(2):
+        slots.append({
+            "stream": torch.cuda.Stream(device),
+            "dev_in": [torch.empty_like(t, device=device) for t in host_in],
+            "out": torch.empty((B, T, H, Dv), dtype=inp.q.dtype, device=device),
+            "sf": torch.empty((B, H, Dk, Dv), dtype=torch.float32, device=device),
+            "ws": ws if not slots else rda.new_workspace(ws.numel(), device),
+            "host_out": torch.empty((B, T, H, Dv), dtype=inp.q.dtype).pin_memory(),
+            "host_sf": torch.empty((B, H, Dk, Dv), dtype=torch.float32).pin_memory(),
+        })
+    d2h = (slots[0]["host_out"].numel() * slots[0]["host_out"].element_size() +
+           slots[0]["host_sf"].numel() * slots[0]["host_sf"].element_size())
 
-    def e2e_step():
-        for hd, dd in zip(host_in, dev_in):
-            dd.copy_(hd, non_blocking=True)
-        q, k, v, la, be, s0 = dev_in
-        rda.rda_prefill_chunked(q, k, v, la, be, initial_state=s0, out=out, final_state=sf,
-                                workspace=ws)
-        host_out.copy_(out, non_blocking=True)
-        host_sf.copy_(sf, non_blocking=True)
+    def e2e_step(i):
+        sl = slots[i % 2]
+        with torch.cuda.stream(sl["stream"]):
+            for hd, dd in zip(host_in, sl["dev_in"]):
+                dd.copy_(hd, non_blocking=True)
+            q, k, v, la, be, s0 = sl["dev_in"]
+            rda.rda_prefill_chunked(q, k, v, la, be, initial_state=s0, out=sl["out"], final_state=sl["sf"],
+                                    workspace=sl["ws"])
+            sl["host_out"].copy_(sl["out"], non_blocking=True)
+            sl["host_sf"].copy_(sl["sf"], non_blocking=True)
 
-    e2e_steps = max(3, min(args.steps, 50))
-    for _ in range(3):
-        e2e_step()
+    e2e_steps = max(4, min(args.steps, 50))
+    for i in range(4):
+        e2e_step(i)
     torch.cuda.synchronize()
     if dist:
         dist.barrier()
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     e0.record(stream)
-    for _ in range(e2e_steps):
-        e2e_step()
+    for sl in slots:
+        sl["stream"].wait_event(e0)
+    for i in range(e2e_steps):
+        e2e_step(i)
+    for sl in slots:
+        stream.wait_stream(sl["stream"])
     e1.record(stream)
     torch.cuda.synchronize()
     e2e_ms = e0.elapsed_time(e1) / e2e_steps
@@ -231,6 +255,10 @@ def run_ours(args, rank, world, device):
         t = torch.tensor([e2e_ms], device=device)
         dist.all_reduce(t, op=dist.ReduceOp.MAX)
         e2e_ms = float(t.item())
+    # the pipelined result must match the device-resident run
+    assert torch.equal(slots[0]["host_out"], out.cpu()) and torch.equal(slots[1]["host_sf"], sf.cpu()), \
+        "end-to-end result differs from the device-resident step"
+    del slots
 
     # ---- decode: 128 consecutive steps over B=256 (state larger than L2)
     dec = None
@@ -308,8 +336,9 @@ def run_ours(args, rank, world, device):
                      "tensor": {"achieved_tflops": tflops, "peak_tflops": tf,
                                 "frac": tflops / tf, "algorithmic_flops_per_launch": alg_flops}},
         "e2e": {"value": tokens * world / (e2e_ms * 1e-3), "unit": "tokens/s",
-                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms},
-        "gpu_launches": args.steps,
+                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms,
+                "pipeline": "2 slots on 2 streams: copies of one step overlap the next step's"},
+        "gpu_launches": args.steps * LAUNCHES_PER_PREFILL,
         "clocks": clocks,
         "decode": dec,
         **extra,
