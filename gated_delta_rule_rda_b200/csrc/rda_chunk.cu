@@ -31,7 +31,8 @@
 //     Value columns are independent under the rule, so slicing is exact.
 //     Writes the state entering each chunk and U as operand images.
 //  3. output operands (chunk-parallel): P and diag(e^g) Q.  Independent of
-//     1 and 2, so it runs on a side stream alongside them.
+//     1 and 2, so it runs on a side stream alongside the prep (short scans) or
+//     alongside the scan (long ones).
 //  4. outputs (chunk-parallel): O = scale [diag(e^g) Q | P] [S_c ; U], one
 //     tcgen05 accumulation chain.
 //
@@ -1217,6 +1218,8 @@ cudaError_t init_attrs() {
     return attr;
 }
 
+constexpr long kSMs = 148;
+
 // The output-operand kernel depends only on the inputs, so it runs on a side
 // stream next to the prep and the state scan (which leaves SMs and shared
 // memory idle), forked from and joined back to the caller's stream with
@@ -1267,19 +1270,32 @@ cudaError_t launch_nv(const PrefillArgs &a, long chunks_grid, cudaStream_t s) {
     const uint32_t scan_smem = ScanSmem<NV>::BYTES;
     const dim3 chunk_grid((unsigned)chunks_grid, a.H, 1);
 
+    // Where to fork the output operands: next to the prep when the scan is short
+    // (they would outlast it), else after the prep, next to the scan alone (the
+    // scan is latency-bound and leaves room; the prep is not).  The scan's length
+    // in chunk steps: waves of its CTAs times the chunks of an average sequence.
+    const long scan_ctas = (long)scan_grid.x * scan_grid.y * scan_grid.z;
+    const long seq_chunks = (chunks_grid + a.num_seqs - 1) / (a.num_seqs > 0 ? a.num_seqs : 1);
+    const bool fork_after_prep = (scan_ctas + kSMs - 1) / kSMs * seq_chunks >= 128;
+
     std::lock_guard<std::mutex> lk(g_side_mu);
     SideStream *ss = nullptr;
+    auto fork_qk = [&]() -> cudaError_t {
+        // the output operands wait for everything already on the caller's stream
+        // (a previous call's output kernel may still read the same workspace)
+        cudaError_t r;
+        if ((r = cudaEventRecord(ss->fork, s)) != cudaSuccess) return r;
+        if ((r = cudaStreamWaitEvent(ss->stream, ss->fork, 0)) != cudaSuccess) return r;
+        qk_kernel<<<chunk_grid, kQkThreads, kQkSmem, ss->stream>>>(pm, a);
+        if ((r = cudaGetLastError()) != cudaSuccess) return r;
+        return cudaEventRecord(ss->join, ss->stream);
+    };
     if (chunks_grid > 0) {
         if ((e = side_stream(&ss)) != cudaSuccess) return e;
-        // fork: the output operands wait for everything already on the caller's stream
-        // (a previous call's output kernel may still read the same workspace)
-        if ((e = cudaEventRecord(ss->fork, s)) != cudaSuccess) return e;
-        if ((e = cudaStreamWaitEvent(ss->stream, ss->fork, 0)) != cudaSuccess) return e;
-        qk_kernel<<<chunk_grid, kQkThreads, kQkSmem, ss->stream>>>(pm, a);
-        if ((e = cudaGetLastError()) != cudaSuccess) return e;
-        if ((e = cudaEventRecord(ss->join, ss->stream)) != cudaSuccess) return e;
+        if (!fork_after_prep && (e = fork_qk()) != cudaSuccess) return e;
         prep_kernel<NV><<<chunk_grid, kPrepThreads, kPrepSmem, s>>>(pm, a);
         if ((e = cudaGetLastError()) != cudaSuccess) return e;
+        if (fork_after_prep && (e = fork_qk()) != cudaSuccess) return e;
     }
     scan_kernel<NV><<<scan_grid, kScanThreads, scan_smem, s>>>(sm, a);
     if ((e = cudaGetLastError()) != cudaSuccess || chunks_grid == 0) return e;
