@@ -146,12 +146,15 @@ __device__ __forceinline__ void mma_tf32(float *d, const uint32_t *a, const uint
         : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b[0]), "r"(b[1]));
 }
 
-// T = (I + A)^{-1}, A strictly lower triangular 64x64 (fp32, stride kLd),
-// by 16x16 blocks: diagonal blocks by forward substitution (fp32), then
-//   T_ij = -T_ii * (sum_{m=j}^{i-1} A_im T_mj),  level by level in i - j,
-// each product on the tensor cores (tf32 mma.sync, fp32 accumulate).
+// T = (I + A)^{-1}, A strictly lower triangular 64x64 (fp32, stride kLd), by
+// 16x16 blocks.  Diagonal blocks by forward substitution (fp32); then, by
+// recursive doubling on [[X, 0], [Y, Z]]^-1 = [[X^-1, 0], [-Z^-1 Y X^-1, Z^-1]]:
+//   the 16x16 blocks T_10 and T_32 (inside each 32-row half), then the 32x32
+//   block T[32:64, 0:32] = -T[32:64, 32:64] A[32:64, 0:32] T[0:32, 0:32],
+// each product on the tensor cores (tf32 mma.sync, fp32 accumulate).  The
+// unused upper-right 32x32 block of A holds the intermediate product.
 // Called by the 128 threads of one warpgroup (cw = 0..127).
-__device__ __forceinline__ void ut_solve(const float *Af, float *Tf, float *Xs, int cw) {
+__device__ __forceinline__ void ut_solve(float *Af, float *Tf, float *Xs, int cw) {
     const int wq = cw >> 5, lane = cw & 31;
     if (cw < 64) {
         const int b = cw >> 4, j = cw & 15;
@@ -181,56 +184,108 @@ __device__ __forceinline__ void ut_solve(const float *Af, float *Tf, float *Xs, 
     }
     named_bar_sync(1, 128);
     const int g = lane >> 2, tg = lane & 3;
-    float *xs = Xs + wq * 128;   // per-warp 16x8 scratch
-#pragma unroll 1
-    for (int L = 1; L <= 3; ++L) {
-        const int units = 2 * (4 - L);
-#pragma unroll 1
-        for (int u = wq; u < units; u += 4) {
-            const int j = u >> 1, nt = u & 1, i = j + L;
-            // X (16x8) = A[16i.., 16j .. 16i) * T[16j .. 16i, 16j + 8nt ..]
-            float x[4] = {0.f, 0.f, 0.f, 0.f};
-#pragma unroll 1
-            for (int k0 = 16 * j; k0 < 16 * i; k0 += 8) {
-                uint32_t a[4], bb[2];
-                const float *ar = Af + (16 * i + g) * kLd + k0 + tg;
-                a[0] = f2tf32(ar[0]);
-                a[1] = f2tf32(ar[8 * kLd]);
-                a[2] = f2tf32(ar[4]);
-                a[3] = f2tf32(ar[8 * kLd + 4]);
-                const float *br = Tf + (k0 + tg) * kLd + 16 * j + 8 * nt + g;
-                bb[0] = f2tf32(br[0]);
-                bb[1] = f2tf32(br[4 * kLd]);
-                mma_tf32(x, a, bb);
-            }
-            xs[g * 8 + 2 * tg] = x[0];
-            xs[g * 8 + 2 * tg + 1] = x[1];
-            xs[(g + 8) * 8 + 2 * tg] = x[2];
-            xs[(g + 8) * 8 + 2 * tg + 1] = x[3];
-            __syncwarp();
-            // Z = T_ii X ; T_ij = -Z
-            float z[4] = {0.f, 0.f, 0.f, 0.f};
+    // a tf32 A fragment (16x8) at (r0, k0) and B fragment (8x8) at (k0, c0) of
+    // row-major fp32 matrices with stride kLd
+    auto frag_a = [&](const float *m, int r0, int k0, uint32_t *a) {
+        const float *ar = m + (r0 + g) * kLd + k0 + tg;
+        a[0] = f2tf32(ar[0]);
+        a[1] = f2tf32(ar[8 * kLd]);
+        a[2] = f2tf32(ar[4]);
+        a[3] = f2tf32(ar[8 * kLd + 4]);
+    };
+    auto frag_b = [&](const float *m, int k0, int c0, uint32_t *b) {
+        const float *br = m + (k0 + tg) * kLd + c0 + g;
+        b[0] = f2tf32(br[0]);
+        b[1] = f2tf32(br[4 * kLd]);
+    };
+    {
+        // T_{j+1,j}, j = 0 (warps 0, 1) or 2 (warps 2, 3), 8 columns per warp:
+        // X = A_{j+1,j} T_jj, then -T_{j+1,j+1} X
+        const int j = 2 * (wq >> 1), i = j + 1, c0 = 16 * j + 8 * (wq & 1);
+        float *xs = Xs + wq * 128;       // per-warp 16x8 scratch
+        float x[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
-            for (int ks = 0; ks < 2; ++ks) {
-                uint32_t a[4], bb[2];
-                const float *ar = Tf + (16 * i + g) * kLd + 16 * i + 8 * ks + tg;
-                a[0] = f2tf32(ar[0]);
-                a[1] = f2tf32(ar[8 * kLd]);
-                a[2] = f2tf32(ar[4]);
-                a[3] = f2tf32(ar[8 * kLd + 4]);
-                bb[0] = f2tf32(xs[(8 * ks + tg) * 8 + g]);
-                bb[1] = f2tf32(xs[(8 * ks + tg + 4) * 8 + g]);
-                mma_tf32(z, a, bb);
-            }
-            float *tr = Tf + (16 * i + g) * kLd + 16 * j + 8 * nt + 2 * tg;
-            tr[0] = -z[0];
-            tr[1] = -z[1];
-            tr[8 * kLd] = -z[2];
-            tr[8 * kLd + 1] = -z[3];
-            __syncwarp();
+        for (int k0 = 16 * j; k0 < 16 * i; k0 += 8) {
+            uint32_t a[4], b[2];
+            frag_a(Af, 16 * i, k0, a);
+            frag_b(Tf, k0, c0, b);
+            mma_tf32(x, a, b);
         }
-        named_bar_sync(1, 128);
+        xs[g * 8 + 2 * tg] = x[0];
+        xs[g * 8 + 2 * tg + 1] = x[1];
+        xs[(g + 8) * 8 + 2 * tg] = x[2];
+        xs[(g + 8) * 8 + 2 * tg + 1] = x[3];
+        __syncwarp();
+        float z[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+        for (int ks = 0; ks < 2; ++ks) {
+            uint32_t a[4], b[2];
+            frag_a(Tf, 16 * i, 16 * i + 8 * ks, a);
+            b[0] = f2tf32(xs[(8 * ks + tg) * 8 + g]);
+            b[1] = f2tf32(xs[(8 * ks + tg + 4) * 8 + g]);
+            mma_tf32(z, a, b);
+        }
+        float *tr = Tf + (16 * i + g) * kLd + c0 + 2 * tg;
+        tr[0] = -z[0];
+        tr[1] = -z[1];
+        tr[8 * kLd] = -z[2];
+        tr[8 * kLd + 1] = -z[3];
     }
+    named_bar_sync(1, 128);
+    // each warp one 16x16 quadrant (rows r0, columns c0) of the 32x32 products
+    const int r0 = 16 * (wq >> 1), c0 = 16 * (wq & 1);
+    {
+        // Y = A[32:64, 0:32] T[0:32, 0:32] -> A[0:32, 32:64]  (T lower triangular:
+        // rows above c0 contribute nothing to columns from c0)
+        float y[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
+#pragma unroll
+        for (int k0 = 0; k0 < 32; k0 += 8) {
+            if (k0 < c0) continue;
+            uint32_t a[4];
+            frag_a(Af, 32 + r0, k0, a);
+#pragma unroll
+            for (int nt = 0; nt < 2; ++nt) {
+                uint32_t b[2];
+                frag_b(Tf, k0, c0 + 8 * nt, b);
+                mma_tf32(y[nt], a, b);
+            }
+        }
+#pragma unroll
+        for (int nt = 0; nt < 2; ++nt) {
+            float *yr = Af + (r0 + g) * kLd + 32 + c0 + 8 * nt + 2 * tg;
+            yr[0] = y[nt][0];
+            yr[1] = y[nt][1];
+            yr[8 * kLd] = y[nt][2];
+            yr[8 * kLd + 1] = y[nt][3];
+        }
+    }
+    named_bar_sync(1, 128);
+    {
+        // T[32:64, 0:32] = -T[32:64, 32:64] Y  (T lower triangular: columns past
+        // the quadrant's last row contribute nothing)
+        float z[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
+#pragma unroll
+        for (int k0 = 0; k0 < 32; k0 += 8) {
+            if (k0 >= r0 + 16) continue;
+            uint32_t a[4];
+            frag_a(Tf, 32 + r0, 32 + k0, a);
+#pragma unroll
+            for (int nt = 0; nt < 2; ++nt) {
+                uint32_t b[2];
+                frag_b(Af, k0, 32 + c0 + 8 * nt, b);
+                mma_tf32(z[nt], a, b);
+            }
+        }
+#pragma unroll
+        for (int nt = 0; nt < 2; ++nt) {
+            float *tr = Tf + (32 + r0 + g) * kLd + c0 + 8 * nt + 2 * tg;
+            tr[0] = -z[nt][0];
+            tr[1] = -z[nt][1];
+            tr[8 * kLd] = -z[nt][2];
+            tr[8 * kLd + 1] = -z[nt][3];
+        }
+    }
+    named_bar_sync(1, 128);
 }
 
 // ---------------------------------------------------------------------------
