@@ -415,6 +415,9 @@ prep_kernel(const __grid_constant__ PrepMaps maps, const PrefillArgs a) {
     extern __shared__ uint8_t smem_raw[];
     uint8_t *sm = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     ChunkLoc loc;
+    // the scan may be scheduled once every prep CTA has started (it waits for
+    // this grid's completion before reading anything the prep writes)
+    if (threadIdx.x == 0) pdl_launch_dependents();
     if (!locate_chunk(a, blockIdx.x, loc)) return;     // uniform across the CTA
     const long gc = loc.gc;
     const int h = blockIdx.y;
@@ -911,6 +914,7 @@ scan_kernel(const __grid_constant__ ScanMaps maps, const PrefillArgs a) {
     if (warp == kScanWarps) {
         // ------------------------------------------------------------ producer
         if (lane == 0) {
+            pdl_wait_primary();      // the prep's images are complete and visible
             for (int c = 0; c < nchunks; ++c) {
                 const int st = c % kScanStages;
                 if (c >= kScanStages &&
@@ -1352,7 +1356,23 @@ cudaError_t launch_nv(const PrefillArgs &a, long chunks_grid, cudaStream_t s) {
         if ((e = cudaGetLastError()) != cudaSuccess) return e;
         if (fork_after_prep && (e = fork_qk()) != cudaSuccess) return e;
     }
-    scan_kernel<NV><<<scan_grid, kScanThreads, scan_smem, s>>>(sm, a);
+    {
+        // programmatic stream serialization: the scan's launch and prologue overlap
+        // the prep's last CTAs; its producer waits for the prep before loading
+        cudaLaunchConfig_t cfg = {};
+        cfg.gridDim = scan_grid;
+        cfg.blockDim = dim3(kScanThreads);
+        cfg.dynamicSmemBytes = scan_smem;
+        cfg.stream = s;
+        cudaLaunchAttribute attr[1];
+        attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+        // (not when the output operands fork after the prep: they would queue
+        // behind scan CTAs that sit waiting for the prep; measured slower)
+        attr[0].val.programmaticStreamSerializationAllowed = chunks_grid > 0 && !fork_after_prep ? 1 : 0;
+        cfg.attrs = attr;
+        cfg.numAttrs = 1;
+        if ((e = cudaLaunchKernelEx(&cfg, scan_kernel<NV>, sm, a)) != cudaSuccess) return e;
+    }
     if ((e = cudaGetLastError()) != cudaSuccess || chunks_grid == 0) return e;
     if ((e = cudaStreamWaitEvent(s, ss->join, 0)) != cudaSuccess) return e;      // join
     out_kernel<<<chunk_grid, kOutThreads, kOutSmem, s>>>(a);
