@@ -67,11 +67,7 @@ constexpr uint64_t kWaitNs = 4000000000ull;   // bounded waits: 4 s
 constexpr uint32_t kImgW = 0;          // -W, bf16 K-major SW128, 2 halves of 8 KiB (64 rows x 64 cols)
 constexpr uint32_t kImgQ = 16384;      // diag(e^g) Q, same layout
 constexpr uint32_t kImgP = 32768;      // P, bf16 K-major SW128, 8 KiB
-constexpr uint32_t kImgS = 40960;      // state entering the chunk, bf16 MN-major SW128:
-                                       // atoms of 64 value columns, [128 key rows x 128 B] each
-constexpr uint32_t kImgV = 73728;      // U = U' - W S_c, bf16 MN-major SW128: atoms of 64 value
-                                       // columns, [64 token rows x 128 B] each (written by the scan)
-constexpr uint32_t kImgU = 90112;      // U', bf16, value slices of width NV, each [64][NV];
+constexpr uint32_t kImgU = 40960;      // U', bf16, value slices of width NV, each [64][NV];
                                        // then e^{g_t} and e^{g_C - g_t}: 2 x 64 fp32
 
 __device__ __forceinline__ uint64_t globaltimer() {
@@ -415,9 +411,6 @@ prep_kernel(const __grid_constant__ PrepMaps maps, const PrefillArgs a) {
     extern __shared__ uint8_t smem_raw[];
     uint8_t *sm = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     ChunkLoc loc;
-    // the scan may be scheduled once every prep CTA has started (it waits for
-    // this grid's completion before reading anything the prep writes)
-    if (threadIdx.x == 0) pdl_launch_dependents();
     if (!locate_chunk(a, blockIdx.x, loc)) return;     // uniform across the CTA
     const long gc = loc.gc;
     const int h = blockIdx.y;
@@ -782,17 +775,18 @@ qk_kernel(const __grid_constant__ PrepMaps maps, const PrefillArgs a) {
 // ---------------------------------------------------------------------------
 constexpr int kScanWarps = 4;
 constexpr int kScanThreads = (kScanWarps + 1) * 32;
-constexpr int kScanStages = 4;
+constexpr int kScanStages = 3;
 // per-stage shared memory (bytes): -W 16K | K 16K | U' <= 4K | decay 512
-constexpr uint32_t SS_W = 0, SS_K = 16384, SS_U = 32768, SS_G = 36864;
-constexpr uint32_t SS_STAGE = 37888;                          // multiple of 1024
+constexpr uint32_t SS_W = 0, SS_K = 16384, SS_Q = 32768, SS_P = 49152, SS_U = 57344, SS_G = 61440;
+constexpr uint32_t SS_STAGE = 62464;                          // multiple of 1024
 enum ScanBar { SB_FULL = 0, SB_EMPTY = kScanStages, kScanBars = 2 * kScanStages };
 // then: state [128][RS] bf16, U~ [64][RS], barriers, flags (RS = 2 NV + 16)
 template <int NV> struct ScanSmem {
     static constexpr uint32_t RS = NV * 2 + 16;
     static constexpr uint32_t SS = kScanStages * SS_STAGE;
     static constexpr uint32_t UT = SS + 128 * RS;
-    static constexpr uint32_t BAR = UT + 64 * RS;
+    static constexpr uint32_t UU = UT + 64 * RS;       // U (unscaled), the B operand of P U
+    static constexpr uint32_t BAR = UU + 64 * RS;
     static constexpr uint32_t FLAGS = BAR + kScanBars * 8;
     static constexpr uint32_t BYTES = FLAGS + 16 + 1024;
 };
@@ -858,11 +852,6 @@ __device__ __forceinline__ void ld_b(uint32_t base, int k0, int n0, int lane, ui
         for (int i = 0; i < NW / 16; ++i) ldsm_x4_t(b_addr_rm(base, k0, n0 + 16 * i, lane, rs), bf + 4 * i);
     }
 }
-// Byte offset of value column j of row `row` in an MN-major SW128 image whose
-// 64-column atoms have `atom_bytes` (rows of 128 B).
-__device__ __forceinline__ uint32_t mn_off(int row, int j, uint32_t atom_bytes) {
-    return (j >> 6) * atom_bytes + swz(row, (j & 63) >> 3, 128) + (j & 7) * 2;
-}
 
 template <int NV>
 __global__ void __launch_bounds__(kScanThreads, 1)
@@ -914,7 +903,6 @@ scan_kernel(const __grid_constant__ ScanMaps maps, const PrefillArgs a) {
     if (warp == kScanWarps) {
         // ------------------------------------------------------------ producer
         if (lane == 0) {
-            pdl_wait_primary();      // the prep's images are complete and visible
             for (int c = 0; c < nchunks; ++c) {
                 const int st = c % kScanStages;
                 if (c >= kScanStages &&
@@ -923,11 +911,13 @@ scan_kernel(const __grid_constant__ ScanMaps maps, const PrefillArgs a) {
                 uint64_t *full = &bars[SB_FULL + st];
                 uint8_t *stg = sm + st * SS_STAGE;
                 const uint8_t *img = a.workspace_chunks + ((size_t)(gc0 + c) * H + h) * a.chunk_bytes;
-                mbar_arrive_expect_tx(full, 16384 * 2 + UBYTES + 512);
+                mbar_arrive_expect_tx(full, 16384 * 3 + 8192 + UBYTES + 512);
                 const int r0 = (int)(t0 + (long)c * kC);
                 tma_load_3d(stg + SS_K, &maps.k, full, 0, h, r0);
                 tma_load_3d(stg + SS_K + 8192, &maps.k, full, 64, h, r0);
                 bulk_load(stg + SS_W, img + kImgW, 16384, full);
+                bulk_load(stg + SS_Q, img + kImgQ, 16384, full);
+                bulk_load(stg + SS_P, img + kImgP, 8192, full);
                 bulk_load(stg + SS_U, img + kImgU + (size_t)slice * UBYTES, UBYTES, full);
                 bulk_load(stg + SS_G, img + kImgU + 64 * Dv * 2, 512, full);
             }
@@ -961,9 +951,7 @@ scan_kernel(const __grid_constant__ ScanMaps maps, const PrefillArgs a) {
         const uint32_t stg = smb + st * SS_STAGE;
         const float *eg_s = reinterpret_cast<const float *>(sm + st * SS_STAGE + SS_G);
         const float *ed_s = eg_s + 64;
-        uint8_t *cimg = a.workspace_chunks + ((size_t)(gc0 + c) * H + h) * a.chunk_bytes;
-        // ---- S -> bf16: row-major [d][j] in shared memory (the B operand
-        //      below) and the MN-major image the output kernel reads
+        // ---- S -> bf16: row-major [d][j] in shared memory (the B operand below)
 #pragma unroll
         for (int mt = 0; mt < 2; ++mt)
 #pragma unroll
@@ -973,7 +961,6 @@ scan_kernel(const __grid_constant__ ScanMaps maps, const PrefillArgs a) {
                     const int d = 32 * rg + 16 * mt + g + 8 * hh, j = c0 + 8 * nt + 2 * tg;
                     const uint32_t v = pack_bf16(S[mt][nt][2 * hh], S[mt][nt][2 * hh + 1]);
                     *reinterpret_cast<uint32_t *>(sm + SC_SS + d * RS + j * 2) = v;
-                    *reinterpret_cast<uint32_t *>(cimg + kImgS + mn_off(d, j0 + j, 16384)) = v;
                 }
         if (tid == 0 && !wait_bar(&bars[SB_FULL + st], (c / kScanStages) & 1, abort_flag, a.err)) *abort_flag = 1;
         named_bar_sync(1, NCW);
@@ -990,32 +977,40 @@ scan_kernel(const __grid_constant__ ScanMaps maps, const PrefillArgs a) {
             acc[0][nt][0] = fa.x; acc[0][nt][1] = fa.y; acc[0][nt][2] = fb.x; acc[0][nt][3] = fb.y;
             acc[1][nt][0] = acc[1][nt][1] = acc[1][nt][2] = acc[1][nt][3] = 0.f;
         }
+        // O = diag(e^g) Q S_c (+ P U below) for the same rows: it shares the state
+        // operand fragments with U
+        float ao[NT][4];
+#pragma unroll
+        for (int nt = 0; nt < NT; ++nt) ao[nt][0] = ao[nt][1] = ao[nt][2] = ao[nt][3] = 0.f;
         // operands of a group of k-steps are loaded before its MMAs are issued, so
         // the shared-memory latency is paid once per group
-        constexpr int KGU = NW >= 32 ? 4 : 8;
+        constexpr int KGU = NW >= 32 ? 2 : 4;
 #pragma unroll
         for (int k0 = 0; k0 < 8; k0 += KGU) {
-            uint32_t af[KGU][4], bf[KGU][NW / 4 > 4 ? NW / 4 : 4];
+            uint32_t af[KGU][4], aq[KGU][4], bf[KGU][NW / 4 > 4 ? NW / 4 : 4];
 #pragma unroll
             for (int kk = 0; kk < KGU; ++kk) {
                 ldsm_x4(a_addr_sw128(stg + SS_W, 16 * rg, 16 * (k0 + kk), lane, 8192), af[kk]);
                 ld_b<NW>(ssb, 16 * (k0 + kk), c0, lane, RS, bf[kk]);
+                ldsm_x4(a_addr_sw128(stg + SS_Q, 16 * rg, 16 * (k0 + kk), lane, 8192), aq[kk]);
             }
 #pragma unroll
             for (int kk = 0; kk < KGU; ++kk)
 #pragma unroll
-                for (int nt = 0; nt < NT; ++nt)
+                for (int nt = 0; nt < NT; ++nt) {
                     mma16816(acc[kk & 1][nt], af[kk], bf[kk][2 * nt], bf[kk][2 * nt + 1]);
+                    mma16816(ao[nt], aq[kk], bf[kk][2 * nt], bf[kk][2 * nt + 1]);
+                }
         }
-        // ---- U -> image for the output kernel; U~ = e^{g_C - g_t} U -> shared memory
+        // ---- U and U~ = e^{g_C - g_t} U -> shared memory (B operands of P U and K^T U~)
         const float da = ed_s[ta], db = ed_s[tb];
 #pragma unroll
         for (int nt = 0; nt < NT; ++nt) {
             const int j = c0 + 8 * nt + 2 * tg;
             const float u0 = acc[0][nt][0] + acc[1][nt][0], u1 = acc[0][nt][1] + acc[1][nt][1];
             const float u2 = acc[0][nt][2] + acc[1][nt][2], u3 = acc[0][nt][3] + acc[1][nt][3];
-            *reinterpret_cast<uint32_t *>(cimg + kImgV + mn_off(ta, j0 + j, 8192)) = pack_bf16(u0, u1);
-            *reinterpret_cast<uint32_t *>(cimg + kImgV + mn_off(tb, j0 + j, 8192)) = pack_bf16(u2, u3);
+            *reinterpret_cast<uint32_t *>(sm + L::UU + ta * RS + j * 2) = pack_bf16(u0, u1);
+            *reinterpret_cast<uint32_t *>(sm + L::UU + tb * RS + j * 2) = pack_bf16(u2, u3);
             *reinterpret_cast<uint32_t *>(sm + SC_UT + ta * RS + j * 2) = pack_bf16(u0 * da, u1 * da);
             *reinterpret_cast<uint32_t *>(sm + SC_UT + tb * RS + j * 2) = pack_bf16(u2 * db, u3 * db);
         }
@@ -1056,7 +1051,32 @@ scan_kernel(const __grid_constant__ ScanMaps maps, const PrefillArgs a) {
 #pragma unroll
                 for (int i = 0; i < 4; ++i)
                     S[mt][nt][i] = fmaf(eC, S[mt][nt][i], ds[0][mt][nt][i] + ds[1][mt][nt][i]);
+        // ---- O += P U for rows t = 16rg .. 16rg+15, then the store (masked tail)
+        {
+            const uint32_t uub = smb + L::UU;
+#pragma unroll
+            for (int kk = 0; kk < 4; ++kk) {
+                uint32_t ap[4], bu[NW / 4 > 4 ? NW / 4 : 4];
+                ldsm_x4(a_addr_sw128(stg + SS_P, 16 * rg, 16 * kk, lane, 8192), ap);
+                ld_b<NW>(uub, 16 * kk, c0, lane, RS, bu);
+#pragma unroll
+                for (int nt = 0; nt < NT; ++nt) mma16816(ao[nt], ap, bu[2 * nt], bu[2 * nt + 1]);
+            }
+        }
         mbar_arrive(&bars[SB_EMPTY + st]);
+        {
+            const int lenc = (int)min((long)kC, len - (long)c * kC);
+            __nv_bfloat16 *ob = static_cast<__nv_bfloat16 *>(a.out) + ((size_t)(t0 + (long)c * kC) * H + h) * Dv + j0;
+            const float sc = a.scale;
+#pragma unroll
+            for (int nt = 0; nt < NT; ++nt) {
+                const int j = c0 + 8 * nt + 2 * tg;
+                if (ta < lenc)
+                    *reinterpret_cast<uint32_t *>(ob + (size_t)ta * H * Dv + j) = pack_bf16(sc * ao[nt][0], sc * ao[nt][1]);
+                if (tb < lenc)
+                    *reinterpret_cast<uint32_t *>(ob + (size_t)tb * H * Dv + j) = pack_bf16(sc * ao[nt][2], sc * ao[nt][3]);
+            }
+        }
         // No barrier here: the next chunk writes the state buffer after every
         // warp passed this chunk's second barrier (its reads of the state are
         // done), and U~ after the next first barrier (every warp is past this
@@ -1073,115 +1093,6 @@ scan_kernel(const __grid_constant__ ScanMaps maps, const PrefillArgs a) {
                     *reinterpret_cast<float2 *>(s_out + sb + (size_t)d * Dv + j) =
                         make_float2(S[mt][nt][2 * hh], S[mt][nt][2 * hh + 1]);
                 }
-    }
-}
-
-// ---------------------------------------------------------------------------
-// Kernel 3: outputs.  One CTA per (global chunk, head), all value columns:
-//     O = scale [diag(e^g) Q | P] [S_c ; U]        (M = 64, N = Dv, K = 192)
-// one tcgen05 accumulation chain of 12 instructions over images the prep and
-// scan kernels left in the workspace.
-// ---------------------------------------------------------------------------
-constexpr int kOutThreads = 192;      // warp 0 loads, warp 1 MMA, warps 2..5 epilogue
-constexpr uint32_t kOutTmemCols = 128;
-constexpr uint32_t OS_Q = 0;          // diag(e^g) Q: 2 halves of 8 KiB (K-major SW128)
-constexpr uint32_t OS_P = 16384;      // P (8 KiB)
-constexpr uint32_t OS_S = 24576;      // S_c: Dv/64 atoms of 16 KiB (MN-major SW128)
-constexpr uint32_t OS_V = 57344;      // U:   Dv/64 atoms of 8 KiB  (MN-major SW128)
-constexpr uint32_t OS_BAR = 73728;
-constexpr uint32_t OS_TMEMPTR = OS_BAR + 2 * 8;
-constexpr uint32_t OS_FLAGS = OS_TMEMPTR + 4;
-constexpr uint32_t kOutSmem = OS_FLAGS + 4 + 1024;
-enum OutBar { OB_FULL = 0, OB_DONE };
-
-__global__ void __launch_bounds__(kOutThreads, 3)
-out_kernel(const PrefillArgs a) {
-    extern __shared__ uint8_t smem_raw[];
-    uint8_t *sm = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-    ChunkLoc loc;
-    if (!locate_chunk(a, blockIdx.x, loc)) return;
-    const long gc = loc.gc;
-    const int h = blockIdx.y;
-    const int H = a.H, Dv = a.Dv;
-    const int lenc = (int)min((long)kC, loc.len - (long)loc.c * kC);
-    const long row0 = loc.t0 + (long)loc.c * kC;
-    uint64_t *bars = reinterpret_cast<uint64_t *>(sm + OS_BAR);
-    uint32_t *tmem_ptr = reinterpret_cast<uint32_t *>(sm + OS_TMEMPTR);
-    volatile int *abort_flag = reinterpret_cast<volatile int *>(sm + OS_FLAGS);
-    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const uint8_t *img = a.workspace_chunks + ((size_t)gc * H + h) * a.chunk_bytes;
-
-    if (threadIdx.x == 0) {
-        for (int i = 0; i < 2; ++i) mbar_init(&bars[i], 1);
-        *abort_flag = 0;
-        fence_mbar_init();
-    }
-    if (warp == 1) {
-        tmem_alloc(tmem_ptr, kOutTmemCols);
-        tmem_relinquish();
-    }
-    tc_fence_before();
-    __syncthreads();
-    tc_fence_after();
-    const uint32_t tmem = *tmem_ptr;
-
-    if (warp == 0) {
-        if (lane == 0) {
-            uint64_t *full = &bars[OB_FULL];
-            const uint32_t atoms = (uint32_t)(Dv / 64);
-            mbar_arrive_expect_tx(full, 16384 + 8192 + atoms * (16384 + 8192));
-            bulk_load(sm + OS_Q, img + kImgQ, 16384, full);
-            bulk_load(sm + OS_P, img + kImgP, 8192, full);
-            bulk_load(sm + OS_S, img + kImgS, atoms * 16384, full);
-            bulk_load(sm + OS_V, img + kImgV, atoms * 8192, full);
-        }
-    } else if (warp == 1) {
-        if (lane == 0) {
-            const uint32_t qq = smem_u32(sm + OS_Q), pp = smem_u32(sm + OS_P);
-            const uint32_t ss = smem_u32(sm + OS_S), vv = smem_u32(sm + OS_V);
-            const uint32_t id = Dv == 128 ? idesc_bf16(64, 128, 0, 1) : idesc_bf16(64, 64, 0, 1);
-            if (wait_bar(&bars[OB_FULL], 0, abort_flag, a.err)) {
-                tc_fence_after();
-#pragma unroll
-                for (int kk = 0; kk < 8; ++kk)
-                    mma_bf16(tmem, smem_desc(qq + (kk >> 2) * 8192 + (kk & 3) * 32, 16, 1024, kSw128),
-                             smem_desc(ss + kk * 2048, 16384, 1024, kSw128), id, kk > 0);
-#pragma unroll
-                for (int kk = 0; kk < 4; ++kk)
-                    mma_bf16(tmem, smem_desc(pp + kk * 32, 16, 1024, kSw128),
-                             smem_desc(vv + kk * 2048, 8192, 1024, kSw128), id, 1);
-                mma_commit(&bars[OB_DONE]);
-            }
-        }
-    } else {
-        const int cw = threadIdx.x - 64;
-        const int q4 = warp & 3;
-        const uint32_t tq = tmem + ((uint32_t)(32 * q4) << 16);
-        const int t = 16 * q4 + lane;            // accumulator row (M = 64 layout), lanes < 16
-        if (cw == 0 && !wait_bar(&bars[OB_DONE], 0, abort_flag, a.err)) *abort_flag = 1;
-        named_bar_sync(1, 128);
-        if (!*abort_flag) {
-            tc_fence_after();
-            __nv_bfloat16 *orow = static_cast<__nv_bfloat16 *>(a.out) + ((size_t)(row0 + t) * H + h) * Dv;
-            for (int j16 = 0; j16 < Dv; j16 += 16) {
-                float x[16];
-                tmem_ld16(tq + j16, x);
-                tmem_wait_ld();
-                if (lane < 16 && t < lenc) {
-#pragma unroll
-                    for (int e = 0; e < 16; ++e) x[e] *= a.scale;
-                    *reinterpret_cast<uint4 *>(orow + j16) = pack8(x);
-                    *reinterpret_cast<uint4 *>(orow + j16 + 8) = pack8(x + 8);
-                }
-            }
-        }
-    }
-
-    tc_fence_before();
-    __syncthreads();
-    if (warp == 1) {
-        tc_fence_after();
-        tmem_dealloc(tmem, kOutTmemCols);
     }
 }
 
@@ -1272,12 +1183,9 @@ cudaError_t init_attrs() {
         attr = set_smem(prep_kernel<NV>, kPrepSmem);
         if (attr == cudaSuccess) attr = set_smem(qk_kernel, kQkSmem);
         if (attr == cudaSuccess) attr = set_smem(scan_kernel<NV>, ScanSmem<NV>::BYTES);
-        if (attr == cudaSuccess) attr = set_smem(out_kernel, kOutSmem);
     });
     return attr;
 }
-
-constexpr long kSMs = 148;
 
 // The output-operand kernel depends only on the inputs, so it runs on a side
 // stream next to the prep and the state scan (which leaves SMs and shared
@@ -1329,53 +1237,23 @@ cudaError_t launch_nv(const PrefillArgs &a, long chunks_grid, cudaStream_t s) {
     const uint32_t scan_smem = ScanSmem<NV>::BYTES;
     const dim3 chunk_grid((unsigned)chunks_grid, a.H, 1);
 
-    // Where to fork the output operands: next to the prep when the scan is short
-    // (they would outlast it), else after the prep, next to the scan alone (the
-    // scan is latency-bound and leaves room; the prep is not).  The scan's length
-    // in chunk steps: waves of its CTAs times the chunks of an average sequence.
-    const long scan_ctas = (long)scan_grid.x * scan_grid.y * scan_grid.z;
-    const long seq_chunks = (chunks_grid + a.num_seqs - 1) / (a.num_seqs > 0 ? a.num_seqs : 1);
-    const bool fork_after_prep = (scan_ctas + kSMs - 1) / kSMs * seq_chunks >= 128;
-
     std::lock_guard<std::mutex> lk(g_side_mu);
     SideStream *ss = nullptr;
-    auto fork_qk = [&]() -> cudaError_t {
-        // the output operands wait for everything already on the caller's stream
-        // (a previous call's output kernel may still read the same workspace)
-        cudaError_t r;
-        if ((r = cudaEventRecord(ss->fork, s)) != cudaSuccess) return r;
-        if ((r = cudaStreamWaitEvent(ss->stream, ss->fork, 0)) != cudaSuccess) return r;
-        qk_kernel<<<chunk_grid, kQkThreads, kQkSmem, ss->stream>>>(pm, a);
-        if ((r = cudaGetLastError()) != cudaSuccess) return r;
-        return cudaEventRecord(ss->join, ss->stream);
-    };
     if (chunks_grid > 0) {
         if ((e = side_stream(&ss)) != cudaSuccess) return e;
-        if (!fork_after_prep && (e = fork_qk()) != cudaSuccess) return e;
+        // fork: the output operands wait for everything already on the caller's
+        // stream (a previous call's scan may still read the same workspace) and
+        // run beside the prep; the scan waits for both
+        if ((e = cudaEventRecord(ss->fork, s)) != cudaSuccess) return e;
+        if ((e = cudaStreamWaitEvent(ss->stream, ss->fork, 0)) != cudaSuccess) return e;
+        qk_kernel<<<chunk_grid, kQkThreads, kQkSmem, ss->stream>>>(pm, a);
+        if ((e = cudaGetLastError()) != cudaSuccess) return e;
+        if ((e = cudaEventRecord(ss->join, ss->stream)) != cudaSuccess) return e;
         prep_kernel<NV><<<chunk_grid, kPrepThreads, kPrepSmem, s>>>(pm, a);
         if ((e = cudaGetLastError()) != cudaSuccess) return e;
-        if (fork_after_prep && (e = fork_qk()) != cudaSuccess) return e;
+        if ((e = cudaStreamWaitEvent(s, ss->join, 0)) != cudaSuccess) return e;      // join
     }
-    {
-        // programmatic stream serialization: the scan's launch and prologue overlap
-        // the prep's last CTAs; its producer waits for the prep before loading
-        cudaLaunchConfig_t cfg = {};
-        cfg.gridDim = scan_grid;
-        cfg.blockDim = dim3(kScanThreads);
-        cfg.dynamicSmemBytes = scan_smem;
-        cfg.stream = s;
-        cudaLaunchAttribute attr[1];
-        attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
-        // (not when the output operands fork after the prep: they would queue
-        // behind scan CTAs that sit waiting for the prep; measured slower)
-        attr[0].val.programmaticStreamSerializationAllowed = chunks_grid > 0 && !fork_after_prep ? 1 : 0;
-        cfg.attrs = attr;
-        cfg.numAttrs = 1;
-        if ((e = cudaLaunchKernelEx(&cfg, scan_kernel<NV>, sm, a)) != cudaSuccess) return e;
-    }
-    if ((e = cudaGetLastError()) != cudaSuccess || chunks_grid == 0) return e;
-    if ((e = cudaStreamWaitEvent(s, ss->join, 0)) != cudaSuccess) return e;      // join
-    out_kernel<<<chunk_grid, kOutThreads, kOutSmem, s>>>(a);
+    scan_kernel<NV><<<scan_grid, kScanThreads, scan_smem, s>>>(sm, a);
     return cudaGetLastError();
 }
 

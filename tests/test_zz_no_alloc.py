@@ -48,7 +48,7 @@ def test_noalloc_matches_workspace_entry_point_twice(cuda_device):
 
 def test_noalloc_rejects_sizes_beyond_its_array(cuda_device):
     import gated_delta_rule_rda_b200 as rda
-    big = rda_gen.fixed_inputs(1, 4096, 16, 128, 128, dtype=torch.bfloat16, seed=63, s0=False).to("cuda")
+    big = rda_gen.fixed_inputs(1, 8192, 16, 128, 128, dtype=torch.bfloat16, seed=63, s0=False).to("cuda")
     out = torch.empty_like(big.v)
     sf = torch.empty(1, 16, 128, 128, device="cuda")
     assert _noalloc(rda.lib, big, 1.0, out, sf) == 4          # RDA_ERR_WORKSPACE, nothing launched
