@@ -17,24 +17,24 @@
 //
 // which equals the token-by-token rule exactly in real arithmetic.
 //
-// Four kernels on the caller's stream (one of them forked onto a side stream):
+// Three kernels on the caller's stream (one of them forked onto a side stream):
 //
 //  1. prep (chunk-parallel; one CTA per (chunk, head) over every chunk of
-//     every sequence at once): what the state scan needs from a chunk.  g,
+//     every sequence at once): what the state chain needs from a chunk.  g,
 //     K K^T on the tensor cores, A, the UT transform (diagonal 16x16 blocks by
-//     forward substitution, off-diagonal blocks by tf32 mma.sync), then W and
-//     U' on the tensor cores.  Writes -W as a ready-to-use swizzled operand
-//     image, U' in value slices and the decay factors.
-//  2. scan (sequential over the chunks of one (sequence, head, value slice)).
-//     Carries the fp32 state in registers; per chunk U = U' - W S, then
-//     S <- e^{g_C} S + K^T diag(e^{g_C - g}) U on register-fragment MMAs.
-//     Value columns are independent under the rule, so slicing is exact.
-//     Writes the state entering each chunk and U as operand images.
-//  3. output operands (chunk-parallel): P and diag(e^g) Q.  Independent of
-//     1 and 2, so it runs on a side stream alongside the prep (short scans) or
-//     alongside the scan (long ones).
-//  4. outputs (chunk-parallel): O = scale [diag(e^g) Q | P] [S_c ; U], one
-//     tcgen05 accumulation chain.
+//     forward substitution, off-diagonal blocks by recursive doubling on tf32
+//     mma.sync), then W and U' on the tensor cores.  Writes -W as a
+//     ready-to-use swizzled operand image, U' in value slices and the decay
+//     factors.
+//  2. output operands (chunk-parallel): P and diag(e^g) Q, the chunk-local
+//     operands of the outputs.  Independent of the prep, so it runs on a side
+//     stream beside it; the scan waits for both.
+//  3. scan (sequential over the chunks of one (sequence, head, value slice)).
+//     Carries the fp32 state in registers; per chunk U = U' - W S and the
+//     outputs O = scale (diag(e^g) Q S + P U) -- the two products with S share
+//     its operand fragments -- then S <- e^{g_C} S + K^T diag(e^{g_C - g}) U, on
+//     register-fragment MMAs.  Value columns are independent under the rule,
+//     so slicing is exact.
 //
 // The prep is split from the output operands so that each chunk-parallel
 // kernel fits several CTAs per SM: the prep needs 72 KiB of shared memory and
@@ -622,8 +622,8 @@ prep_kernel(const __grid_constant__ PrepMaps maps, const PrefillArgs a) {
 
 // ---------------------------------------------------------------------------
 // Kernel 1b: output operands.  One CTA per (global chunk, head): P = (Q K^T) o
-// Gamma (causal, diagonal kept) and diag(e^g) Q, the chunk-local half of the
-// output product, as the output kernel's shared-memory images.
+// Gamma (causal, diagonal kept) and diag(e^g) Q, the chunk-local operands of
+// the outputs, as the scan's shared-memory images.
 // ---------------------------------------------------------------------------
 constexpr int kQkThreads = 192;       // warp 0 TMA, warp 1 MMA, warps 2..5 compute
 constexpr uint32_t kQkTmemCols = 64;
@@ -763,24 +763,25 @@ qk_kernel(const __grid_constant__ PrepMaps maps, const PrefillArgs a) {
 // 64xNV).  On tcgen05 each such instruction costs about 90 cycles of pipe
 // time whatever its size, plus a commit round trip, so this latency-bound
 // chain runs on register-fragment tensor-core MMAs (mma.sync m16n8k16, bf16
-// in, fp32 accumulate) with ldmatrix operands.  The outputs are left to the
-// output kernel, which reads the state entering each chunk and U from the
-// workspace.
+// in, fp32 accumulate) with ldmatrix operands.  The outputs of the chunk's
+// rows come out of the same pass: diag(e^g) Q S with the operand fragments of
+// S that U uses, and P U once U is in shared memory.
 //   warps 0..3  warp w owns key rows 32w..32w+31 of the fp32 state (as
-//               accumulator fragments) across the slice's NV value columns;
-//               (splitting the columns over twice the warps doubles the
-//               operand traffic through shared memory and measured slower)
-//   warp 4      producer: the K tile by TMA, -W, U' and the decay factors by
-//               bulk copies, into a 4-stage ring.
+//               accumulator fragments) and token rows 16w..16w+15 of U and O,
+//               across the slice's NV value columns (splitting the columns
+//               over twice the warps doubles the operand traffic through
+//               shared memory and measured slower)
+//   warp 4      producer: the K tile by TMA, -W, diag(e^g) Q, P, U' and the
+//               decay factors by bulk copies, into a 3-stage ring.
 // ---------------------------------------------------------------------------
 constexpr int kScanWarps = 4;
 constexpr int kScanThreads = (kScanWarps + 1) * 32;
 constexpr int kScanStages = 3;
-// per-stage shared memory (bytes): -W 16K | K 16K | U' <= 4K | decay 512
+// per-stage shared memory (bytes): -W 16K | K 16K | diag(e^g) Q 16K | P 8K | U' <= 4K | decay 512
 constexpr uint32_t SS_W = 0, SS_K = 16384, SS_Q = 32768, SS_P = 49152, SS_U = 57344, SS_G = 61440;
 constexpr uint32_t SS_STAGE = 62464;                          // multiple of 1024
 enum ScanBar { SB_FULL = 0, SB_EMPTY = kScanStages, kScanBars = 2 * kScanStages };
-// then: state [128][RS] bf16, U~ [64][RS], barriers, flags (RS = 2 NV + 16)
+// then: state [128][RS] bf16, U~ [64][RS], U [64][RS], barriers, flags (RS = 2 NV + 16)
 template <int NV> struct ScanSmem {
     static constexpr uint32_t RS = NV * 2 + 16;
     static constexpr uint32_t SS = kScanStages * SS_STAGE;
