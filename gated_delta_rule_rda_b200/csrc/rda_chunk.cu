@@ -78,24 +78,32 @@ __device__ __forceinline__ uint64_t globaltimer() {
 
 // Bounded mbarrier wait.  try_wait suspends the thread in hardware until the
 // phase completes or a short limit passes; the loop adds the overall bound.
-__device__ __noinline__ bool wait_bar_slow(uint64_t *bar, uint32_t parity, volatile int *abort_flag,
+// Gives up when `stop` or `mine` is set, and sets `mine` when the bound runs
+// out.  Threads that branch around named barriers on a flag pass it as both;
+// a single-thread agent (TMA / MMA issue) passes its own `mine`, so that it
+// never changes a flag such threads read.
+__device__ __noinline__ bool wait_bar_slow(uint64_t *bar, uint32_t parity, volatile int *stop, volatile int *mine,
                                            int32_t *err) {
     const uint64_t t0 = globaltimer();
     for (uint32_t i = 0;; ++i) {
         if (mbar_try_wait(bar, parity)) return true;
         if ((i & 63) == 63) {
-            if (*abort_flag) return false;
+            if (*stop || *mine) return false;
             if (globaltimer() - t0 > kWaitNs) {
-                *abort_flag = 1;
+                *mine = 1;
                 atomicCAS(err, 0, (int32_t)RDA_ERR_TIMEOUT);
                 return false;
             }
         }
     }
 }
-__device__ __forceinline__ bool wait_bar(uint64_t *bar, uint32_t parity, volatile int *abort_flag, int32_t *err) {
+__device__ __forceinline__ bool wait_bar2(uint64_t *bar, uint32_t parity, volatile int *stop, volatile int *mine,
+                                          int32_t *err) {
     if (mbar_try_wait(bar, parity)) return true;
-    return wait_bar_slow(bar, parity, abort_flag, err);
+    return wait_bar_slow(bar, parity, stop, mine, err);
+}
+__device__ __forceinline__ bool wait_bar(uint64_t *bar, uint32_t parity, volatile int *flag, int32_t *err) {
+    return wait_bar2(bar, parity, flag, flag, err);
 }
 
 // Bounded wait that ignores the abort flag: used only to let copies or MMAs
@@ -287,27 +295,33 @@ __device__ __forceinline__ void ut_solve(float *Af, float *Tf, float *Xs, int cw
 // ---------------------------------------------------------------------------
 // Kernel 1: prep.  One CTA per (global chunk, head): everything the scan
 // needs from a chunk -- g, A from K K^T, the UT transform T, then W and U'.
+// Four CTAs share an SM (shared memory <= 55 KiB, 128 TMEM columns, <= 96
+// registers): three regions are reused as the chunk's work moves along.
 // ---------------------------------------------------------------------------
-constexpr int kPrepThreads = 192;     // warp 0 TMA, warp 1 MMA, warps 2..5 compute
+constexpr int kPrepThreads = 160;     // warp 0 TMA + MMA issue, warps 1..4 compute
 constexpr uint32_t kPrepTmemCols = 128;
 // shared memory (bytes from a 1024-aligned base)
-constexpr uint32_t PS_K = 0;           // K [64 x 128]: halves of 8 KiB (SW128)
-constexpr uint32_t PS_V = 16384;       // V [64 x Dv]: halves of 8 KiB (SW128); later U' staging
-constexpr uint32_t PS_AF = 32768;      // A fp32 [64][kLd]; later the T images
-constexpr uint32_t PS_TF = PS_AF + 64 * kLd * 4;     // T fp32 [64][kLd]; later -W staging
+constexpr uint32_t PS_K = 0;           // K [64 x 128]: halves of 8 KiB (SW128); later the -W image
+constexpr uint32_t PS_AF = 16384;      // A fp32 [64][kLd]; after the solve V [64 x Dv] (halves
+                                       // of 8 KiB, SW128), after the U' MMA the U' slices
+constexpr uint32_t PS_TF = PS_AF + 64 * kLd * 4;     // T fp32 [64][kLd]; later the two T images
 constexpr uint32_t PS_XS = PS_TF + 64 * kLd * 4;     // 4 x 16x8 fp32
 constexpr uint32_t PS_G = PS_XS + 4 * 128 * 4;       // g, beta, beta*gamma, e^{ref-g}, e^g, e^{g_C-g}: 6 x 64 fp32
 constexpr uint32_t PS_BAR = PS_G + 6 * 64 * 4;
 constexpr uint32_t PS_TMEMPTR = PS_BAR + 8 * 8;
 constexpr uint32_t PS_FLAGS = PS_TMEMPTR + 4;
-constexpr uint32_t kPrepSmem = PS_FLAGS + 4 + 1024;
-constexpr uint32_t PS_TBG = PS_AF;            // T diag(beta e^g), over A (after the solve)
-constexpr uint32_t PS_TB = PS_AF + 8192;      // T diag(beta gamma)
-constexpr uint32_t PS_WIMG = PS_TF;           // -W image, over T (after the W MMA)
+constexpr uint32_t kPrepSmem = PS_FLAGS + 8 + 1024;   // flags: compute threads', TMA / MMA thread's
+constexpr uint32_t PS_V = PS_AF;              // V, over A (loaded after the solve)
+constexpr uint32_t PS_TBG = PS_TF;            // T diag(beta e^g), over T
+constexpr uint32_t PS_TB = PS_TF + 8192;      // T diag(beta gamma)
+constexpr uint32_t PS_WIMG = PS_K;            // -W image, over K (after the W MMA)
 constexpr uint32_t PS_UIMG = PS_V;            // U' slices, over V (after the U' MMA)
+static_assert(PS_AF % 1024 == 0 && PS_TF % 1024 == 0, "SW128 tiles need 1024-byte alignment");
+static_assert(4 * (kPrepSmem + 1024) <= 233472, "four prep CTAs per SM");
 // TMEM columns: K K^T, then W, then U' (one at a time)
 constexpr uint32_t PT_KK = 0, PT_W = 0, PT_U = 0;
-enum PrepBar { PB_FULL = 0, PB_KK, PB_TREADY, PB_W, PB_WFREE, PB_U, PB_DRAIN, kPrepBars };
+enum PrepBar { PB_FULL = 0, PB_VFULL, PB_KK, PB_TREADY, PB_W, PB_WFREE, PB_U, PB_DRAIN, kPrepBars };
+static_assert(kPrepBars <= 8, "barrier area");
 
 struct PrepMaps {
     CUtensorMap q, k, v;
@@ -382,31 +396,43 @@ __device__ __forceinline__ void chunk_gates(const PrefillArgs &a, long row0, int
     named_bar_sync(1, 128);
 }
 
-// Row t of a decayed, masked 64x64 Gram matrix from an M=64 TMEM accumulator
-// (lane quarter of this warp, this thread's row): y[s] = w * X[t][s] e^{g_t - g_s}
-// for s < t (strict) or s <= t, in pieces of 16 columns handed to `emit`.
-template <bool STRICT, typename F>
-__device__ __forceinline__ void gram_row(uint32_t taddr, int t, float w, const float *g_s, F emit) {
+// Two rows of a decayed, masked 64x64 Gram matrix from an M=64 TMEM accumulator
+// (taddr at the warp's lane quarter), read with 16x256b loads so that all 32
+// lanes hold data: thread l gets rows ta = 16 q + l/4 and ta + 8, and of each
+// 8-column block kb the columns s = 8 kb + 2 (l%4) and s + 1, in
+// v[4 kb .. 4 kb + 3] = (ta, s), (ta, s+1), (ta+8, s), (ta+8, s+1).
+// On return v holds y = w_t X[t][s] e^{g_t - g_s} for s < t (strict) or s <= t,
+// else 0; w_t = w_s[t], or 1 without w_s.
+template <bool STRICT>
+__device__ __forceinline__ void gram_rows(uint32_t taddr, int ta, int lane, const float *w_s, const float *g_s,
+                                          float (&v)[32]) {
     const float *eb_s = g_s + 192;
-    const float gt = g_s[t & 63];
+    tmem_ld_16x256b_x4(taddr, v);
+    tmem_ld_16x256b_x4(taddr + 32, v + 16);
+    tmem_wait_ld();
+    const int j2 = 2 * (lane & 3);
 #pragma unroll
-    for (int b = 0; b < 4; ++b) {
-        float x[16];
-        tmem_ld16(taddr + 16 * b, x);
-        tmem_wait_ld();
-        // e^{g_t - g_s} = e^{g_t - ref(s)} e^{ref(s) - g_s}, both factors bounded
-        const float ea = (16 * b <= t) ? w * __expf(gt - g_s[16 * b]) : 0.f;
+    for (int rr = 0; rr < 2; ++rr) {
+        const int t = ta + 8 * rr;
+        const float gt = g_s[t];
+        const float w = w_s ? w_s[t] : 1.f;
+        float ea[4];       // e^{g_t - g_s} = e^{g_t - ref(s)} e^{ref(s) - g_s}, both factors bounded
 #pragma unroll
-        for (int e = 0; e < 16; ++e) {
-            const int s = 16 * b + e;
-            x[e] = (STRICT ? s < t : s <= t) ? x[e] * ea * eb_s[s] : 0.f;
+        for (int b = 0; b < 4; ++b) ea[b] = (16 * b <= t) ? w * __expf(gt - g_s[16 * b]) : 0.f;
+#pragma unroll
+        for (int kb = 0; kb < 8; ++kb) {
+#pragma unroll
+            for (int e = 0; e < 2; ++e) {
+                const int s = 8 * kb + j2 + e;
+                float &x = v[4 * kb + 2 * rr + e];
+                x = (STRICT ? s < t : s <= t) ? x * ea[kb >> 1] * eb_s[s] : 0.f;
+            }
         }
-        emit(b, x);
     }
 }
 
 template <int NV>
-__global__ void __launch_bounds__(kPrepThreads, 3)
+__global__ void __launch_bounds__(kPrepThreads, 4)
 prep_kernel(const __grid_constant__ PrepMaps maps, const PrefillArgs a) {
     extern __shared__ uint8_t smem_raw[];
     uint8_t *sm = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -421,6 +447,7 @@ prep_kernel(const __grid_constant__ PrepMaps maps, const PrefillArgs a) {
     uint64_t *bars = reinterpret_cast<uint64_t *>(sm + PS_BAR);
     uint32_t *tmem_ptr = reinterpret_cast<uint32_t *>(sm + PS_TMEMPTR);
     volatile int *abort_flag = reinterpret_cast<volatile int *>(sm + PS_FLAGS);
+    volatile int *agent_flag = abort_flag + 1;
     float *g_s = reinterpret_cast<float *>(sm + PS_G);
     const float *b_s = g_s + 64, *bg_s = g_s + 128, *eg_s = g_s + 256;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -428,9 +455,10 @@ prep_kernel(const __grid_constant__ PrepMaps maps, const PrefillArgs a) {
     if (threadIdx.x == 0) {
         for (int i = 0; i < kPrepBars; ++i) mbar_init(&bars[i], 1);
         *abort_flag = 0;
+        *agent_flag = 0;
         fence_mbar_init();
     }
-    if (warp == 1) {
+    if (warp == 0) {
         tmem_alloc(tmem_ptr, kPrepTmemCols);
         tmem_relinquish();
     }
@@ -442,23 +470,19 @@ prep_kernel(const __grid_constant__ PrepMaps maps, const PrefillArgs a) {
 
     if (warp == 0) {
         if (lane == 0) {
-            uint64_t *full = &bars[PB_FULL];
-            mbar_arrive_expect_tx(full, 16384 + 64 * Dv * 2);
+            // K now; V once the solve has freed A's region (the load overlaps the
+            // T images, W and its extraction)
             const int r0 = (int)row0;
-            tma_load_3d(sm + PS_K, &maps.k, full, 0, h, r0);
-            tma_load_3d(sm + PS_K + 8192, &maps.k, full, 64, h, r0);
-            tma_load_3d(sm + PS_V, &maps.v, full, 0, h, r0);
-            if (Dv == 128) tma_load_3d(sm + PS_V + 8192, &maps.v, full, 64, h, r0);
-            drain_bar(full, 0);      // the CTA may not exit with the copies in flight
-        }
-    } else if (warp == 1) {
-        if (lane == 0) {
+            mbar_arrive_expect_tx(&bars[PB_FULL], 16384);
+            tma_load_3d(sm + PS_K, &maps.k, &bars[PB_FULL], 0, h, r0);
+            tma_load_3d(sm + PS_K + 8192, &maps.k, &bars[PB_FULL], 64, h, r0);
+            bool v_issued = false;
             const uint32_t kk_ = smem_u32(sm + PS_K), vv = smem_u32(sm + PS_V);
             const uint32_t tbg = smem_u32(sm + PS_TBG), tb = smem_u32(sm + PS_TB);
             constexpr uint32_t ID_KK = idesc_bf16(64, 64, 0, 0);
             constexpr uint32_t ID_W = idesc_bf16(64, 128, 0, 1);
             const uint32_t ID_U = Dv == 128 ? idesc_bf16(64, 128, 0, 1) : idesc_bf16(64, 64, 0, 1);
-            bool ok = wait_bar(&bars[PB_FULL], 0, abort_flag, a.err);
+            bool ok = wait_bar2(&bars[PB_FULL], 0, abort_flag, agent_flag, a.err);
             if (ok) {
                 tc_fence_after();
 #pragma unroll
@@ -468,16 +492,23 @@ prep_kernel(const __grid_constant__ PrepMaps maps, const PrefillArgs a) {
                              smem_desc(kk_ + off, 16, 1024, kSw128), ID_KK, kk > 0);
                 }
                 mma_commit(&bars[PB_KK]);
-                ok = wait_bar(&bars[PB_TREADY], 0, abort_flag, a.err);
+                ok = wait_bar2(&bars[PB_TREADY], 0, abort_flag, agent_flag, a.err);
             }
             if (ok) {
+                // the compute threads fenced their generic accesses to A's region
+                // before the barrier that preceded TREADY
+                mbar_arrive_expect_tx(&bars[PB_VFULL], 64 * Dv * 2);
+                tma_load_3d(sm + PS_V, &maps.v, &bars[PB_VFULL], 0, h, r0);
+                if (Dv == 128) tma_load_3d(sm + PS_V + 8192, &maps.v, &bars[PB_VFULL], 64, h, r0);
+                v_issued = true;
                 tc_fence_after();
 #pragma unroll
                 for (int kk = 0; kk < 4; ++kk)       // W = T diag(beta e^g) K  (B = K, MN-major)
                     mma_bf16(tmem + PT_W, smem_desc(tbg + kk * 32, 16, 1024, kSw128),
                              smem_desc(kk_ + kk * 2048, 8192, 1024, kSw128), ID_W, kk > 0);
                 mma_commit(&bars[PB_W]);
-                ok = wait_bar(&bars[PB_WFREE], 0, abort_flag, a.err);
+                ok = wait_bar2(&bars[PB_WFREE], 0, abort_flag, agent_flag, a.err) &&
+                     wait_bar2(&bars[PB_VFULL], 0, abort_flag, agent_flag, a.err);
             }
             if (ok) {
                 tc_fence_after();
@@ -489,13 +520,15 @@ prep_kernel(const __grid_constant__ PrepMaps maps, const PrefillArgs a) {
             }
             mma_commit(&bars[PB_DRAIN]);      // every MMA issued has completed before TMEM is freed
             drain_bar(&bars[PB_DRAIN], 0);
+            drain_bar(&bars[PB_FULL], 0);     // the CTA may not exit with copies in flight
+            if (v_issued) drain_bar(&bars[PB_VFULL], 0);
         }
     } else {
-        const int cw = threadIdx.x - 64;
+        const int cw = threadIdx.x - 32;
         const int q4 = warp & 3;
         const int r = 32 * q4 + lane;              // TMEM lane
-        const bool lo = lane < 16;
-        const int m = 16 * q4 + lane;              // row of an M=64 accumulator (if lo)
+        // rows ta, ta + 8 and column pairs 8 kb + j2 of the M=64 accumulators (16x256b loads)
+        const int ta = 16 * q4 + (lane >> 2), j2 = 2 * (lane & 3);
         const uint32_t tq = tmem + ((uint32_t)(32 * q4) << 16);
         float *Af = reinterpret_cast<float *>(sm + PS_AF);
         float *Tf = reinterpret_cast<float *>(sm + PS_TF);
@@ -506,40 +539,49 @@ prep_kernel(const __grid_constant__ PrepMaps maps, const PrefillArgs a) {
         named_bar_sync(1, 128);
         if (!*abort_flag) {
             tc_fence_after();
-            // A row m: beta_m (K K^T)[m][s] e^{g_m - g_s}, s < m  (all four warps load: the
-            // TMEM load is warp-wide; lanes >= 16 hold no row and store nothing)
-            gram_row<true>(tq + PT_KK, m, b_s[m & 63], g_s, [&](int b, const float *x) {
-                if (lo) {
+            // A rows ta, ta + 8: beta_t (K K^T)[t][s] e^{g_t - g_s}, s < t
+            float v[32];
+            gram_rows<true>(tq + PT_KK, ta, lane, b_s, g_s, v);
 #pragma unroll
-                    for (int c4 = 0; c4 < 4; ++c4)
-                        *reinterpret_cast<float4 *>(Af + m * kLd + 16 * b + 4 * c4) =
-                            make_float4(x[4 * c4], x[4 * c4 + 1], x[4 * c4 + 2], x[4 * c4 + 3]);
-                }
-            });
+            for (int kb = 0; kb < 8; ++kb) {
+                const int s = 8 * kb + j2;
+                *reinterpret_cast<float2 *>(Af + ta * kLd + s) = make_float2(v[4 * kb], v[4 * kb + 1]);
+                *reinterpret_cast<float2 *>(Af + (ta + 8) * kLd + s) = make_float2(v[4 * kb + 2], v[4 * kb + 3]);
+            }
             tc_fence_before();
         }
         named_bar_sync(1, 128);
         if (!*abort_flag) {
             ut_solve(Af, Tf, Xs, cw);      // ends with a barrier: A is dead from here
-            // T diag(beta e^g) and T diag(beta gamma) as bf16 K-major SW128 images, over A
+            // T diag(beta e^g) and T diag(beta gamma) as bf16 K-major SW128 images,
+            // over T: every thread reads its part of T before any image is written
             const int t = cw >> 1, half = cw & 1;
+            uint4 y1[4], y2[4];
 #pragma unroll
             for (int cc = 0; cc < 4; ++cc) {
                 const int s0 = 32 * half + 8 * cc;
                 const float4 t0 = *reinterpret_cast<const float4 *>(Tf + t * kLd + s0);
                 const float4 t1 = *reinterpret_cast<const float4 *>(Tf + t * kLd + s0 + 4);
                 const float tv[8] = {t0.x, t0.y, t0.z, t0.w, t1.x, t1.y, t1.z, t1.w};
-                float y1[8], y2[8];
+                float z1[8], z2[8];
 #pragma unroll
                 for (int e = 0; e < 8; ++e) {
-                    y1[e] = tv[e] * b_s[s0 + e] * eg_s[s0 + e];
-                    y2[e] = tv[e] * bg_s[s0 + e];
+                    z1[e] = tv[e] * b_s[s0 + e] * eg_s[s0 + e];
+                    z2[e] = tv[e] * bg_s[s0 + e];
                 }
-                *reinterpret_cast<uint4 *>(sm + PS_TBG + swz(t, 4 * half + cc, 128)) = pack8(y1);
-                *reinterpret_cast<uint4 *>(sm + PS_TB + swz(t, 4 * half + cc, 128)) = pack8(y2);
+                y1[cc] = pack8(z1);
+                y2[cc] = pack8(z2);
             }
-            fence_proxy_async_smem();
+            named_bar_sync(1, 128);
+#pragma unroll
+            for (int cc = 0; cc < 4; ++cc) {
+                *reinterpret_cast<uint4 *>(sm + PS_TBG + swz(t, 4 * half + cc, 128)) = y1[cc];
+                *reinterpret_cast<uint4 *>(sm + PS_TB + swz(t, 4 * half + cc, 128)) = y2[cc];
+            }
         }
+        // generic accesses to A's region (reused by the V load) and the T images
+        // (read by the MMAs) before the async proxy touches them
+        fence_proxy_async_smem();
         named_bar_sync(1, 128);
         if (cw == 0 && !*abort_flag) {
             mbar_arrive(&bars[PB_TREADY]);
@@ -548,23 +590,19 @@ prep_kernel(const __grid_constant__ PrepMaps maps, const PrefillArgs a) {
         named_bar_sync(1, 128);
         if (!*abort_flag) {
             tc_fence_after();
-            // -W rows -> bf16 K-major SW128 image (2 halves of 64 columns), over T
+            // -W rows -> bf16 K-major SW128 image (2 halves of 64 columns), over K
 #pragma unroll
             for (int half = 0; half < 2; ++half) {
+                float v[32];
+                tmem_ld_16x256b_x4(tq + PT_W + 64 * half, v);
+                tmem_ld_16x256b_x4(tq + PT_W + 64 * half + 32, v + 16);
+                tmem_wait_ld();
+                uint8_t *wi = sm + PS_WIMG + half * 8192 + 2 * j2;
 #pragma unroll
-                for (int p = 0; p < 2; ++p) {
-                    float x[32];
-                    tmem_ld16(tq + PT_W + 64 * half + 32 * p, x);
-                    tmem_ld16(tq + PT_W + 64 * half + 32 * p + 16, x + 16);
-                    tmem_wait_ld();
-                    if (lo) {
-#pragma unroll
-                        for (int i = 0; i < 32; ++i) x[i] = -x[i];
-#pragma unroll
-                        for (int cc = 0; cc < 4; ++cc)
-                            *reinterpret_cast<uint4 *>(sm + PS_WIMG + half * 8192 + swz(m, 4 * p + cc, 128)) =
-                                pack8(x + 8 * cc);
-                    }
+                for (int kb = 0; kb < 8; ++kb) {
+                    *reinterpret_cast<uint32_t *>(wi + swz(ta, kb, 128)) = pack_bf16(-v[4 * kb], -v[4 * kb + 1]);
+                    *reinterpret_cast<uint32_t *>(wi + swz(ta + 8, kb, 128)) =
+                        pack_bf16(-v[4 * kb + 2], -v[4 * kb + 3]);
                 }
             }
             fence_proxy_async_smem();
@@ -580,23 +618,18 @@ prep_kernel(const __grid_constant__ PrepMaps maps, const PrefillArgs a) {
         named_bar_sync(1, 128);
         if (!*abort_flag) {
             tc_fence_after();
-            // U' rows -> bf16, value slices of width NV: slice s at s*64*NV*2, row m at m*NV*2
+            // U' rows -> bf16, value slices of width NV: slice s at s*64*NV*2, row t at t*NV*2
             for (int half = 0; half < Dv / 64; ++half) {
+                float v[32];
+                tmem_ld_16x256b_x4(tq + PT_U + 64 * half, v);
+                tmem_ld_16x256b_x4(tq + PT_U + 64 * half + 32, v + 16);
+                tmem_wait_ld();
 #pragma unroll
-                for (int p = 0; p < 2; ++p) {
-                    float x[32];
-                    tmem_ld16(tq + PT_U + 64 * half + 32 * p, x);
-                    tmem_ld16(tq + PT_U + 64 * half + 32 * p + 16, x + 16);
-                    tmem_wait_ld();
-                    if (lo) {
-#pragma unroll
-                        for (int cc = 0; cc < 4; ++cc) {
-                            const int col = 64 * half + 32 * p + 8 * cc;
-                            const int sl = col / NV, cin = col % NV;
-                            *reinterpret_cast<uint4 *>(sm + PS_UIMG + sl * (64 * NV * 2) + m * (NV * 2) + cin * 2) =
-                                pack8(x + 8 * cc);
-                        }
-                    }
+                for (int kb = 0; kb < 8; ++kb) {
+                    const int col = 64 * half + 8 * kb + j2;
+                    uint8_t *ui = sm + PS_UIMG + (col / NV) * (64 * NV * 2) + (col % NV) * 2;
+                    *reinterpret_cast<uint32_t *>(ui + ta * (NV * 2)) = pack_bf16(v[4 * kb], v[4 * kb + 1]);
+                    *reinterpret_cast<uint32_t *>(ui + (ta + 8) * (NV * 2)) = pack_bf16(v[4 * kb + 2], v[4 * kb + 3]);
                 }
             }
             fence_proxy_async_smem();
@@ -614,7 +647,7 @@ prep_kernel(const __grid_constant__ PrepMaps maps, const PrefillArgs a) {
 
     tc_fence_before();
     __syncthreads();
-    if (warp == 1) {
+    if (warp == 0) {
         tc_fence_after();
         tmem_dealloc(tmem, kPrepTmemCols);
     }
@@ -634,7 +667,7 @@ constexpr uint32_t QS_G = 40960;      // gates (6 x 64 fp32)
 constexpr uint32_t QS_BAR = QS_G + 6 * 64 * 4;
 constexpr uint32_t QS_TMEMPTR = QS_BAR + 4 * 8;
 constexpr uint32_t QS_FLAGS = QS_TMEMPTR + 4;
-constexpr uint32_t kQkSmem = QS_FLAGS + 4 + 1024;
+constexpr uint32_t kQkSmem = QS_FLAGS + 8 + 1024;   // flags: compute threads', MMA thread's
 enum QkBar { QB_FULL = 0, QB_QK, QB_DRAIN, kQkBars };
 
 __global__ void __launch_bounds__(kQkThreads, 4)
@@ -651,6 +684,7 @@ qk_kernel(const __grid_constant__ PrepMaps maps, const PrefillArgs a) {
     uint64_t *bars = reinterpret_cast<uint64_t *>(sm + QS_BAR);
     uint32_t *tmem_ptr = reinterpret_cast<uint32_t *>(sm + QS_TMEMPTR);
     volatile int *abort_flag = reinterpret_cast<volatile int *>(sm + QS_FLAGS);
+    volatile int *agent_flag = abort_flag + 1;
     float *g_s = reinterpret_cast<float *>(sm + QS_G);
     const float *eg_s = g_s + 256;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -658,6 +692,7 @@ qk_kernel(const __grid_constant__ PrepMaps maps, const PrefillArgs a) {
     if (threadIdx.x == 0) {
         for (int i = 0; i < kQkBars; ++i) mbar_init(&bars[i], 1);
         *abort_flag = 0;
+        *agent_flag = 0;
         fence_mbar_init();
     }
     if (warp == 1) {
@@ -685,7 +720,7 @@ qk_kernel(const __grid_constant__ PrepMaps maps, const PrefillArgs a) {
         if (lane == 0) {
             const uint32_t qq = smem_u32(sm + QS_Q), kk_ = smem_u32(sm + QS_K);
             constexpr uint32_t ID_QK = idesc_bf16(64, 64, 0, 0);
-            if (wait_bar(&bars[QB_FULL], 0, abort_flag, a.err)) {
+            if (wait_bar2(&bars[QB_FULL], 0, abort_flag, agent_flag, a.err)) {
                 tc_fence_after();
 #pragma unroll
                 for (int kk = 0; kk < 8; ++kk) {
@@ -702,21 +737,22 @@ qk_kernel(const __grid_constant__ PrepMaps maps, const PrefillArgs a) {
         const int cw = threadIdx.x - 64;
         const int q4 = warp & 3;
         const int r = 32 * q4 + lane;
-        const bool lo = lane < 16;
-        const int m = 16 * q4 + lane;
+        const int ta = 16 * q4 + (lane >> 2), j2 = 2 * (lane & 3);
         const uint32_t tq = tmem + ((uint32_t)(32 * q4) << 16);
         chunk_gates(a, row0, lenc, h, r, lane, g_s);
         if (cw == 0 && !wait_bar(&bars[QB_QK], 0, abort_flag, a.err)) *abort_flag = 1;
         named_bar_sync(1, 128);
         if (!*abort_flag) {
             tc_fence_after();
-            // P row m: (Q K^T)[m][s] e^{g_m - g_s}, s <= m  -> bf16 K-major SW128 image
-            gram_row<false>(tq, m, 1.f, g_s, [&](int b, const float *x) {
-                if (lo) {
-                    *reinterpret_cast<uint4 *>(sm + QS_P + swz(m, 2 * b, 128)) = pack8(x);
-                    *reinterpret_cast<uint4 *>(sm + QS_P + swz(m, 2 * b + 1, 128)) = pack8(x + 8);
-                }
-            });
+            // P rows ta, ta + 8: (Q K^T)[t][s] e^{g_t - g_s}, s <= t  -> bf16 K-major SW128 image
+            float v[32];
+            gram_rows<false>(tq, ta, lane, nullptr, g_s, v);
+#pragma unroll
+            for (int kb = 0; kb < 8; ++kb) {
+                *reinterpret_cast<uint32_t *>(sm + QS_P + swz(ta, kb, 128) + 2 * j2) = pack_bf16(v[4 * kb], v[4 * kb + 1]);
+                *reinterpret_cast<uint32_t *>(sm + QS_P + swz(ta + 8, kb, 128) + 2 * j2) =
+                    pack_bf16(v[4 * kb + 2], v[4 * kb + 3]);
+            }
             // diag(e^g) Q in place (Q was read only by the MMA): row cw/2, 64 columns per thread
             const int t = cw >> 1, half = cw & 1;
             const float e = eg_s[t];
@@ -863,6 +899,7 @@ scan_kernel(const __grid_constant__ ScanMaps maps, const PrefillArgs a) {
     constexpr uint32_t SC_SS = L::SS, SC_UT = L::UT;
     uint64_t *bars = reinterpret_cast<uint64_t *>(sm + L::BAR);
     volatile int *abort_flag = reinterpret_cast<volatile int *>(sm + L::FLAGS);
+    volatile int *agent_flag = abort_flag + 1;     // the producer's
     constexpr int NW = NV * 4 / kScanWarps;     // value columns per warp
     constexpr int NT = NW / 8;                  // n-tiles of 8 columns per warp
     constexpr uint32_t RS = NV * 2 + 16;        // padded row stride of the S / U~ buffers
@@ -895,6 +932,7 @@ scan_kernel(const __grid_constant__ ScanMaps maps, const PrefillArgs a) {
             mbar_init(&bars[SB_EMPTY + i], NCW);
         }
         *abort_flag = 0;
+        *agent_flag = 0;
         fence_mbar_init();
         if (nchunks > 0) prefetch_tensormap(&maps.k);
     }
@@ -907,7 +945,7 @@ scan_kernel(const __grid_constant__ ScanMaps maps, const PrefillArgs a) {
             for (int c = 0; c < nchunks; ++c) {
                 const int st = c % kScanStages;
                 if (c >= kScanStages &&
-                    !wait_bar(&bars[SB_EMPTY + st], (c / kScanStages - 1) & 1, abort_flag, a.err))
+                    !wait_bar2(&bars[SB_EMPTY + st], (c / kScanStages - 1) & 1, abort_flag, agent_flag, a.err))
                     break;
                 uint64_t *full = &bars[SB_FULL + st];
                 uint8_t *stg = sm + st * SS_STAGE;
