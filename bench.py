@@ -30,9 +30,9 @@ sys.path.insert(0, ROOT)
 
 METRIC = "RDA prefill tokens/s (H=16,D=128) and decode state GB/s on 1 B200 vs roofline"
 WORKLOAD = "nano_prefill_b1_t4096_h16_d128"
-# kernels one fixed-length bf16 prefill call enqueues (prep, output operands,
-# state scan with the outputs)
-LAUNCHES_PER_PREFILL = 3
+# kernels one fixed-length bf16 prefill call enqueues (prep with the output
+# operands, state scan with the outputs)
+LAUNCHES_PER_PREFILL = 2
 CHUNK = 64
 
 

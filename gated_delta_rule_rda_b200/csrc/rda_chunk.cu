@@ -17,28 +17,23 @@
 //
 // which equals the token-by-token rule exactly in real arithmetic.
 //
-// Three kernels on the caller's stream (one of them forked onto a side stream):
+// Two kernels on the caller's stream:
 //
 //  1. prep (chunk-parallel; one CTA per (chunk, head) over every chunk of
-//     every sequence at once): what the state chain needs from a chunk.  g,
-//     K K^T on the tensor cores, A, the UT transform (diagonal 16x16 blocks by
-//     forward substitution, off-diagonal blocks by recursive doubling on tf32
-//     mma.sync), then W and U' on the tensor cores.  Writes -W as a
-//     ready-to-use swizzled operand image, U' in value slices and the decay
-//     factors.
-//  2. output operands (chunk-parallel): P and diag(e^g) Q, the chunk-local
-//     operands of the outputs.  Independent of the prep, so it runs on a side
-//     stream beside it; the scan waits for both.
-//  3. scan (sequential over the chunks of one (sequence, head, value slice)).
+//     every sequence at once): everything the state chain and the outputs
+//     need from a chunk.  g, K K^T and Q K^T on the tensor cores, A and P from
+//     them, diag(e^g) Q, the UT transform (diagonal 16x16 blocks by forward
+//     substitution, off-diagonal blocks by recursive doubling on tf32
+//     mma.sync), then W and U' on the tensor cores.  Writes -W, diag(e^g) Q
+//     and P as ready-to-use swizzled operand images, U' in value slices and
+//     the decay factors.  Four CTAs per SM (55 KiB of shared memory, 128 TMEM
+//     columns each): the Q, K, V, A and T tiles share three regions in turn.
+//  2. scan (sequential over the chunks of one (sequence, head, value slice)).
 //     Carries the fp32 state in registers; per chunk U = U' - W S and the
 //     outputs O = scale (diag(e^g) Q S + P U) -- the two products with S share
 //     its operand fragments -- then S <- e^{g_C} S + K^T diag(e^{g_C - g}) U, on
 //     register-fragment MMAs.  Value columns are independent under the rule,
 //     so slicing is exact.
-//
-// The prep is split from the output operands so that each chunk-parallel
-// kernel fits several CTAs per SM: the prep needs 72 KiB of shared memory and
-// 128 TMEM columns (three per SM), the output operands 43 KiB and 64 columns.
 //
 // Operands: bf16 in shared memory, fp32 accumulators in TMEM (tcgen05.mma),
 // Q/K/V tiles by TMA, workspace images by bulk copies.  Every wait is
@@ -294,7 +289,9 @@ __device__ __forceinline__ void ut_solve(float *Af, float *Tf, float *Xs, int cw
 
 // ---------------------------------------------------------------------------
 // Kernel 1: prep.  One CTA per (global chunk, head): everything the scan
-// needs from a chunk -- g, A from K K^T, the UT transform T, then W and U'.
+// needs from a chunk -- g, A from K K^T, the UT transform T, then W and U' --
+// and the chunk-local operands of the outputs, P = (Q K^T) o Gamma (causal,
+// diagonal kept) and diag(e^g) Q.
 // Four CTAs share an SM (shared memory <= 55 KiB, 128 TMEM columns, <= 96
 // registers): three regions are reused as the chunk's work moves along.
 // ---------------------------------------------------------------------------
@@ -304,24 +301,26 @@ constexpr uint32_t kPrepTmemCols = 128;
 constexpr uint32_t PS_K = 0;           // K [64 x 128]: halves of 8 KiB (SW128); later the -W image
 constexpr uint32_t PS_AF = 16384;      // A fp32 [64][kLd]; after the solve V [64 x Dv] (halves
                                        // of 8 KiB, SW128), after the U' MMA the U' slices
-constexpr uint32_t PS_TF = PS_AF + 64 * kLd * 4;     // T fp32 [64][kLd]; later the two T images
+constexpr uint32_t PS_TF = PS_AF + 64 * kLd * 4;     // Q [64 x 128] (halves of 8 KiB, SW128) until the
+                                                     // solve; T fp32 [64][kLd]; then the two T images
 constexpr uint32_t PS_XS = PS_TF + 64 * kLd * 4;     // 4 x 16x8 fp32
 constexpr uint32_t PS_G = PS_XS + 4 * 128 * 4;       // g, beta, beta*gamma, e^{ref-g}, e^g, e^{g_C-g}: 6 x 64 fp32
 constexpr uint32_t PS_BAR = PS_G + 6 * 64 * 4;
-constexpr uint32_t PS_TMEMPTR = PS_BAR + 8 * 8;
+constexpr uint32_t PS_TMEMPTR = PS_BAR + 10 * 8;
 constexpr uint32_t PS_FLAGS = PS_TMEMPTR + 4;
 constexpr uint32_t kPrepSmem = PS_FLAGS + 8 + 1024;   // flags: compute threads', TMA / MMA thread's
 constexpr uint32_t PS_V = PS_AF;              // V, over A (loaded after the solve)
+constexpr uint32_t PS_Q = PS_TF;              // Q, where T goes later
 constexpr uint32_t PS_TBG = PS_TF;            // T diag(beta e^g), over T
 constexpr uint32_t PS_TB = PS_TF + 8192;      // T diag(beta gamma)
 constexpr uint32_t PS_WIMG = PS_K;            // -W image, over K (after the W MMA)
 constexpr uint32_t PS_UIMG = PS_V;            // U' slices, over V (after the U' MMA)
 static_assert(PS_AF % 1024 == 0 && PS_TF % 1024 == 0, "SW128 tiles need 1024-byte alignment");
 static_assert(4 * (kPrepSmem + 1024) <= 233472, "four prep CTAs per SM");
-// TMEM columns: K K^T, then W, then U' (one at a time)
-constexpr uint32_t PT_KK = 0, PT_W = 0, PT_U = 0;
-enum PrepBar { PB_FULL = 0, PB_VFULL, PB_KK, PB_TREADY, PB_W, PB_WFREE, PB_U, PB_DRAIN, kPrepBars };
-static_assert(kPrepBars <= 8, "barrier area");
+// TMEM columns: K K^T and Q K^T side by side, then W, then U' (one at a time)
+constexpr uint32_t PT_KK = 0, PT_QK = 64, PT_W = 0, PT_U = 0;
+enum PrepBar { PB_FULL = 0, PB_VFULL, PB_KK, PB_QK, PB_TREADY, PB_W, PB_WFREE, PB_U, PB_DRAIN, kPrepBars };
+static_assert(kPrepBars <= 10, "barrier area");
 
 struct PrepMaps {
     CUtensorMap q, k, v;
@@ -470,14 +469,16 @@ prep_kernel(const __grid_constant__ PrepMaps maps, const PrefillArgs a) {
 
     if (warp == 0) {
         if (lane == 0) {
-            // K now; V once the solve has freed A's region (the load overlaps the
-            // T images, W and its extraction)
+            // K and Q now; V once the solve has freed A's region (the load overlaps
+            // the T images, W and its extraction)
             const int r0 = (int)row0;
-            mbar_arrive_expect_tx(&bars[PB_FULL], 16384);
+            mbar_arrive_expect_tx(&bars[PB_FULL], 32768);
             tma_load_3d(sm + PS_K, &maps.k, &bars[PB_FULL], 0, h, r0);
             tma_load_3d(sm + PS_K + 8192, &maps.k, &bars[PB_FULL], 64, h, r0);
+            tma_load_3d(sm + PS_Q, &maps.q, &bars[PB_FULL], 0, h, r0);
+            tma_load_3d(sm + PS_Q + 8192, &maps.q, &bars[PB_FULL], 64, h, r0);
             bool v_issued = false;
-            const uint32_t kk_ = smem_u32(sm + PS_K), vv = smem_u32(sm + PS_V);
+            const uint32_t kk_ = smem_u32(sm + PS_K), qq = smem_u32(sm + PS_Q), vv = smem_u32(sm + PS_V);
             const uint32_t tbg = smem_u32(sm + PS_TBG), tb = smem_u32(sm + PS_TB);
             constexpr uint32_t ID_KK = idesc_bf16(64, 64, 0, 0);
             constexpr uint32_t ID_W = idesc_bf16(64, 128, 0, 1);
@@ -492,6 +493,13 @@ prep_kernel(const __grid_constant__ PrepMaps maps, const PrefillArgs a) {
                              smem_desc(kk_ + off, 16, 1024, kSw128), ID_KK, kk > 0);
                 }
                 mma_commit(&bars[PB_KK]);
+#pragma unroll
+                for (int kk = 0; kk < 8; ++kk) {     // Q K^T: A = the Q tile, B = the K tile (K-major)
+                    const uint32_t off = (kk >> 2) * 8192 + (kk & 3) * 32;
+                    mma_bf16(tmem + PT_QK, smem_desc(qq + off, 16, 1024, kSw128),
+                             smem_desc(kk_ + off, 16, 1024, kSw128), ID_KK, kk > 0);
+                }
+                mma_commit(&bars[PB_QK]);
                 ok = wait_bar2(&bars[PB_TREADY], 0, abort_flag, agent_flag, a.err);
             }
             if (ok) {
@@ -550,7 +558,41 @@ prep_kernel(const __grid_constant__ PrepMaps maps, const PrefillArgs a) {
             }
             tc_fence_before();
         }
+        if (cw == 0 && !*abort_flag && !wait_bar(&bars[PB_QK], 0, abort_flag, a.err)) *abort_flag = 1;
         named_bar_sync(1, 128);
+        if (!*abort_flag) {
+            // the Q tile landed before the Q K^T product was issued; this wait (complete
+            // already) makes the copy visible to these threads
+            wait_bar(&bars[PB_FULL], 0, abort_flag, a.err);
+            tc_fence_after();
+            // P rows ta, ta + 8: (Q K^T)[t][s] e^{g_t - g_s}, s <= t -> bf16 K-major
+            // SW128 image, stored from registers
+            float v[32];
+            gram_rows<false>(tq + PT_QK, ta, lane, nullptr, g_s, v);
+            uint8_t *pi = img + kImgP + 2 * j2;
+#pragma unroll
+            for (int kb = 0; kb < 8; ++kb) {
+                *reinterpret_cast<uint32_t *>(pi + swz(ta, kb, 128)) = pack_bf16(v[4 * kb], v[4 * kb + 1]);
+                *reinterpret_cast<uint32_t *>(pi + swz(ta + 8, kb, 128)) = pack_bf16(v[4 * kb + 2], v[4 * kb + 3]);
+            }
+            // diag(e^g) Q: the same byte layout as the loaded Q tile; 16-byte pieces,
+            // consecutive threads on consecutive pieces
+#pragma unroll
+            for (int k = 0; k < 8; ++k) {
+                const uint32_t off = 16u * (uint32_t)(cw + 128 * k);
+                const float e = eg_s[(off & 8191u) >> 7];
+                const uint4 u = *reinterpret_cast<const uint4 *>(sm + PS_Q + off);
+                uint32_t wv[4] = {u.x, u.y, u.z, u.w};
+#pragma unroll
+                for (int i = 0; i < 4; ++i) {
+                    const float2 f = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(&wv[i]));
+                    wv[i] = pack_bf16(f.x * e, f.y * e);
+                }
+                *reinterpret_cast<uint4 *>(img + kImgQ + off) = make_uint4(wv[0], wv[1], wv[2], wv[3]);
+            }
+            tc_fence_before();
+        }
+        named_bar_sync(1, 128);      // Q is dead: T goes there
         if (!*abort_flag) {
             ut_solve(Af, Tf, Xs, cw);      // ends with a barrier: A is dead from here
             // T diag(beta e^g) and T diag(beta gamma) as bf16 K-major SW128 images,
@@ -650,144 +692,6 @@ prep_kernel(const __grid_constant__ PrepMaps maps, const PrefillArgs a) {
     if (warp == 0) {
         tc_fence_after();
         tmem_dealloc(tmem, kPrepTmemCols);
-    }
-}
-
-// ---------------------------------------------------------------------------
-// Kernel 1b: output operands.  One CTA per (global chunk, head): P = (Q K^T) o
-// Gamma (causal, diagonal kept) and diag(e^g) Q, the chunk-local operands of
-// the outputs, as the scan's shared-memory images.
-// ---------------------------------------------------------------------------
-constexpr int kQkThreads = 192;       // warp 0 TMA, warp 1 MMA, warps 2..5 compute
-constexpr uint32_t kQkTmemCols = 64;
-constexpr uint32_t QS_Q = 0;          // Q [64 x 128]: halves of 8 KiB (SW128), scaled in place
-constexpr uint32_t QS_K = 16384;      // K [64 x 128]
-constexpr uint32_t QS_P = 32768;      // P image (8 KiB)
-constexpr uint32_t QS_G = 40960;      // gates (6 x 64 fp32)
-constexpr uint32_t QS_BAR = QS_G + 6 * 64 * 4;
-constexpr uint32_t QS_TMEMPTR = QS_BAR + 4 * 8;
-constexpr uint32_t QS_FLAGS = QS_TMEMPTR + 4;
-constexpr uint32_t kQkSmem = QS_FLAGS + 8 + 1024;   // flags: compute threads', MMA thread's
-enum QkBar { QB_FULL = 0, QB_QK, QB_DRAIN, kQkBars };
-
-__global__ void __launch_bounds__(kQkThreads, 4)
-qk_kernel(const __grid_constant__ PrepMaps maps, const PrefillArgs a) {
-    extern __shared__ uint8_t smem_raw[];
-    uint8_t *sm = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-    ChunkLoc loc;
-    if (!locate_chunk(a, blockIdx.x, loc)) return;
-    const long gc = loc.gc;
-    const int h = blockIdx.y;
-    const int H = a.H;
-    const int lenc = (int)min((long)kC, loc.len - (long)loc.c * kC);
-    const long row0 = loc.t0 + (long)loc.c * kC;
-    uint64_t *bars = reinterpret_cast<uint64_t *>(sm + QS_BAR);
-    uint32_t *tmem_ptr = reinterpret_cast<uint32_t *>(sm + QS_TMEMPTR);
-    volatile int *abort_flag = reinterpret_cast<volatile int *>(sm + QS_FLAGS);
-    volatile int *agent_flag = abort_flag + 1;
-    float *g_s = reinterpret_cast<float *>(sm + QS_G);
-    const float *eg_s = g_s + 256;
-    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-
-    if (threadIdx.x == 0) {
-        for (int i = 0; i < kQkBars; ++i) mbar_init(&bars[i], 1);
-        *abort_flag = 0;
-        *agent_flag = 0;
-        fence_mbar_init();
-    }
-    if (warp == 1) {
-        tmem_alloc(tmem_ptr, kQkTmemCols);
-        tmem_relinquish();
-    }
-    tc_fence_before();
-    __syncthreads();
-    tc_fence_after();
-    const uint32_t tmem = *tmem_ptr;
-    uint8_t *img = a.workspace_chunks + ((size_t)gc * H + h) * a.chunk_bytes;
-
-    if (warp == 0) {
-        if (lane == 0) {
-            uint64_t *full = &bars[QB_FULL];
-            mbar_arrive_expect_tx(full, 32768);
-            const int r0 = (int)row0;
-            tma_load_3d(sm + QS_Q, &maps.q, full, 0, h, r0);
-            tma_load_3d(sm + QS_Q + 8192, &maps.q, full, 64, h, r0);
-            tma_load_3d(sm + QS_K, &maps.k, full, 0, h, r0);
-            tma_load_3d(sm + QS_K + 8192, &maps.k, full, 64, h, r0);
-            drain_bar(full, 0);
-        }
-    } else if (warp == 1) {
-        if (lane == 0) {
-            const uint32_t qq = smem_u32(sm + QS_Q), kk_ = smem_u32(sm + QS_K);
-            constexpr uint32_t ID_QK = idesc_bf16(64, 64, 0, 0);
-            if (wait_bar2(&bars[QB_FULL], 0, abort_flag, agent_flag, a.err)) {
-                tc_fence_after();
-#pragma unroll
-                for (int kk = 0; kk < 8; ++kk) {
-                    const uint32_t off = (kk >> 2) * 8192 + (kk & 3) * 32;
-                    mma_bf16(tmem, smem_desc(qq + off, 16, 1024, kSw128), smem_desc(kk_ + off, 16, 1024, kSw128),
-                             ID_QK, kk > 0);
-                }
-                mma_commit(&bars[QB_QK]);
-            }
-            mma_commit(&bars[QB_DRAIN]);
-            drain_bar(&bars[QB_DRAIN], 0);
-        }
-    } else {
-        const int cw = threadIdx.x - 64;
-        const int q4 = warp & 3;
-        const int r = 32 * q4 + lane;
-        const int ta = 16 * q4 + (lane >> 2), j2 = 2 * (lane & 3);
-        const uint32_t tq = tmem + ((uint32_t)(32 * q4) << 16);
-        chunk_gates(a, row0, lenc, h, r, lane, g_s);
-        if (cw == 0 && !wait_bar(&bars[QB_QK], 0, abort_flag, a.err)) *abort_flag = 1;
-        named_bar_sync(1, 128);
-        if (!*abort_flag) {
-            tc_fence_after();
-            // P rows ta, ta + 8: (Q K^T)[t][s] e^{g_t - g_s}, s <= t  -> bf16 K-major SW128 image
-            float v[32];
-            gram_rows<false>(tq, ta, lane, nullptr, g_s, v);
-#pragma unroll
-            for (int kb = 0; kb < 8; ++kb) {
-                *reinterpret_cast<uint32_t *>(sm + QS_P + swz(ta, kb, 128) + 2 * j2) = pack_bf16(v[4 * kb], v[4 * kb + 1]);
-                *reinterpret_cast<uint32_t *>(sm + QS_P + swz(ta + 8, kb, 128) + 2 * j2) =
-                    pack_bf16(v[4 * kb + 2], v[4 * kb + 3]);
-            }
-            // diag(e^g) Q in place (Q was read only by the MMA): row cw/2, 64 columns per thread
-            const int t = cw >> 1, half = cw & 1;
-            const float e = eg_s[t];
-            uint8_t *row = sm + QS_Q + half * 8192;
-#pragma unroll
-            for (int cc = 0; cc < 8; ++cc) {
-                uint4 *pq = reinterpret_cast<uint4 *>(row + swz(t, cc, 128));
-                uint4 u = *pq;
-                uint32_t wv[4] = {u.x, u.y, u.z, u.w};
-#pragma unroll
-                for (int i = 0; i < 4; ++i) {
-                    float2 f = __bfloat1622float2(*reinterpret_cast<__nv_bfloat162 *>(&wv[i]));
-                    wv[i] = pack_bf16(f.x * e, f.y * e);
-                }
-                *pq = make_uint4(wv[0], wv[1], wv[2], wv[3]);
-            }
-            tc_fence_before();
-        }
-        fence_proxy_async_smem();
-        named_bar_sync(1, 128);
-        if (cw == 0) {
-            if (!*abort_flag) {
-                bulk_store(img + kImgP, sm + QS_P, 8192);
-                bulk_store(img + kImgQ, sm + QS_Q, 16384);
-                bulk_commit();
-            }
-            bulk_wait_reads();
-        }
-    }
-
-    tc_fence_before();
-    __syncthreads();
-    if (warp == 1) {
-        tc_fence_after();
-        tmem_dealloc(tmem, kQkTmemCols);
     }
 }
 
@@ -1220,42 +1124,9 @@ cudaError_t init_attrs() {
     static cudaError_t attr = cudaSuccess;
     std::call_once(once, [] {
         attr = set_smem(prep_kernel<NV>, kPrepSmem);
-        if (attr == cudaSuccess) attr = set_smem(qk_kernel, kQkSmem);
         if (attr == cudaSuccess) attr = set_smem(scan_kernel<NV>, ScanSmem<NV>::BYTES);
     });
     return attr;
-}
-
-// The output-operand kernel depends only on the inputs, so it runs on a side
-// stream next to the prep and the state scan (which leaves SMs and shared
-// memory idle), forked from and joined back to the caller's stream with
-// events.  One side stream and event pair per device, created on first use;
-// a mutex keeps the record / wait pairs of concurrent callers apart.
-struct SideStream {
-    cudaStream_t stream = nullptr;
-    cudaEvent_t fork = nullptr, join = nullptr;
-    bool ready = false;
-};
-std::mutex g_side_mu;
-SideStream g_side[64];
-
-cudaError_t side_stream(SideStream **out) {
-    int dev = 0;
-    cudaError_t e = cudaGetDevice(&dev);
-    if (e != cudaSuccess) return e;
-    if (dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
-    SideStream &ss = g_side[dev];
-    if (!ss.ready) {
-        int least = 0, greatest = 0;
-        if ((e = cudaDeviceGetStreamPriorityRange(&least, &greatest)) != cudaSuccess) return e;
-        if (!ss.stream && (e = cudaStreamCreateWithPriority(&ss.stream, cudaStreamNonBlocking, least)) != cudaSuccess)
-            return e;
-        if (!ss.fork && (e = cudaEventCreateWithFlags(&ss.fork, cudaEventDisableTiming)) != cudaSuccess) return e;
-        if (!ss.join && (e = cudaEventCreateWithFlags(&ss.join, cudaEventDisableTiming)) != cudaSuccess) return e;
-        ss.ready = true;
-    }
-    *out = &ss;
-    return cudaSuccess;
 }
 
 template <int NV>
@@ -1276,21 +1147,9 @@ cudaError_t launch_nv(const PrefillArgs &a, long chunks_grid, cudaStream_t s) {
     const uint32_t scan_smem = ScanSmem<NV>::BYTES;
     const dim3 chunk_grid((unsigned)chunks_grid, a.H, 1);
 
-    std::lock_guard<std::mutex> lk(g_side_mu);
-    SideStream *ss = nullptr;
     if (chunks_grid > 0) {
-        if ((e = side_stream(&ss)) != cudaSuccess) return e;
-        // fork: the output operands wait for everything already on the caller's
-        // stream (a previous call's scan may still read the same workspace) and
-        // run beside the prep; the scan waits for both
-        if ((e = cudaEventRecord(ss->fork, s)) != cudaSuccess) return e;
-        if ((e = cudaStreamWaitEvent(ss->stream, ss->fork, 0)) != cudaSuccess) return e;
-        qk_kernel<<<chunk_grid, kQkThreads, kQkSmem, ss->stream>>>(pm, a);
-        if ((e = cudaGetLastError()) != cudaSuccess) return e;
-        if ((e = cudaEventRecord(ss->join, ss->stream)) != cudaSuccess) return e;
         prep_kernel<NV><<<chunk_grid, kPrepThreads, kPrepSmem, s>>>(pm, a);
         if ((e = cudaGetLastError()) != cudaSuccess) return e;
-        if ((e = cudaStreamWaitEvent(s, ss->join, 0)) != cudaSuccess) return e;      // join
     }
     scan_kernel<NV><<<scan_grid, kScanThreads, scan_smem, s>>>(sm, a);
     return cudaGetLastError();

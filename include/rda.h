@@ -39,13 +39,10 @@
  *   enqueues its work on `stream` (a cudaStream_t, passed as void*; NULL is the
  *   legacy default stream) and returns without synchronising.  Calls are
  *   thread-safe.  Input buffers must not be modified, and outputs not read,
- *   until the stream has reached the call.  The chunked prefill forks one of
- *   its kernels onto a library-owned side stream and joins it back with events
- *   (one non-blocking, lowest-priority stream and two events per device,
- *   created by the first such call on that device and kept until exit); the
- *   call stays ordered on `stream` as a whole, and a CUDA graph captured from
- *   `stream` records the fork and the join.  Make the first call on a device
- *   outside stream capture.
+ *   until the stream has reached the call.  The first call of an entry point
+ *   in a process sets kernel attributes (host-side, once); make it outside
+ *   stream capture.  Later calls only enqueue kernels, so a CUDA graph
+ *   captured from `stream` replays them.
  *
  * ALIASING
  *   final_state may equal initial_state (updated in place).  No other output
@@ -111,9 +108,9 @@ size_t rda_prefill_workspace_bytes(int B, int T, int H, int Dk, int Dv, int num_
  *
  * Defined by the gated delta rule above; the chunked form it uses reaches the
  * same result up to rounding: 64-token chunks, a UT transform of each chunk
- * and its products on the tensor cores (chunk-parallel), a sequential scan of
- * the fp32 state across chunks, then the outputs (chunk-parallel; their
- * chunk-local operands are computed on the side stream meanwhile).  bf16
+ * and its products on the tensor cores, with the chunk-local operands of the
+ * outputs (chunk-parallel), then a sequential scan of the fp32 state across
+ * chunks that also produces the outputs.  bf16
  * inputs take this path when Dk = 128; fp32 inputs, and bf16 with Dk = 64,
  * take a token-sequential fp32 path (fp32 inputs are held to fp32 accuracy,
  * which bf16 tensor-core operands cannot give).  Several kernels are

@@ -1,10 +1,9 @@
 """Prefill calls on several streams, from several host threads, and replayed
 from a captured CUDA graph.
 
-One prefill call enqueues kernels on the caller's stream and forks one of them
-onto a library-owned side stream, joined back with an event before the output
-kernel.  These checks run calls that overlap on the GPU (each with its own
-workspace) and compare every result bit for bit with the same call run alone:
+One prefill call enqueues its kernels on the caller's stream only.  These
+checks run calls that overlap on the GPU (each with its own workspace) and
+compare every result bit for bit with the same call run alone:
 the kernels are deterministic, so any cross-call interference shows as a
 mismatch.  The single-call results are themselves checked against the fp64
 oracle.
@@ -92,8 +91,8 @@ def test_calls_from_two_host_threads(cuda_device):
 
 
 def test_graph_capture_and_replay(cuda_device):
-    """The fork onto the side stream and the join are events, which stream
-    capture records; the replayed graph gives the eager result."""
+    """A captured call (kernel launches only, no host work inside) replays to
+    the eager result."""
     import gated_delta_rule_rda_b200 as rda
     d = _inputs(1)[0]
     ref = _alone(rda, [d])[0]
@@ -101,7 +100,7 @@ def test_graph_capture_and_replay(cuda_device):
     out = torch.empty_like(ref[0])
     sf = torch.empty_like(ref[1])
     st = torch.cuda.Stream()
-    with torch.cuda.stream(st):      # first call outside capture (creates the side stream)
+    with torch.cuda.stream(st):      # first call outside capture (one-time setup: kernel attributes)
         rda.rda_prefill_chunked(d.q, d.k, d.v, d.log_alpha, d.beta, write_gate=d.gamma,
                                 initial_state=d.initial_state, out=out, final_state=sf, workspace=ws)
     st.synchronize()
