@@ -435,6 +435,9 @@ __global__ void __launch_bounds__(kPrepThreads, 4)
 prep_kernel(const __grid_constant__ PrepMaps maps, const PrefillArgs a) {
     extern __shared__ uint8_t smem_raw[];
     uint8_t *sm = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    // the scan may launch (and run its prologue) once every prep CTA has started;
+    // it waits for this grid's completion before it reads the workspace
+    if (threadIdx.x == 0) pdl_launch_dependents();
     ChunkLoc loc;
     if (!locate_chunk(a, blockIdx.x, loc)) return;     // uniform across the CTA
     const long gc = loc.gc;
@@ -846,6 +849,7 @@ scan_kernel(const __grid_constant__ ScanMaps maps, const PrefillArgs a) {
     if (warp == kScanWarps) {
         // ------------------------------------------------------------ producer
         if (lane == 0) {
+            pdl_wait_primary();      // the prep's images are complete and visible
             for (int c = 0; c < nchunks; ++c) {
                 const int st = c % kScanStages;
                 if (c >= kScanStages &&
@@ -1151,8 +1155,19 @@ cudaError_t launch_nv(const PrefillArgs &a, long chunks_grid, cudaStream_t s) {
         prep_kernel<NV><<<chunk_grid, kPrepThreads, kPrepSmem, s>>>(pm, a);
         if ((e = cudaGetLastError()) != cudaSuccess) return e;
     }
-    scan_kernel<NV><<<scan_grid, kScanThreads, scan_smem, s>>>(sm, a);
-    return cudaGetLastError();
+    // programmatic stream serialization: the scan's launch and prologue overlap
+    // the prep's last CTAs; only its producer waits for the prep to complete
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = scan_grid;
+    cfg.blockDim = dim3(kScanThreads, 1, 1);
+    cfg.dynamicSmemBytes = scan_smem;
+    cfg.stream = s;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = chunks_grid > 0 ? 1 : 0;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, scan_kernel<NV>, sm, a);
 }
 
 size_t image_bytes(int Dv) { return (size_t)kImgU + 64 * (size_t)Dv * 2 + 512; }
