@@ -22,16 +22,16 @@
 //  1. prep (chunk-parallel; one CTA per (chunk, head) over every chunk of
 //     every sequence at once): everything the state chain and the outputs
 //     need from a chunk.  g, K K^T and Q K^T on the tensor cores, A and P from
-//     them, diag(e^g) Q, the UT transform (diagonal 16x16 blocks by forward
-//     substitution, off-diagonal blocks by recursive doubling on tf32
-//     mma.sync), then W and U' on the tensor cores.  Writes -W, diag(e^g) Q
-//     and P as ready-to-use swizzled operand images, U' in value slices and
-//     the decay factors.  Four CTAs per SM (55 KiB of shared memory, 128 TMEM
+//     them, the UT transform (diagonal 16x16 blocks by forward substitution,
+//     off-diagonal blocks by recursive doubling on tf32 mma.sync), then W and
+//     U' on the tensor cores.  Writes -W and P as ready-to-use swizzled
+//     operand images, U' in value slices and the decay factors.  Four CTAs per SM (55 KiB of shared memory, 128 TMEM
 //     columns each): the Q, K, V, A and T tiles share three regions in turn.
 //  2. scan (sequential over the chunks of one (sequence, head, value slice)).
 //     Carries the fp32 state in registers; per chunk U = U' - W S and the
-//     outputs O = scale (diag(e^g) Q S + P U) -- the two products with S share
-//     its operand fragments -- then S <- e^{g_C} S + K^T diag(e^{g_C - g}) U, on
+//     outputs O = scale (diag(e^g) (Q S) + P U) -- the two products with S
+//     share its operand fragments; Q comes from the input by TMA -- then
+//     S <- e^{g_C} S + K^T diag(e^{g_C - g}) U, on
 //     register-fragment MMAs.  Value columns are independent under the rule,
 //     so slicing is exact.
 //
@@ -60,9 +60,8 @@ constexpr uint64_t kWaitNs = 4000000000ull;   // bounded waits: 4 s
 
 // Per (chunk, head) image in the workspace (bytes).
 constexpr uint32_t kImgW = 0;          // -W, bf16 K-major SW128, 2 halves of 8 KiB (64 rows x 64 cols)
-constexpr uint32_t kImgQ = 16384;      // diag(e^g) Q, same layout
-constexpr uint32_t kImgP = 32768;      // P, bf16 K-major SW128, 8 KiB
-constexpr uint32_t kImgU = 40960;      // U', bf16, value slices of width NV, each [64][NV];
+constexpr uint32_t kImgP = 16384;      // P, bf16 K-major SW128, 8 KiB
+constexpr uint32_t kImgU = 24576;      // U', bf16, value slices of width NV, each [64][NV];
                                        // then e^{g_t} and e^{g_C - g_t}: 2 x 64 fp32
 
 __device__ __forceinline__ uint64_t globaltimer() {
@@ -290,8 +289,8 @@ __device__ __forceinline__ void ut_solve(float *Af, float *Tf, float *Xs, int cw
 // ---------------------------------------------------------------------------
 // Kernel 1: prep.  One CTA per (global chunk, head): everything the scan
 // needs from a chunk -- g, A from K K^T, the UT transform T, then W and U' --
-// and the chunk-local operands of the outputs, P = (Q K^T) o Gamma (causal,
-// diagonal kept) and diag(e^g) Q.
+// and the chunk-local operand of the outputs, P = (Q K^T) o Gamma (causal,
+// diagonal kept).
 // Four CTAs share an SM (shared memory <= 55 KiB, 128 TMEM columns, <= 96
 // registers): three regions are reused as the chunk's work moves along.
 // ---------------------------------------------------------------------------
@@ -578,21 +577,6 @@ prep_kernel(const __grid_constant__ PrepMaps maps, const PrefillArgs a) {
                 *reinterpret_cast<uint32_t *>(pi + swz(ta, kb, 128)) = pack_bf16(v[4 * kb], v[4 * kb + 1]);
                 *reinterpret_cast<uint32_t *>(pi + swz(ta + 8, kb, 128)) = pack_bf16(v[4 * kb + 2], v[4 * kb + 3]);
             }
-            // diag(e^g) Q: the same byte layout as the loaded Q tile; 16-byte pieces,
-            // consecutive threads on consecutive pieces
-#pragma unroll
-            for (int k = 0; k < 8; ++k) {
-                const uint32_t off = 16u * (uint32_t)(cw + 128 * k);
-                const float e = eg_s[(off & 8191u) >> 7];
-                const uint4 u = *reinterpret_cast<const uint4 *>(sm + PS_Q + off);
-                uint32_t wv[4] = {u.x, u.y, u.z, u.w};
-#pragma unroll
-                for (int i = 0; i < 4; ++i) {
-                    const float2 f = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(&wv[i]));
-                    wv[i] = pack_bf16(f.x * e, f.y * e);
-                }
-                *reinterpret_cast<uint4 *>(img + kImgQ + off) = make_uint4(wv[0], wv[1], wv[2], wv[3]);
-            }
             tc_fence_before();
         }
         named_bar_sync(1, 128);      // Q is dead: T goes there
@@ -707,20 +691,20 @@ prep_kernel(const __grid_constant__ PrepMaps maps, const PrefillArgs a) {
 // time whatever its size, plus a commit round trip, so this latency-bound
 // chain runs on register-fragment tensor-core MMAs (mma.sync m16n8k16, bf16
 // in, fp32 accumulate) with ldmatrix operands.  The outputs of the chunk's
-// rows come out of the same pass: diag(e^g) Q S with the operand fragments of
-// S that U uses, and P U once U is in shared memory.
+// rows come out of the same pass: Q S with the operand fragments of S that U
+// uses (rows then scaled by e^{g_t}), and P U once U is in shared memory.
 //   warps 0..3  warp w owns key rows 32w..32w+31 of the fp32 state (as
 //               accumulator fragments) and token rows 16w..16w+15 of U and O,
 //               across the slice's NV value columns (splitting the columns
 //               over twice the warps doubles the operand traffic through
 //               shared memory and measured slower)
-//   warp 4      producer: the K tile by TMA, -W, diag(e^g) Q, P, U' and the
-//               decay factors by bulk copies, into a 3-stage ring.
+//   warp 4      producer: the K and Q tiles by TMA, -W, P, U' and the decay
+//               factors by bulk copies, into a 3-stage ring.
 // ---------------------------------------------------------------------------
 constexpr int kScanWarps = 4;
 constexpr int kScanThreads = (kScanWarps + 1) * 32;
 constexpr int kScanStages = 3;
-// per-stage shared memory (bytes): -W 16K | K 16K | diag(e^g) Q 16K | P 8K | U' <= 4K | decay 512
+// per-stage shared memory (bytes): -W 16K | K 16K | Q 16K | P 8K | U' <= 4K | decay 512
 constexpr uint32_t SS_W = 0, SS_K = 16384, SS_Q = 32768, SS_P = 49152, SS_U = 57344, SS_G = 61440;
 constexpr uint32_t SS_STAGE = 62464;                          // multiple of 1024
 enum ScanBar { SB_FULL = 0, SB_EMPTY = kScanStages, kScanBars = 2 * kScanStages };
@@ -736,7 +720,7 @@ template <int NV> struct ScanSmem {
 };
 
 struct ScanMaps {
-    CUtensorMap k;
+    CUtensorMap k, q;
 };
 
 __device__ __forceinline__ void ldsm_x4(uint32_t addr, uint32_t *r) {
@@ -863,7 +847,8 @@ scan_kernel(const __grid_constant__ ScanMaps maps, const PrefillArgs a) {
                 tma_load_3d(stg + SS_K, &maps.k, full, 0, h, r0);
                 tma_load_3d(stg + SS_K + 8192, &maps.k, full, 64, h, r0);
                 bulk_load(stg + SS_W, img + kImgW, 16384, full);
-                bulk_load(stg + SS_Q, img + kImgQ, 16384, full);
+                tma_load_3d(stg + SS_Q, &maps.q, full, 0, h, r0);
+                tma_load_3d(stg + SS_Q + 8192, &maps.q, full, 64, h, r0);
                 bulk_load(stg + SS_P, img + kImgP, 8192, full);
                 bulk_load(stg + SS_U, img + kImgU + (size_t)slice * UBYTES, UBYTES, full);
                 bulk_load(stg + SS_G, img + kImgU + 64 * Dv * 2, 512, full);
@@ -924,8 +909,8 @@ scan_kernel(const __grid_constant__ ScanMaps maps, const PrefillArgs a) {
             acc[0][nt][0] = fa.x; acc[0][nt][1] = fa.y; acc[0][nt][2] = fb.x; acc[0][nt][3] = fb.y;
             acc[1][nt][0] = acc[1][nt][1] = acc[1][nt][2] = acc[1][nt][3] = 0.f;
         }
-        // O = diag(e^g) Q S_c (+ P U below) for the same rows: it shares the state
-        // operand fragments with U
+        // O = diag(e^g) (Q S_c) (+ P U below) for the same rows: Q S_c shares the
+        // state operand fragments with U
         float ao[NT][4];
 #pragma unroll
         for (int nt = 0; nt < NT; ++nt) ao[nt][0] = ao[nt][1] = ao[nt][2] = ao[nt][3] = 0.f;
@@ -948,6 +933,16 @@ scan_kernel(const __grid_constant__ ScanMaps maps, const PrefillArgs a) {
                     mma16816(acc[kk & 1][nt], af[kk], bf[kk][2 * nt], bf[kk][2 * nt + 1]);
                     mma16816(ao[nt], aq[kk], bf[kk][2 * nt], bf[kk][2 * nt + 1]);
                 }
+        }
+        {
+            const float ea = eg_s[ta], eb = eg_s[tb];     // e^{g_t}
+#pragma unroll
+            for (int nt = 0; nt < NT; ++nt) {
+                ao[nt][0] *= ea;
+                ao[nt][1] *= ea;
+                ao[nt][2] *= eb;
+                ao[nt][3] *= eb;
+            }
         }
         // ---- U and U~ = e^{g_C - g_t} U -> shared memory (B operands of P U and K^T U~)
         const float da = ed_s[ta], db = ed_s[tb];
@@ -1146,6 +1141,7 @@ cudaError_t launch_nv(const PrefillArgs &a, long chunks_grid, cudaStream_t s) {
             !make_map(&pm.v, a.v, a.Dv, a.H, a.total_T, 64))
             return cudaErrorInvalidValue;
         sm.k = pm.k;
+        sm.q = pm.q;
     }
     const dim3 scan_grid(a.Dv / NV, a.H, a.num_seqs);
     const uint32_t scan_smem = ScanSmem<NV>::BYTES;

@@ -18,7 +18,7 @@
 namespace {
 
 // Largest scratch this entry point can use, bytes: enough for the chunked
-// path's per-chunk images of about 1,150 (chunk, head) pairs at Dv = 128,
+// path's per-chunk images of about 1,600 (chunk, head) pairs at Dv = 128,
 // e.g. B = 1, T = 4096, H = 16.
 constexpr size_t kNoAllocScratchBytes = size_t(64) << 20;
 

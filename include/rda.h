@@ -95,8 +95,8 @@ const char *rda_version(void);
  * rda_prefill_varlen (num_seqs = N, pass B = 1 and T = total_T) needs for
  * these sizes, enough for either dtype.  Always >= 256: the first 256 bytes
  * hold the device error word.  When the chunked tensor-core path can run
- * (Dk = 128) it also holds that path's per-chunk scratch, about 56.5 KiB
- * per 64-token chunk and head at Dv = 128 (e.g. 59 MB for B=1, T=4096, H=16).
+ * (Dk = 128) it also holds that path's per-chunk scratch, about 40.5 KiB
+ * per 64-token chunk and head at Dv = 128 (e.g. 42 MB for B=1, T=4096, H=16).
  * The workspace must be 256-byte aligned; its contents need no
  * initialisation beyond a cleared error word, and are overwritten by each
  * call.  Returns 0 for unsupported sizes.
@@ -215,7 +215,7 @@ rda_status_t rda_decode_tokens(const void *q, const void *k, const void *v,
  * this library holds until the process exits.  Problems whose
  * rda_prefill_workspace_bytes(B,T,H,Dk,Dv,0) exceeds 64 MiB are rejected with
  * RDA_ERR_WORKSPACE before anything is enqueued (at Dv = 128 the limit is
- * about 1,150 chunk-head pairs, e.g. B = 1, T = 4096, H = 16).  The first call on
+ * about 1,600 chunk-head pairs, e.g. B = 1, T = 4096, H = 16).  The first call on
  * a device looks up the array's device address; make that first call before
  * any stream capture.  All calls on a device share the array, which keeps the
  * last call's contents: calls whose work overlaps on the GPU (unordered
