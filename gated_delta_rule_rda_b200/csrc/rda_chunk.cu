@@ -360,18 +360,28 @@ __device__ __forceinline__ bool locate_chunk(const PrefillArgs &a, long idx, Chu
     return true;
 }
 
-// Gates of one chunk, by the 128 compute threads (r = 0..127): g = cumsum of
-// log alpha (masked past the end), beta, beta*gamma and the decay factors.
-// Ends with a barrier of the compute threads.
-__device__ __forceinline__ void chunk_gates(const PrefillArgs &a, long row0, int lenc, int h, int r, int lane,
-                                            float *g_s) {
+// Row r's gates (r < 64; zero decay and strength past the chunk's end).
+struct RowGates {
+    float la, be, ga;
+};
+__device__ __forceinline__ RowGates load_gates(const PrefillArgs &a, long row0, int lenc, int h, int r) {
+    RowGates x{0.f, 0.f, 1.f};
+    if (r < 64 && r < lenc) {
+        const size_t row = (size_t)(row0 + r) * a.H + h;
+        x.la = a.log_alpha[row];
+        x.be = a.beta[row];
+        if (a.gamma) x.ga = a.gamma[row];
+    }
+    return x;
+}
+// Gates of one chunk, by the 128 compute threads (r = 0..127), from the rows'
+// loaded gates: g = cumsum of log alpha (masked past the end), beta,
+// beta*gamma and the decay factors.  Ends with a barrier of the compute threads.
+__device__ __forceinline__ void chunk_gates(RowGates x, int r, int lane, float *g_s) {
     float *b_s = g_s + 64, *bg_s = g_s + 128, *eb_s = g_s + 192, *eg_s = g_s + 256, *ed_s = g_s + 320;
     if (r < 64) {
-        const bool valid = r < lenc;
-        const size_t row = (size_t)(row0 + r) * a.H + h;
-        float la = valid ? a.log_alpha[row] : 0.f;
-        const float be = valid ? a.beta[row] : 0.f;
-        const float ga = (valid && a.gamma) ? a.gamma[row] : 1.f;
+        float la = x.la;
+        const float be = x.be, ga = x.ga;
 #pragma unroll
         for (int off = 1; off < 32; off <<= 1) {
             const float y = __shfl_up_sync(0xffffffffu, la, off);
@@ -444,6 +454,12 @@ prep_kernel(const __grid_constant__ PrepMaps maps, const PrefillArgs a) {
     const int H = a.H, Dv = a.Dv;
     const int lenc = (int)min((long)kC, loc.len - (long)loc.c * kC);
     const long row0 = loc.t0 + (long)loc.c * kC;
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    // the compute threads' gate loads go out before the setup below (their
+    // latency is the first thing a chunk waits for)
+    const int q4 = warp & 3;
+    const int r = 32 * q4 + lane;              // TMEM lane of a compute thread
+    const RowGates gates = warp > 0 ? load_gates(a, row0, lenc, h, r) : RowGates{0.f, 0.f, 1.f};
 
     uint64_t *bars = reinterpret_cast<uint64_t *>(sm + PS_BAR);
     uint32_t *tmem_ptr = reinterpret_cast<uint32_t *>(sm + PS_TMEMPTR);
@@ -451,7 +467,6 @@ prep_kernel(const __grid_constant__ PrepMaps maps, const PrefillArgs a) {
     volatile int *agent_flag = abort_flag + 1;
     float *g_s = reinterpret_cast<float *>(sm + PS_G);
     const float *b_s = g_s + 64, *bg_s = g_s + 128, *eg_s = g_s + 256;
-    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
 
     if (threadIdx.x == 0) {
         for (int i = 0; i < kPrepBars; ++i) mbar_init(&bars[i], 1);
@@ -535,8 +550,6 @@ prep_kernel(const __grid_constant__ PrepMaps maps, const PrefillArgs a) {
         }
     } else {
         const int cw = threadIdx.x - 32;
-        const int q4 = warp & 3;
-        const int r = 32 * q4 + lane;              // TMEM lane
         // rows ta, ta + 8 and column pairs 8 kb + j2 of the M=64 accumulators (16x256b loads)
         const int ta = 16 * q4 + (lane >> 2), j2 = 2 * (lane & 3);
         const uint32_t tq = tmem + ((uint32_t)(32 * q4) << 16);
@@ -544,7 +557,7 @@ prep_kernel(const __grid_constant__ PrepMaps maps, const PrefillArgs a) {
         float *Tf = reinterpret_cast<float *>(sm + PS_TF);
         float *Xs = reinterpret_cast<float *>(sm + PS_XS);
 
-        chunk_gates(a, row0, lenc, h, r, lane, g_s);
+        chunk_gates(gates, r, lane, g_s);
         if (cw == 0 && !wait_bar(&bars[PB_KK], 0, abort_flag, a.err)) *abort_flag = 1;
         named_bar_sync(1, 128);
         if (!*abort_flag) {
