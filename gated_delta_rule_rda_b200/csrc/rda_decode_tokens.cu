@@ -17,7 +17,11 @@
 //     o_t = scale (c_t b_t + sum_{i<=t} w_i (k_i . q_t))
 // and the new state is written once: S_new = c_T S_old + sum_i w_i k_i^T.
 // The state is read and written once whatever T is, so T tokens cost about
-// the HBM time of one decode step.
+// the HBM time of one decode step.  From three tokens (at Dk = Dv = 128) the
+// products with the state and its update run on tf32 tensor-core MMAs with
+// split operands (fp32 accuracy); below that, on paired fp32 FMAs.
+#include <type_traits>
+
 #include "rda_internal.h"
 #include "rda_io.cuh"
 
@@ -170,6 +174,214 @@ decode_tokens_kernel(DecodeArgs a) {
     }
 }
 
+// ---------------------------------------------------------------------------
+// Dk = Dv = 128 on the tensor cores.  Warp w holds value columns
+// j0 = 16w .. 16w+15 of the state for every key dim, in the accumulator layout
+// of an m16n8k8 tf32 MMA whose rows are value columns (row m <-> column
+// j0 + 2(m%8) + m/8) and whose columns are key dims: for key block nb
+// (dims 8nb .. 8nb+7), with d = 8nb + 2tg and j = j0 + 2g (g = lane/4, tg = lane%4),
+//     s[nb] = { S[d][j], S[d+1][j], S[d][j+1], S[d+1][j+1] }
+// so that each thread moves the state in pairs of adjacent columns.  The same
+// registers, in the order {0, 2, 1, 3}, are the A operand of the products with
+// the new keys and queries when the reduction index of block nb is read in the
+// order 0,2,4,6,1,3,5,7 (A column tg is key dim d, column tg+4 is d+1; the B rows
+// follow the same order), and the accumulator of the update
+// S_new^T = c S^T + W K (M = value columns, K = tokens, N = key dims).  fp32
+// accuracy from tf32 MMAs: every fp32 operand is split into a tf32 head and a
+// tf32 tail (x = hi + lo + O(2^-22 |x|)) and hi*hi + lo*hi + hi*lo are
+// accumulated in fp32; bf16 keys and queries are exact in tf32 (no tail).
+// ---------------------------------------------------------------------------
+constexpr int kTcD = 128;
+constexpr int kTcKP = kTcD + 8;     // row stride of the key / query rows (conflict-free float2 B loads)
+constexpr int kTcWP = kTcD + 4;     // row stride of the coefficient rows
+
+__device__ __forceinline__ uint32_t tf32_of(float x) {
+    uint32_t r;
+    asm("cvt.rna.tf32.f32 %0, %1;" : "=r"(r) : "f"(x));
+    return r;
+}
+__device__ __forceinline__ void split_tf32(float x, uint32_t &hi, uint32_t &lo) {
+    hi = tf32_of(x);
+    lo = tf32_of(x - __uint_as_float(hi));
+}
+// D += A(16x8, row) * B(8x8, col), tf32 inputs, fp32 accumulate.
+__device__ __forceinline__ void mma_tf32_m16n8k8(float *d, uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3,
+                                                 uint32_t b0, uint32_t b1) {
+    asm volatile(
+        "mma.sync.aligned.m16n8k8.row.col.f32.tf32.tf32.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
+        "{%0,%1,%2,%3};"
+        : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+        : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
+}
+// acc += a * b for an fp32 A fragment and a B fragment given as tf32 head / tail
+// (no tail when EXACT_B).
+template <bool EXACT_B>
+__device__ __forceinline__ void mma_f32_split(float *acc, const float *a, uint32_t bh0, uint32_t bh1, uint32_t bl0,
+                                              uint32_t bl1) {
+    uint32_t ah[4], al[4];
+#pragma unroll
+    for (int i = 0; i < 4; ++i) split_tf32(a[i], ah[i], al[i]);
+    mma_tf32_m16n8k8(acc, ah[0], ah[1], ah[2], ah[3], bh0, bh1);
+    mma_tf32_m16n8k8(acc, al[0], al[1], al[2], al[3], bh0, bh1);
+    if (!EXACT_B) mma_tf32_m16n8k8(acc, ah[0], ah[1], ah[2], ah[3], bl0, bl1);
+}
+
+template <typename Tio>
+__global__ void __launch_bounds__(kThreads, 2)
+decode_tokens_tc_kernel(DecodeArgs a) {
+    constexpr int D = kTcD;
+    constexpr bool kExact = !std::is_same<Tio, float>::value;    // bf16 keys / queries are tf32-exact
+    __shared__ __align__(16) float k_s[kMaxT][kTcKP];      // k_t[d], rows past T zero
+    __shared__ __align__(16) float q_s[kMaxT][kTcKP];
+    __shared__ float v_s[kMaxT][D];                        // v_t (times gamma_t below)
+    __shared__ __align__(16) float ab_s[2][kMaxT][D];      // a_t = s_0 . k_t, b_t = s_0 . q_t per column
+    __shared__ float w_s[kMaxT][kTcWP];                    // final coefficients w_t per column, rows past T zero
+    __shared__ float gp_s[kThreads / 32][2][kMaxT][kMaxT]; // Gram partials per warp (16 key dims each)
+    __shared__ float kk_s[kMaxT][kMaxT];                   // [i][t] = k_i . k_t
+    __shared__ float kq_s[kMaxT][kMaxT];                   // [i][t] = k_i . q_t
+    __shared__ float g_s[3][kMaxT];                        // alpha, beta, gamma
+    __shared__ float c_s;
+
+    const int T = a.T, H = a.H;
+    const int bh = blockIdx.x, b = bh / H, h = bh % H;
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int g = lane >> 2, tg = lane & 3;
+    const int jc = 16 * warp + 2 * g;                      // this thread's column pair
+    float *st = a.state + (size_t)bh * D * D;
+    auto tok = [&](int t) { return ((size_t)b * T + t) * H + h; };
+
+    // the state reads first (each instruction: 4 rows x 64 contiguous bytes)
+    float s[16][4];
+#pragma unroll
+    for (int nb = 0; nb < 16; ++nb) {
+        const float *p = st + (size_t)(8 * nb + 2 * tg) * D + jc;
+        const float2 r0 = __ldcs(reinterpret_cast<const float2 *>(p));
+        const float2 r1 = __ldcs(reinterpret_cast<const float2 *>(p + D));
+        s[nb][0] = r0.x;
+        s[nb][2] = r0.y;
+        s[nb][1] = r1.x;
+        s[nb][3] = r1.y;
+    }
+    if (threadIdx.x < kMaxT) {
+        const int t = threadIdx.x;
+        const bool live = t < T;
+        g_s[0][t] = live ? expf(a.log_alpha[tok(t)]) : 1.f;
+        g_s[1][t] = live ? a.beta[tok(t)] : 0.f;
+        g_s[2][t] = live && a.gamma ? a.gamma[tok(t)] : 1.f;
+    }
+    for (int i = threadIdx.x; i < kMaxT * D; i += kThreads) {
+        const int t = i / D, d = i % D;
+        const bool live = t < T;
+        k_s[t][d] = live ? Io<Tio>::ld(static_cast<const Tio *>(a.k) + tok(t) * D + d) : 0.f;
+        q_s[t][d] = live ? Io<Tio>::ld(static_cast<const Tio *>(a.q) + tok(t) * D + d) : 0.f;
+        if (live) v_s[t][d] = Io<Tio>::ld(static_cast<const Tio *>(a.v) + tok(t) * D + d);
+    }
+    __syncthreads();
+
+    {
+        // a_t and b_t for this warp's 16 columns: S^T [k q] over the 128 key dims
+        // (B column n = token g; rows of block nb in the order of the A columns)
+        float pk[4] = {0.f, 0.f, 0.f, 0.f}, pq[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+        for (int nb = 0; nb < 16; ++nb) {
+            const float af[4] = {s[nb][0], s[nb][2], s[nb][1], s[nb][3]};
+            const float2 kb = *reinterpret_cast<const float2 *>(&k_s[g][8 * nb + 2 * tg]);
+            const float2 qb = *reinterpret_cast<const float2 *>(&q_s[g][8 * nb + 2 * tg]);
+            uint32_t kh0, kl0, kh1, kl1, qh0, ql0, qh1, ql1;
+            split_tf32(kb.x, kh0, kl0);
+            split_tf32(kb.y, kh1, kl1);
+            split_tf32(qb.x, qh0, ql0);
+            split_tf32(qb.y, qh1, ql1);
+            mma_f32_split<kExact>(pk, af, kh0, kh1, kl0, kl1);
+            mma_f32_split<kExact>(pq, af, qh0, qh1, ql0, ql1);
+        }
+        // accumulator: column jc (+1), token 2tg (+1)
+        if (2 * tg < T) {
+            ab_s[0][2 * tg][jc] = pk[0];
+            ab_s[0][2 * tg][jc + 1] = pk[2];
+            ab_s[1][2 * tg][jc] = pq[0];
+            ab_s[1][2 * tg][jc + 1] = pq[2];
+        }
+        if (2 * tg + 1 < T) {
+            ab_s[0][2 * tg + 1][jc] = pk[1];
+            ab_s[0][2 * tg + 1][jc + 1] = pk[3];
+            ab_s[1][2 * tg + 1][jc] = pq[1];
+            ab_s[1][2 * tg + 1][jc + 1] = pq[3];
+        }
+        // token Gram values over this warp's 16 key dims: K [K Q]^T (A rows = tokens
+        // g; rows g + 8 zero)
+        float gk[4] = {0.f, 0.f, 0.f, 0.f}, gq[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+        for (int ks = 2 * warp; ks < 2 * warp + 2; ++ks) {
+            const float af[4] = {k_s[g][8 * ks + tg], 0.f, k_s[g][8 * ks + tg + 4], 0.f};
+            uint32_t kh0, kl0, kh1, kl1, qh0, ql0, qh1, ql1;
+            split_tf32(k_s[g][8 * ks + tg], kh0, kl0);
+            split_tf32(k_s[g][8 * ks + tg + 4], kh1, kl1);
+            split_tf32(q_s[g][8 * ks + tg], qh0, ql0);
+            split_tf32(q_s[g][8 * ks + tg + 4], qh1, ql1);
+            mma_f32_split<kExact>(gk, af, kh0, kh1, kl0, kl1);
+            mma_f32_split<kExact>(gq, af, qh0, qh1, ql0, ql1);
+        }
+        gp_s[warp][0][g][2 * tg] = gk[0];
+        gp_s[warp][0][g][2 * tg + 1] = gk[1];
+        gp_s[warp][1][g][2 * tg] = gq[0];
+        gp_s[warp][1][g][2 * tg + 1] = gq[1];
+    }
+    __syncthreads();
+    if (threadIdx.x < 2 * kMaxT * kMaxT) {
+        const int which = threadIdx.x >> 6, i = (threadIdx.x >> 3) & 7, t = threadIdx.x & 7;
+        float x = 0.f;
+#pragma unroll
+        for (int w = 0; w < kThreads / 32; ++w) x += gp_s[w][which][i][t];
+        (which ? kq_s : kk_s)[i][t] = x;
+    }
+    __syncthreads();
+
+    // the token recurrence, one value column per thread
+    if (threadIdx.x < D) {
+        const int j = threadIdx.x;
+        float c = 1.f;
+        float w[kMaxT];
+#pragma unroll
+        for (int t = 0; t < kMaxT; ++t) {
+            if (t >= T) break;
+            float p = c * ab_s[0][t][j];
+#pragma unroll
+            for (int i = 0; i < t; ++i) p = fmaf(w[i], kk_s[i][t], p);
+            const float al = g_s[0][t];
+#pragma unroll
+            for (int i = 0; i < t; ++i) w[i] *= al;
+            w[t] = g_s[1][t] * (g_s[2][t] * v_s[t][j] - al * p);
+            c *= al;
+            float o = c * ab_s[1][t][j];
+#pragma unroll
+            for (int i = 0; i <= t; ++i) o = fmaf(w[i], kq_s[i][t], o);
+            Io<Tio>::st(static_cast<Tio *>(a.out) + tok(t) * D + j, a.scale * o);
+        }
+#pragma unroll
+        for (int t = 0; t < kMaxT; ++t) w_s[t][j] = t < T ? w[t] : 0.f;
+        if (j == 0) c_s = c;
+    }
+    __syncthreads();
+
+    // S_new^T = c S^T + W K: A = W (value columns x tokens), B = K (tokens x key
+    // dims), accumulated into the state registers
+    const float c = c_s;
+    const float wf[4] = {w_s[tg][jc], w_s[tg][jc + 1], w_s[tg + 4][jc], w_s[tg + 4][jc + 1]};
+#pragma unroll
+    for (int nb = 0; nb < 16; ++nb) {
+        uint32_t bh0, bl0, bh1, bl1;
+        split_tf32(k_s[tg][8 * nb + g], bh0, bl0);
+        split_tf32(k_s[tg + 4][8 * nb + g], bh1, bl1);
+#pragma unroll
+        for (int i = 0; i < 4; ++i) s[nb][i] *= c;
+        mma_f32_split<kExact>(s[nb], wf, bh0, bh1, bl0, bl1);
+        float *p = st + (size_t)(8 * nb + 2 * tg) * D + jc;
+        __stcs(reinterpret_cast<float2 *>(p), make_float2(s[nb][0], s[nb][2]));
+        __stcs(reinterpret_cast<float2 *>(p + D), make_float2(s[nb][1], s[nb][3]));
+    }
+}
+
 template <typename Tio, int DK, int DV>
 cudaError_t launch_shape(const DecodeArgs &a, cudaStream_t s) {
     constexpr int TPR = DV / 4, RG = kThreads / TPR;
@@ -184,7 +396,13 @@ cudaError_t launch_shape(const DecodeArgs &a, cudaStream_t s) {
 
 template <typename Tio>
 cudaError_t launch_t(const DecodeArgs &a, cudaStream_t s) {
-    if (a.Dk == 128 && a.Dv == 128) return launch_shape<Tio, 128, 128>(a, s);
+    if (a.Dk == 128 && a.Dv == 128) {
+        // one or two tokens: the paired-FMA kernel streams the state in 16-byte
+        // pieces and is faster; from three tokens the products dominate
+        if (a.T <= 2) return launch_shape<Tio, 128, 128>(a, s);
+        decode_tokens_tc_kernel<Tio><<<(unsigned)(a.B * a.H), kThreads, 0, s>>>(a);
+        return cudaGetLastError();
+    }
     if (a.Dk == 128 && a.Dv == 64) return launch_shape<Tio, 128, 64>(a, s);
     if (a.Dk == 64 && a.Dv == 128) return launch_shape<Tio, 64, 128>(a, s);
     return launch_shape<Tio, 64, 64>(a, s);

@@ -34,7 +34,7 @@ def _check(inp, scale=1.0):
 
 
 @pytest.mark.parametrize("dtype", [torch.float32, torch.bfloat16])
-@pytest.mark.parametrize("T", [1, 2, 5, 8])
+@pytest.mark.parametrize("T", [1, 2, 3, 4, 5, 8])
 def test_tokens_d128(cuda_device, dtype, T):
     inp = rda_gen.fixed_inputs(5, T, 4, 128, 128, dtype=dtype, seed=300 + T, s0=True, gamma=True)
     _check(inp, scale=0.5)
