@@ -506,6 +506,29 @@ def run_reference(args):
     }
 
 
+def profile_decode_tokens(T, steps, warmup):
+    """Only the multi-token decode (decode workload shape, T tokens per call):
+    a short, self-contained run for a profiler.  Prints ms per call."""
+    import torch
+    import gated_delta_rule_rda_b200 as rda
+    import rda_gen
+    din = rda_gen.workload("decode_b256_h16_d128_128steps")
+    device = torch.device("cuda", 0)
+    st = din.state.to(device)
+    q, k, v, la, be = [x[0:T].transpose(0, 1).contiguous().to(device)
+                       for x in (din.q, din.k, din.v, din.log_alpha, din.beta)]
+    out = torch.empty((st.shape[0], T, st.shape[1], st.shape[3]), dtype=din.q.dtype, device=device)
+    for _ in range(warmup):
+        rda.rda_decode_tokens(q, k, v, la, be, st, out=out)
+    s, e = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    s.record()
+    for _ in range(steps):
+        rda.rda_decode_tokens(q, k, v, la, be, st, out=out)
+    e.record()
+    torch.cuda.synchronize()
+    print(json.dumps({"decode_tokens_T": T, "ms_per_call": s.elapsed_time(e) / steps}), flush=True)
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -516,9 +539,14 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--all", action="store_true",
                     help="also time the long-context and packed (varlen) prefill workloads")
+    ap.add_argument("--profile-decode-tokens", type=int, default=0, metavar="T",
+                    help="run only the multi-token decode with T tokens per call (for a profiler)")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
+    if args.profile_decode_tokens:
+        profile_decode_tokens(args.profile_decode_tokens, args.steps, args.warmup)
+        return
 
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
