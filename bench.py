@@ -148,6 +148,24 @@ def gpu_id_for(device):
 
 # ------------------------------------------------------------------ our arm
 
+def max_over_ranks(value, device):
+    """The largest of every rank's `value` over the default process group (the
+    job's time is its slowest rank's); `value` itself without one."""
+    import torch
+    import torch.distributed as dist
+    if not (dist.is_available() and dist.is_initialized()) or dist.get_world_size() == 1:
+        return float(value)
+    t = torch.tensor([float(value)], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def whole_job_rate(units_per_rank, world, ms):
+    """Units per second of the whole job: every rank processes `units_per_rank`
+    in `ms` (the max over ranks)."""
+    return units_per_rank * world / (ms * 1e-3)
+
+
 def run_ours(args, rank, world, device):
     import torch
     import gated_delta_rule_rda_b200 as rda
@@ -195,10 +213,7 @@ def run_ours(args, rank, world, device):
         dist.barrier()
     step_ms = [s.elapsed_time(e) for s, e in ev]
     ms_per_step = sum(step_ms) / len(step_ms)
-    if dist:
-        t = torch.tensor([ms_per_step], device=device)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        ms_per_step = float(t.item())
+    ms_per_step = max_over_ranks(ms_per_step, device)
     assert rda.rda_read_device_error(ws) == 0, "device error word set during the benchmark"
 
     # ---- e2e: host (pinned) inputs and outputs, copies inside the timed region.
@@ -251,10 +266,7 @@ def run_ours(args, rank, world, device):
     e1.record(stream)
     torch.cuda.synchronize()
     e2e_ms = e0.elapsed_time(e1) / e2e_steps
-    if dist:
-        t = torch.tensor([e2e_ms], device=device)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        e2e_ms = float(t.item())
+    e2e_ms = max_over_ranks(e2e_ms, device)
     # the pipelined result must match the device-resident run
     assert torch.equal(slots[0]["host_out"], out.cpu()) and torch.equal(slots[1]["host_sf"], sf.cpu()), \
         "end-to-end result differs from the device-resident step"
@@ -284,10 +296,7 @@ def run_ours(args, rank, world, device):
         d1.record(stream)
         torch.cuda.synchronize()
         dms = d0.elapsed_time(d1) / (reps * nsteps)
-        if dist:
-            t = torch.tensor([dms], device=device)
-            dist.all_reduce(t, op=dist.ReduceOp.MAX)
-            dms = float(t.item())
+        dms = max_over_ranks(dms, device)
         Bd = din.q.shape[1]
         bytes_step = Bd * H * decode_bytes_per_seq_head(Dk, Dv, 2)
         hbm, _, _, src = load_peaks()
@@ -315,7 +324,7 @@ def run_ours(args, rank, world, device):
     tflops = alg_flops / (ms_per_step * 1e-3) / 1e12
     return {
         "metric": METRIC,
-        "value": tokens * world / (ms_per_step * 1e-3),
+        "value": whole_job_rate(tokens, world, ms_per_step),
         "unit": "tokens/s",
         "n_gpus": world,
         "steps": args.steps,
@@ -335,7 +344,7 @@ def run_ours(args, rank, world, device):
                      "algorithmic_bytes_per_launch": alg_bytes,
                      "tensor": {"achieved_tflops": tflops, "peak_tflops": tf,
                                 "frac": tflops / tf, "algorithmic_flops_per_launch": alg_flops}},
-        "e2e": {"value": tokens * world / (e2e_ms * 1e-3), "unit": "tokens/s",
+        "e2e": {"value": whole_job_rate(tokens, world, e2e_ms), "unit": "tokens/s",
                 "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms,
                 "pipeline": "2 slots on 2 streams: copies of one step overlap the next step's"},
         "gpu_launches": args.steps * LAUNCHES_PER_PREFILL,
@@ -366,7 +375,7 @@ def other_workloads(device, stream, rank, world, reps=5):
             e.record(stream)
             ts.append((s, e))
         torch.cuda.synchronize()
-        return sorted(a.elapsed_time(b) for a, b in ts)[len(ts) // 2]
+        return max_over_ranks(sorted(a.elapsed_time(b) for a, b in ts)[len(ts) // 2], device)
 
     inp = rda_gen.workload("long_prefill_b1_t32768_h16_d128").to(device)
     B, T, H, Dk = inp.q.shape
