@@ -35,11 +35,12 @@ def load_library(path):
     dp = ctypes.POINTER(ctypes.c_double)
     ip = ctypes.POINTER(ctypes.c_int32)
     lib.rda_oracle_forward.argtypes = [ctypes.c_int] * 5 + [dp] * 9 + [ctypes.c_double, ctypes.c_int]
+    lib.rda_oracle_forward_channel.argtypes = [ctypes.c_int] * 5 + [dp] * 9 + [ctypes.c_double, ctypes.c_int]
     lib.rda_oracle_varlen.argtypes = [ctypes.c_int, ip] + [ctypes.c_int] * 3 + [dp] * 9 + [ctypes.c_double, ctypes.c_int]
     lib.rda_oracle_decode_step.argtypes = [ctypes.c_int] * 4 + [dp] * 8 + [ctypes.c_double, ctypes.c_int]
     lib.rda_oracle_max_threads.argtypes = []
-    for f in (lib.rda_oracle_forward, lib.rda_oracle_varlen, lib.rda_oracle_decode_step,
-              lib.rda_oracle_max_threads):
+    for f in (lib.rda_oracle_forward, lib.rda_oracle_forward_channel, lib.rda_oracle_varlen,
+              lib.rda_oracle_decode_step, lib.rda_oracle_max_threads):
         f.restype = ctypes.c_int
     return lib
 
@@ -76,6 +77,8 @@ def forward(q, k, v, log_alpha, beta, gamma=None, initial_state=None, scale=1.0,
             num_threads=0, lib=None):
     """Token-sequential fp64 recurrence over a fixed-length batch.
 
+    ``log_alpha`` is ``[B,T,H]`` (one decay per token and head) or ``[B,T,H,Dk]``
+    (one per key channel: column i of the state decays by alpha_i).
     Returns ``(out [B,T,H,Dv], final_state [B,H,Dk,Dv])`` as float64 arrays.
     """
     q, k, v = _f64(q), _f64(k), _f64(v)
@@ -83,16 +86,18 @@ def forward(q, k, v, log_alpha, beta, gamma=None, initial_state=None, scale=1.0,
     B, T, H, Dk = q.shape
     Dv = v.shape[-1]
     assert k.shape == q.shape and v.shape == (B, T, H, Dv)
-    assert la.shape == (B, T, H) and be.shape == (B, T, H)
+    per_channel = la.ndim == 4
+    assert la.shape == ((B, T, H, Dk) if per_channel else (B, T, H)) and be.shape == (B, T, H)
     if ga is not None:
         assert ga.shape == (B, T, H)
     if s0 is not None:
         assert s0.shape == (B, H, Dk, Dv)
     out = np.zeros((B, T, H, Dv), np.float64)
     sf = np.zeros((B, H, Dk, Dv), np.float64)
-    rc = _load(lib).rda_oracle_forward(B, T, H, Dk, Dv, _ptr(q), _ptr(k), _ptr(v), _ptr(la),
-                                    _ptr(be), _ptr(ga), _ptr(s0), _ptr(sf), _ptr(out),
-                                    float(scale), int(num_threads))
+    L = _load(lib)
+    fn = L.rda_oracle_forward_channel if per_channel else L.rda_oracle_forward
+    rc = fn(B, T, H, Dk, Dv, _ptr(q), _ptr(k), _ptr(v), _ptr(la), _ptr(be), _ptr(ga), _ptr(s0),
+            _ptr(sf), _ptr(out), float(scale), int(num_threads))
     if rc != 0:
         raise ValueError("oracle.forward: bad arguments")
     return out, sf

@@ -25,6 +25,19 @@ Stacking rows (U: C x Dv, K: C x Dk, V: C x Dv, Q: C x Dk):
     S_C = e^{g_C} S0 + U^T diag(e^{g_C - g}) K.
 
 The unit lower-triangular system is solved with a library triangular solve.
+
+Per-key-channel decay (log alpha per token and key dim; column d of S decays by
+alpha_d): with G_r = sum_{s<=r} log alpha_s a vector over the key dims, the
+same steps give
+
+    S_r = S0 diag(e^{G_r}) + sum_{i<=r} u_i (k_i o e^{G_r - G_i})^T,
+    u_i = beta_i (v_i - S0 (e^{G_i} o k_i) - sum_{j<i} (sum_d k_j[d] k_i[d] e^{G_i[d] - G_j[d]}) u_j),
+
+so A_ri = beta_r sum_d k_r[d] k_i[d] e^{G_r[d] - G_i[d]} (i < r), the right-hand
+side uses K o e^G, O = (Q o e^G) S0^T + P U with P_ri = sum_d q_r[d] k_i[d]
+e^{G_r[d] - G_i[d]} (i <= r), and S_C = S0 diag(e^{G_C}) + U^T (K o e^{G_C - G}).
+The decay Gram is no longer a product of a matrix and a rank-one mask, which is
+what a kernel for this variant has to organise.
 """
 import numpy as np
 from scipy.linalg import solve_triangular
@@ -45,15 +58,34 @@ def _chunk(S0, Q, K, V, la, be, scale):
     return scale * O, S_end
 
 
+def _chunk_channel(S0, Q, K, V, la, be, scale):
+    """One chunk of one head with per-key-channel decay (la: C x Dk)."""
+    C = K.shape[0]
+    G = np.cumsum(la, axis=0)                        # G_r, C x Dk
+    lower_incl = np.tril(np.ones((C, C), dtype=bool))
+    diff = np.where(lower_incl[:, :, None], G[:, None, :] - G[None, :, :], 0.0)   # r, i, d
+    E = np.where(lower_incl[:, :, None], np.exp(diff), 0.0)
+    KK = np.einsum("rd,id,rid->ri", K, K, E)
+    QK = np.einsum("rd,id,rid->ri", Q, K, E)
+    A = np.tril(be[:, None] * KK, -1)
+    rhs = be[:, None] * (V - (K * np.exp(G)) @ S0.T)
+    U = solve_triangular(np.eye(C) + A, rhs, lower=True, unit_diagonal=True)
+    O = (Q * np.exp(G)) @ S0.T + QK @ U
+    S_end = S0 * np.exp(G[-1])[None, :] + U.T @ (K * np.exp(G[-1][None, :] - G))
+    return scale * O, S_end
+
+
 def forward(q, k, v, log_alpha, beta, gamma=None, initial_state=None, scale=1.0,
             chunk=64):
-    """Chunked evaluation; same arguments and returns as :func:`oracle.forward`."""
+    """Chunked evaluation; same arguments and returns as :func:`oracle.forward`
+    (``log_alpha`` ``[B,T,H]``, or ``[B,T,H,Dk]`` for per-key-channel decay)."""
     q = np.asarray(q, np.float64)
     k = np.asarray(k, np.float64)
     v = np.asarray(v, np.float64)
     la = np.asarray(log_alpha, np.float64)
     be = np.asarray(beta, np.float64)
     B, T, H, Dk = q.shape
+    step = _chunk_channel if la.ndim == 4 else _chunk
     Dv = v.shape[-1]
     if gamma is not None:
         v = v * np.asarray(gamma, np.float64)[..., None]
@@ -65,8 +97,8 @@ def forward(q, k, v, log_alpha, beta, gamma=None, initial_state=None, scale=1.0,
                  else np.asarray(initial_state, np.float64)[b, h].T.copy())
             for t0 in range(0, T, chunk):
                 t1 = min(T, t0 + chunk)
-                O, S = _chunk(S, q[b, t0:t1, h], k[b, t0:t1, h], v[b, t0:t1, h],
-                              la[b, t0:t1, h], be[b, t0:t1, h], scale)
+                O, S = step(S, q[b, t0:t1, h], k[b, t0:t1, h], v[b, t0:t1, h],
+                            la[b, t0:t1, h], be[b, t0:t1, h], scale)
                 out[b, t0:t1, h] = O
             sf[b, h] = S.T
     return out, sf

@@ -15,8 +15,11 @@ Test infrastructure only.  Two independent exact evaluations:
 
   products ordered left to right in s.
 
-Here alpha is given directly (a rational), not as its logarithm.  Matrices are
-lists of lists of ``fractions.Fraction``; S is Dv x Dk (math orientation).
+Here alpha is given directly (a rational), not as its logarithm: one per token,
+or one per token and key channel (a list of Dk rationals), in which case the
+decay multiplies column i of S (key dim i) by alpha_i and ``M_s`` becomes
+``diag(alpha_s) (I - beta_s k_s k_s^T)``.  Matrices are lists of lists of
+``fractions.Fraction``; S is Dv x Dk (math orientation).
 """
 from fractions import Fraction
 
@@ -54,18 +57,25 @@ def _matvec(a, x):
     return [sum((a[i][l] * x[l] for l in range(len(x))), Fraction(0)) for i in range(len(a))]
 
 
+def _per_channel(a):
+    return isinstance(a, (list, tuple))
+
+
 def sequential(q, k, v, alpha, beta, S0=None, gamma=None, scale=Fraction(1)):
     """Exact token-sequential recurrence for one head.
 
-    q, k: T lists of Dk Fractions; v: T lists of Dv; alpha, beta, gamma: T
-    Fractions.  Returns ``(outs, S)`` with outs a T-list of Dv-lists and S the
-    final Dv x Dk state.
+    q, k: T lists of Dk Fractions; v: T lists of Dv; beta, gamma: T Fractions;
+    alpha: T Fractions, or T lists of Dk Fractions (per key channel).  Returns
+    ``(outs, S)`` with outs a T-list of Dv-lists and S the final Dv x Dk state.
     """
     T, Dk, Dv = len(k), len(k[0]), len(v[0])
     S = [row[:] for row in S0] if S0 is not None else _zeros(Dv, Dk)
     outs = []
     for t in range(T):
-        S = _scal(alpha[t], S)                                     # decay
+        if _per_channel(alpha[t]):                                 # decay
+            S = [[S[j][i] * alpha[t][i] for i in range(Dk)] for j in range(Dv)]
+        else:
+            S = _scal(alpha[t], S)
         g = gamma[t] if gamma is not None else Fraction(1)
         pred = _matvec(S, k[t])
         err = [g * v[t][j] - pred[j] for j in range(Dv)]           # error
@@ -79,7 +89,13 @@ def closed_form(k, v, alpha, beta, S0=None, gamma=None):
     T, Dk, Dv = len(k), len(k[0]), len(v[0])
 
     def M(s):
-        return _scal(alpha[s], _add(_eye(Dk), _scal(-beta[s], _outer(k[s], k[s]))))
+        P = _add(_eye(Dk), _scal(-beta[s], _outer(k[s], k[s])))
+        if _per_channel(alpha[s]):
+            D = _zeros(Dk, Dk)
+            for i in range(Dk):
+                D[i][i] = alpha[s][i]
+            return _matmul(D, P)
+        return _scal(alpha[s], P)
 
     def prod(lo):
         P = _eye(Dk)

@@ -18,7 +18,13 @@
  *   o_t = scale * S_t q_t  (the output reads the post-update state).
  *
  *   Readings taken where the pages are silent:
- *     - decay is a scalar per (token, head), passed as log(alpha);
+ *     - decay is a scalar per (token, head), passed as log(alpha); the
+ *       per-key-channel variant (rda_oracle_forward_channel) takes log(alpha)
+ *       per (token, head, key dim) and scales column i of S (key dim i) by
+ *       alpha_i: S_t = S_{t-1} diag(alpha_t) (I - b_t k_t k_t^T) + b_t v_t k_t^T,
+ *       which is the scalar rule when every channel has the same alpha (the
+ *       same article's section says RDA modifies Kimi Delta Attention, whose
+ *       decay is per channel);
  *     - the write gate gamma multiplies v before the error is formed
  *       (NULL means gamma = 1);
  *     - scale defaults to 1 at the call sites; it multiplies the output only.
@@ -42,17 +48,25 @@
 #endif
 
 /* One token of the recurrence on an fp64 state S[Dv][Dk] (math orientation).
- * e is scratch of length Dv.  Writes o[j*o_stride] for j < Dv when o != NULL. */
+ * e is scratch of length Dv.  Writes o[j*o_stride] for j < Dv when o != NULL.
+ * With la_ch != NULL the decay is per key channel (la_ch[i] for column i) and
+ * log_alpha is not used. */
 static void rda_token(double *S, int Dk, int Dv,
                       const double *q, const double *k, const double *v,
                       double log_alpha, double beta, double gamma, double scale,
-                      double *e, double *o, long o_stride)
+                      double *e, double *o, long o_stride, const double *la_ch)
 {
     const double a = exp(log_alpha);
     /* 1. decay the state */
+    if (la_ch) {
+        for (int j = 0; j < Dv; ++j)
+            for (int i = 0; i < Dk; ++i)
+                S[(long)j * Dk + i] *= exp(la_ch[i]);
+    } else {
     for (int j = 0; j < Dv; ++j)
         for (int i = 0; i < Dk; ++i)
             S[(long)j * Dk + i] *= a;
+    }
     /* 2. error between the (gated) value and the decayed state's prediction */
     for (int j = 0; j < Dv; ++j) {
         double pred = 0.0;
@@ -97,11 +111,14 @@ static void store_state(double *dst, const double *S, int Dk, int Dv)
 }
 
 /* Runs one (sequence, head) unit over tokens [t0, t0+len) of arrays laid out as
- * [.., T_axis, H, D] with the given token stride (in elements). */
+ * [.., T_axis, H, D] with the given token stride (in elements).  la_ch, when
+ * not NULL, is the per-channel log decay [.., T_axis, H, Dk] (log_alpha is then
+ * only indexed, never used). */
 static void rda_unit(int Dk, int Dv, int H, int h, long t0, long len,
                      const double *q, const double *k, const double *v,
                      const double *log_alpha, const double *beta, const double *gamma,
-                     const double *s0, double *sf, double *out, double scale)
+                     const double *s0, double *sf, double *out, double scale,
+                     const double *la_ch)
 {
     double *S = (double *)malloc(sizeof(double) * ((size_t)Dk * Dv + Dv));
     double *e = S + (size_t)Dk * Dv;
@@ -110,7 +127,7 @@ static void rda_unit(int Dk, int Dv, int H, int h, long t0, long len,
         const long row = t * H + h;
         rda_token(S, Dk, Dv, q + row * Dk, k + row * Dk, v + row * Dv,
                   log_alpha[row], beta[row], gamma ? gamma[row] : 1.0, scale,
-                  e, out ? out + row * Dv : NULL, 1);
+                  e, out ? out + row * Dv : NULL, 1, la_ch ? la_ch + row * Dk : NULL);
     }
     store_state(sf, S, Dk, Dv);
     free(S);
@@ -137,7 +154,34 @@ int rda_oracle_forward(int B, int T, int H, int Dk, int Dv,
         const int h = (int)(u % H);
         const long sidx = (b * H + h) * (long)Dk * Dv;
         rda_unit(Dk, Dv, H, h, b * (long)T, T, q, k, v, log_alpha, beta, gamma,
-                 s0 ? s0 + sidx : NULL, sf ? sf + sidx : NULL, out, scale);
+                 s0 ? s0 + sidx : NULL, sf ? sf + sidx : NULL, out, scale, NULL);
+    }
+    return 0;
+}
+
+/* Fixed-length batch with per-key-channel decay: log_alpha_ch [B,T,H,Dk];
+ * everything else as rda_oracle_forward. */
+int rda_oracle_forward_channel(int B, int T, int H, int Dk, int Dv,
+                               const double *q, const double *k, const double *v,
+                               const double *log_alpha_ch, const double *beta, const double *gamma,
+                               const double *s0, double *sf, double *out, double scale,
+                               int num_threads)
+{
+    if (B < 0 || T < 0 || H <= 0 || Dk <= 0 || Dv <= 0 || !log_alpha_ch) return 1;
+    const long units = (long)B * H;
+#ifdef _OPENMP
+    if (num_threads > 0) omp_set_num_threads(num_threads);
+#else
+    (void)num_threads;
+#endif
+#pragma omp parallel for schedule(dynamic, 1)
+    for (long u = 0; u < units; ++u) {
+        const long b = u / H;
+        const int h = (int)(u % H);
+        const long sidx = (b * H + h) * (long)Dk * Dv;
+        /* log_alpha_ch doubles as the (unused) scalar array: it has a row per token */
+        rda_unit(Dk, Dv, H, h, b * (long)T, T, q, k, v, log_alpha_ch, beta, gamma,
+                 s0 ? s0 + sidx : NULL, sf ? sf + sidx : NULL, out, scale, log_alpha_ch);
     }
     return 0;
 }
@@ -167,7 +211,7 @@ int rda_oracle_varlen(int N, const int32_t *cu_seqlens, int H, int Dk, int Dv,
         const long sidx = ((long)n * H + h) * (long)Dk * Dv;
         rda_unit(Dk, Dv, H, h, cu_seqlens[n], (long)cu_seqlens[n + 1] - cu_seqlens[n],
                  q, k, v, log_alpha, beta, gamma,
-                 s0 ? s0 + sidx : NULL, sf ? sf + sidx : NULL, out, scale);
+                 s0 ? s0 + sidx : NULL, sf ? sf + sidx : NULL, out, scale, NULL);
     }
     return 0;
 }
@@ -194,7 +238,7 @@ int rda_oracle_decode_step(int B, int H, int Dk, int Dv,
         const int h = (int)(u % H);
         double *st = state + (b * H + h) * (long)Dk * Dv;
         rda_unit(Dk, Dv, H, h, b, 1, q, k, v, log_alpha, beta, gamma,
-                 st, st, out, scale);
+                 st, st, out, scale, NULL);
     }
     return 0;
 }

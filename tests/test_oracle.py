@@ -307,3 +307,86 @@ def test_workload_generator_shapes_and_ranges():
     assert float(a.min()) > 0.5 and float(a.max()) < 1.0
     again = rda_gen.workload("fp32_parity_b1_t256_h2_d64")
     assert torch.equal(again.v, inp.v)
+
+
+# ---------------------------------------------------------------- per-key-channel decay (next row 2)
+
+@pytest.mark.parametrize("seed", range(3))
+def test_exact_per_channel_sequential_equals_closed_form(seed):
+    """Per-channel decay: the token loop equals the product form with
+    M_s = diag(alpha_s) (I - beta_s k_s k_s^T), exactly."""
+    rng = np.random.default_rng(200 + seed)
+    T, Dk, Dv = 4 + seed, 3, 2 + seed % 2
+    fr = lambda: Fraction(int(rng.integers(-6, 7)), 4)
+    q = [[fr() for _ in range(Dk)] for _ in range(T)]
+    k = [[fr() for _ in range(Dk)] for _ in range(T)]
+    v = [[fr() for _ in range(Dv)] for _ in range(T)]
+    alpha = [[Fraction(int(rng.integers(1, 5)), 4) for _ in range(Dk)] for _ in range(T)]
+    beta = [Fraction(int(rng.integers(0, 5)), 4) for _ in range(T)]
+    gamma = [Fraction(int(rng.integers(1, 9)), 4) for _ in range(T)]
+    S0 = [[fr() for _ in range(Dk)] for _ in range(Dv)]
+    _, S = exact.sequential(q, k, v, alpha, beta, S0=S0, gamma=gamma)
+    assert S == exact.closed_form(k, v, alpha, beta, S0=S0, gamma=gamma)
+
+
+def test_per_channel_oracle_matches_exact_dyadic():
+    """fp64 per-channel oracle within 1e-13 of exact arithmetic (dyadic inputs,
+    per-channel alpha = 2^-m)."""
+    rng = np.random.default_rng(11)
+    T, Dk, Dv = 7, 4, 3
+    qn = rng.integers(-8, 9, (T, Dk)) / 8
+    kn = rng.integers(-8, 9, (T, Dk)) / 8
+    vn = rng.integers(-8, 9, (T, Dv)) / 8
+    m = rng.integers(0, 3, (T, Dk))
+    bn = rng.integers(0, 5, T) / 4
+    gn = rng.integers(1, 9, T) / 4
+    s0n = rng.integers(-8, 9, (Dv, Dk)) / 8
+    fr = lambda x: Fraction(x).limit_denominator(1 << 20)
+    outs, S = exact.sequential([[fr(x) for x in r] for r in qn], [[fr(x) for x in r] for r in kn],
+                               [[fr(x) for x in r] for r in vn],
+                               [[Fraction(1, 2 ** int(x)) for x in r] for r in m],
+                               [fr(x) for x in bn], S0=[[fr(x) for x in r] for r in s0n],
+                               gamma=[fr(x) for x in gn], scale=Fraction(1, 2))
+    out, sf = oracle.forward(qn.reshape(1, T, 1, Dk), kn.reshape(1, T, 1, Dk), vn.reshape(1, T, 1, Dv),
+                             (-m * math.log(2.0)).reshape(1, T, 1, Dk), bn.reshape(1, T, 1),
+                             gamma=gn.reshape(1, T, 1), initial_state=s0n.T.reshape(1, 1, Dk, Dv),
+                             scale=0.5)
+    assert np.allclose(out[0, :, 0], np.array([[float(x) for x in r] for r in outs]), rtol=0, atol=1e-13)
+    assert np.allclose(sf[0, 0].T, np.array([[float(x) for x in r] for r in S]), rtol=0, atol=1e-13)
+
+
+def test_per_channel_with_equal_channels_is_the_scalar_rule():
+    """Every channel at the token's decay: bit-identical to the scalar oracle."""
+    d = _rand(21, 2, 37, 3, 8, 5, gamma=True)
+    o1, s1 = oracle.forward(**d, scale=0.75)
+    d2 = dict(d)
+    d2["log_alpha"] = np.repeat(d["log_alpha"][..., None], 8, axis=-1)
+    o2, s2 = oracle.forward(**d2, scale=0.75)
+    assert np.array_equal(o1, o2) and np.array_equal(s1, s2)
+
+
+def test_per_channel_pure_decay_scales_key_columns():
+    """beta = 0: column i of the (math) state, i.e. row i of the stored
+    [Dk, Dv] state, decays by prod_t alpha_t[i]; Dk != Dv so rows and columns
+    cannot be confused."""
+    d = _rand(22, 1, 19, 2, 6, 4)
+    d["beta"][:] = 0.0
+    rng = np.random.default_rng(5)
+    la = -rng.uniform(0.0, 0.3, (1, 19, 2, 6))
+    d["log_alpha"] = la
+    _, sf = oracle.forward(**d)
+    total = np.exp(la.sum(axis=1))                          # [B,H,Dk]
+    assert np.allclose(sf, d["initial_state"] * total[:, :, :, None], rtol=1e-13, atol=1e-16)
+
+
+@pytest.mark.parametrize("T,decay_hi", [(70, 0.5), (130, 5.0), (64, 2.0)])
+def test_per_channel_chunked_equals_sequential(T, decay_hi):
+    """The independent per-channel chunked derivation (oracle/chunked.py) equals
+    the token-sequential per-channel oracle, ragged T and decays up to
+    log alpha = -5 per channel included."""
+    d = _rand(30 + T, 1, T, 2, 8, 5, gamma=True)
+    rng = np.random.default_rng(T)
+    d["log_alpha"] = -rng.uniform(0.0, decay_hi, (1, T, 2, 8))
+    o, s = oracle.forward(**d, scale=0.5)
+    oc, sc = chunked.forward(**d, scale=0.5, chunk=16)
+    assert _rel(oc, o) <= 1e-12 and _rel(sc, s) <= 1e-12

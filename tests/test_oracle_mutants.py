@@ -14,7 +14,7 @@ import numpy as np
 import pytest
 
 import oracle
-from oracle import chunked
+from oracle import chunked, exact
 
 SRC = os.path.join(os.path.dirname(oracle.__file__), "rda_oracle.c")
 GOLDEN = os.path.join(os.path.dirname(__file__), "golden", "exact_tiny.json")
@@ -75,6 +75,25 @@ def _battery(lib):
     o3, s3 = oracle.forward(**d3, lib=lib)
     if not np.array_equal(s3, d["initial_state"]):
         failed.append("beta0")
+    # per-key-channel decay against exact arithmetic (dyadic inputs, alpha = 2^-m per channel)
+    rng = np.random.default_rng(11)
+    T, Dk, Dv = 7, 4, 3
+    qn, kn = rng.integers(-8, 9, (T, Dk)) / 8, rng.integers(-8, 9, (T, Dk)) / 8
+    vn = rng.integers(-8, 9, (T, Dv)) / 8
+    m = rng.integers(0, 3, (T, Dk))
+    bn = rng.integers(0, 5, T) / 4
+    s0n = rng.integers(-8, 9, (Dv, Dk)) / 8
+    fr = lambda x: Fraction(x).limit_denominator(1 << 20)
+    outs, S = exact.sequential([[fr(x) for x in r] for r in qn], [[fr(x) for x in r] for r in kn],
+                               [[fr(x) for x in r] for r in vn],
+                               [[Fraction(1, 2 ** int(x)) for x in r] for r in m],
+                               [fr(x) for x in bn], S0=[[fr(x) for x in r] for r in s0n])
+    o4, s4 = oracle.forward(qn.reshape(1, T, 1, Dk), kn.reshape(1, T, 1, Dk), vn.reshape(1, T, 1, Dv),
+                            (-m * math.log(2.0)).reshape(1, T, 1, Dk), bn.reshape(1, T, 1),
+                            initial_state=s0n.T.reshape(1, 1, Dk, Dv), lib=lib)
+    if not (np.allclose(o4[0, :, 0], np.array([[float(x) for x in r] for r in outs]), rtol=0, atol=1e-12)
+            and np.allclose(s4[0, 0].T, np.array([[float(x) for x in r] for r in S]), rtol=0, atol=1e-12)):
+        failed.append("per_channel_exact")
     return failed
 
 
@@ -104,6 +123,12 @@ MUTANTS = {
     "read_before_write": _swap_update_and_read,
     "gate_index_shift": lambda s: s.replace("log_alpha[row], beta[row],",
                                             "log_alpha[row], beta[row > h ? row - 1 : row],"),
+    # per-key-channel decay
+    "channel_decay_dropped": lambda s: s.replace("S[(long)j * Dk + i] *= exp(la_ch[i]);",
+                                                 "S[(long)j * Dk + i] *= 1.0;"),
+    "channel_index_reversed": lambda s: s.replace("*= exp(la_ch[i]);", "*= exp(la_ch[Dk - 1 - i]);"),
+    "channel_stride_per_token": lambda s: s.replace("la_ch ? la_ch + row * Dk : NULL",
+                                                    "la_ch ? la_ch + row : NULL"),
 }
 
 
