@@ -23,8 +23,10 @@
  *       per (token, head, key dim) and scales column i of S (key dim i) by
  *       alpha_i: S_t = S_{t-1} diag(alpha_t) (I - b_t k_t k_t^T) + b_t v_t k_t^T,
  *       which is the scalar rule when every channel has the same alpha (the
- *       same article's section says RDA modifies Kimi Delta Attention, whose
- *       decay is per channel);
+ *       model card "tiny-random/raon-1-mini", section "Printing the model",
+ *       shows decay projections f_a_proj / f_b_proj as wide as heads x key
+ *       dims, and the same article names Kimi Delta Attention as what RDA
+ *       modifies);
  *     - the write gate gamma multiplies v before the error is formed
  *       (NULL means gamma = 1);
  *     - scale defaults to 1 at the call sites; it multiplies the output only.
