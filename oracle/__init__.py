@@ -38,9 +38,12 @@ def load_library(path):
     lib.rda_oracle_forward_channel.argtypes = [ctypes.c_int] * 5 + [dp] * 9 + [ctypes.c_double, ctypes.c_int]
     lib.rda_oracle_varlen.argtypes = [ctypes.c_int, ip] + [ctypes.c_int] * 3 + [dp] * 9 + [ctypes.c_double, ctypes.c_int]
     lib.rda_oracle_decode_step.argtypes = [ctypes.c_int] * 4 + [dp] * 8 + [ctypes.c_double, ctypes.c_int]
+    lib.rda_oracle_varlen_channel.argtypes = lib.rda_oracle_varlen.argtypes
+    lib.rda_oracle_decode_step_channel.argtypes = lib.rda_oracle_decode_step.argtypes
     lib.rda_oracle_max_threads.argtypes = []
     for f in (lib.rda_oracle_forward, lib.rda_oracle_forward_channel, lib.rda_oracle_varlen,
-              lib.rda_oracle_decode_step, lib.rda_oracle_max_threads):
+              lib.rda_oracle_varlen_channel, lib.rda_oracle_decode_step,
+              lib.rda_oracle_decode_step_channel, lib.rda_oracle_max_threads):
         f.restype = ctypes.c_int
     return lib
 
@@ -108,7 +111,8 @@ def varlen(q, k, v, log_alpha, beta, cu_seqlens, gamma=None, initial_states=None
     """Token-sequential fp64 recurrence over packed sequences.
 
     q, k ``[total,H,Dk]``; v ``[total,H,Dv]``; log_alpha, beta, gamma
-    ``[total,H]``; cu_seqlens int ``[N+1]``; initial_states ``[N,H,Dk,Dv]``.
+    ``[total,H]`` (log_alpha ``[total,H,Dk]`` for per-key-channel decay);
+    cu_seqlens int ``[N+1]``; initial_states ``[N,H,Dk,Dv]``.
     Returns ``(out [total,H,Dv], final_states [N,H,Dk,Dv])``.
     """
     q, k, v = _f64(q), _f64(k), _f64(v)
@@ -121,9 +125,12 @@ def varlen(q, k, v, log_alpha, beta, cu_seqlens, gamma=None, initial_states=None
     assert cu[0] == 0 and cu[-1] == total
     out = np.zeros((total, H, Dv), np.float64)
     sf = np.zeros((N, H, Dk, Dv), np.float64)
-    rc = _load().rda_oracle_varlen(N, cu.ctypes.data_as(ctypes.POINTER(ctypes.c_int32)), H, Dk, Dv,
-                                   _ptr(q), _ptr(k), _ptr(v), _ptr(la), _ptr(be), _ptr(ga),
-                                   _ptr(s0), _ptr(sf), _ptr(out), float(scale), int(num_threads))
+    assert la.shape == ((total, H, Dk) if la.ndim == 3 else (total, H))
+    L = _load()
+    fn = L.rda_oracle_varlen_channel if la.ndim == 3 else L.rda_oracle_varlen
+    rc = fn(N, cu.ctypes.data_as(ctypes.POINTER(ctypes.c_int32)), H, Dk, Dv,
+            _ptr(q), _ptr(k), _ptr(v), _ptr(la), _ptr(be), _ptr(ga),
+            _ptr(s0), _ptr(sf), _ptr(out), float(scale), int(num_threads))
     if rc != 0:
         raise ValueError("oracle.varlen: bad arguments")
     return out, sf
@@ -133,6 +140,7 @@ def decode_step(q, k, v, log_alpha, beta, state, gamma=None, scale=1.0, num_thre
                 lib=None):
     """One decode step: returns ``(out [B,H,Dv], new_state [B,H,Dk,Dv])``.
 
+    ``log_alpha`` is ``[B,H]``, or ``[B,H,Dk]`` for per-key-channel decay.
     ``state`` is not modified; a float64 copy is updated and returned.
     """
     q, k, v = _f64(q), _f64(k), _f64(v)
@@ -141,9 +149,11 @@ def decode_step(q, k, v, log_alpha, beta, state, gamma=None, scale=1.0, num_thre
     B, H, Dk = q.shape
     Dv = v.shape[-1]
     out = np.zeros((B, H, Dv), np.float64)
-    rc = _load(lib).rda_oracle_decode_step(B, H, Dk, Dv, _ptr(q), _ptr(k), _ptr(v), _ptr(la),
-                                        _ptr(be), _ptr(ga), _ptr(st), _ptr(out), float(scale),
-                                        int(num_threads))
+    assert la.shape == ((B, H, Dk) if la.ndim == 3 else (B, H))
+    L = _load(lib)
+    fn = L.rda_oracle_decode_step_channel if la.ndim == 3 else L.rda_oracle_decode_step
+    rc = fn(B, H, Dk, Dv, _ptr(q), _ptr(k), _ptr(v), _ptr(la), _ptr(be), _ptr(ga), _ptr(st),
+            _ptr(out), float(scale), int(num_threads))
     if rc != 0:
         raise ValueError("oracle.decode_step: bad arguments")
     return out, st

@@ -245,6 +245,60 @@ int rda_oracle_decode_step(int B, int H, int Dk, int Dv,
     return 0;
 }
 
+/* Packed variable-length batch with per-key-channel decay: log_alpha_ch
+ * [total,H,Dk]; everything else as rda_oracle_varlen. */
+int rda_oracle_varlen_channel(int N, const int32_t *cu_seqlens, int H, int Dk, int Dv,
+                              const double *q, const double *k, const double *v,
+                              const double *log_alpha_ch, const double *beta, const double *gamma,
+                              const double *s0, double *sf, double *out, double scale,
+                              int num_threads)
+{
+    if (N < 0 || H <= 0 || Dk <= 0 || Dv <= 0 || !log_alpha_ch) return 1;
+    for (int n = 0; n < N; ++n)
+        if (cu_seqlens[n + 1] < cu_seqlens[n]) return 1;
+    const long units = (long)N * H;
+#ifdef _OPENMP
+    if (num_threads > 0) omp_set_num_threads(num_threads);
+#else
+    (void)num_threads;
+#endif
+#pragma omp parallel for schedule(dynamic, 1)
+    for (long u = 0; u < units; ++u) {
+        const int n = (int)(u / H);
+        const int h = (int)(u % H);
+        const long sidx = ((long)n * H + h) * (long)Dk * Dv;
+        rda_unit(Dk, Dv, H, h, cu_seqlens[n], (long)cu_seqlens[n + 1] - cu_seqlens[n],
+                 q, k, v, log_alpha_ch, beta, gamma,
+                 s0 ? s0 + sidx : NULL, sf ? sf + sidx : NULL, out, scale, log_alpha_ch);
+    }
+    return 0;
+}
+
+/* One decode step with per-key-channel decay: log_alpha_ch [B,H,Dk]; everything
+ * else as rda_oracle_decode_step. */
+int rda_oracle_decode_step_channel(int B, int H, int Dk, int Dv,
+                                   const double *q, const double *k, const double *v,
+                                   const double *log_alpha_ch, const double *beta, const double *gamma,
+                                   double *state, double *out, double scale, int num_threads)
+{
+    if (B < 0 || H <= 0 || Dk <= 0 || Dv <= 0 || !log_alpha_ch) return 1;
+    const long units = (long)B * H;
+#ifdef _OPENMP
+    if (num_threads > 0) omp_set_num_threads(num_threads);
+#else
+    (void)num_threads;
+#endif
+#pragma omp parallel for schedule(dynamic, 1)
+    for (long u = 0; u < units; ++u) {
+        const long b = u / H;
+        const int h = (int)(u % H);
+        double *st = state + (b * H + h) * (long)Dk * Dv;
+        rda_unit(Dk, Dv, H, h, b, 1, q, k, v, log_alpha_ch, beta, gamma,
+                 st, st, out, scale, log_alpha_ch);
+    }
+    return 0;
+}
+
 int rda_oracle_max_threads(void)
 {
 #ifdef _OPENMP

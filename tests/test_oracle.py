@@ -390,3 +390,35 @@ def test_per_channel_chunked_equals_sequential(T, decay_hi):
     o, s = oracle.forward(**d, scale=0.5)
     oc, sc = chunked.forward(**d, scale=0.5, chunk=16)
     assert _rel(oc, o) <= 1e-12 and _rel(sc, s) <= 1e-12
+
+
+def test_per_channel_varlen_equals_per_sequence_loop():
+    rng = np.random.default_rng(41)
+    lens = [5, 0, 70, 33]
+    cu = np.concatenate([[0], np.cumsum(lens)]).astype(np.int32)
+    total, H, Dk, Dv = int(cu[-1]), 2, 8, 5
+    nrm = lambda x: x / np.linalg.norm(x, axis=-1, keepdims=True)
+    q, k = nrm(rng.standard_normal((total, H, Dk))), nrm(rng.standard_normal((total, H, Dk)))
+    v = rng.standard_normal((total, H, Dv))
+    la = -rng.uniform(0.0, 0.5, (total, H, Dk))
+    be, ga = rng.uniform(0, 1, (total, H)), rng.uniform(0.5, 1.5, (total, H))
+    s0 = rng.standard_normal((len(lens), H, Dk, Dv)) * 0.3
+    out, sf = oracle.varlen(q, k, v, la, be, cu, gamma=ga, initial_states=s0, scale=0.5)
+    for n in range(len(lens)):
+        a, b = cu[n], cu[n + 1]
+        o1, s1 = oracle.forward(q[None, a:b], k[None, a:b], v[None, a:b], la[None, a:b], be[None, a:b],
+                                gamma=ga[None, a:b], initial_state=s0[n:n + 1], scale=0.5)
+        assert np.array_equal(out[a:b], o1[0]) and np.array_equal(sf[n], s1[0])
+
+
+def test_per_channel_decode_steps_equal_prefill():
+    d = _rand(43, 3, 9, 2, 8, 5, gamma=True)
+    rng = np.random.default_rng(43)
+    d["log_alpha"] = -rng.uniform(0.0, 0.6, (3, 9, 2, 8))
+    o_ref, s_ref = oracle.forward(**d)
+    st = d["initial_state"]
+    for t in range(9):
+        o, st = oracle.decode_step(d["q"][:, t], d["k"][:, t], d["v"][:, t], d["log_alpha"][:, t],
+                                   d["beta"][:, t], st, gamma=d["gamma"][:, t])
+        assert np.array_equal(o, o_ref[:, t])
+    assert np.array_equal(st, s_ref)
