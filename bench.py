@@ -467,9 +467,18 @@ def oracle_sample_rate(T_sample, threads):
     return T_sample / dt, dt, min(threads, H)
 
 
-def cpu_baseline(target_s=12.0):
+def host_cores():
+    """Cores this process may run on (``nproc``)."""
+    try:
+        return len(os.sched_getaffinity(0))
+    except AttributeError:
+        return os.cpu_count() or 1
+
+
+def cpu_baseline(target_s=12.0, single_core_T=1024):
     """The oracle on the whole workload, repeated until about target_s seconds
-    of CPU work have run; tokens/s of the mean repetition."""
+    of CPU work have run; tokens/s of the mean repetition.  Also the oracle on
+    one core over the first `single_core_T` tokens (all heads)."""
     import oracle
     threads = oracle.max_threads()
     T = 4096
@@ -480,10 +489,15 @@ def cpu_baseline(target_s=12.0):
         _, d, _ = oracle_sample_rate(T, threads)
         total += d
     rate = T * reps / total
+    rate1, dt1, _ = oracle_sample_rate(single_core_T, 1)
     return {"value": rate, "unit": "tokens/s", "cores": cores, "kind": "oracle",
+            "host_nproc": host_cores(), "omp_threads_available": threads,
             "sample": f"fp64 token-sequential oracle over the full {WORKLOAD} workload "
-                      f"(T=4096, all 16 heads, one OpenMP thread per head), {reps} repetitions, "
-                      f"{total:.1f} s"}
+                      f"(T=4096, all 16 heads, OpenMP over the 16 heads: {cores} threads busy on a "
+                      f"{host_cores()}-core host), {reps} repetitions, {total:.1f} s",
+            "single_core": {"value": rate1, "unit": "tokens/s", "cores": 1,
+                            "sample": f"same oracle on one thread, first {single_core_T} tokens of "
+                                      f"{WORKLOAD} (all 16 heads), {dt1:.1f} s"}}
 
 
 def run_reference(args):
@@ -510,7 +524,7 @@ def run_reference(args):
         "config": {"workload": WORKLOAD, "B": 1, "T": 4096, "H": 16, "Dk": 128, "Dv": 128,
                    "chunk": CHUNK, "sample_T": T_sample},
         "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": cores, "kind": "oracle",
-                         "sample": sample},
+                         "host_nproc": host_cores(), "sample": sample},
         "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     }
 

@@ -53,6 +53,8 @@ lib.rda_read_device_error.argtypes = [_vp, ctypes.POINTER(_i), _vp]
 lib.rda_read_device_error.restype = _i
 lib.rda_prefill_chunked_noalloc.argtypes = [_vp] * 9 + [_i] * 6 + [_f, _vp]
 lib.rda_prefill_chunked_noalloc.restype = _i
+lib.rda_debug_set_wait_fault.argtypes = [_i, ctypes.c_ulonglong]
+lib.rda_debug_set_wait_fault.restype = None
 
 RDA_OK = 0
 RDA_F32 = 0
@@ -252,6 +254,12 @@ def rda_prefill_chunked_noalloc(q, k, v, log_alpha, beta, write_gate=None, initi
     return out, final_state
 
 
+def rda_debug_set_wait_fault(drop_chunk=-1, wait_limit_ns=0):
+    """Testing only: bound of the device-side waits and an injected stall of the
+    scan (see include/rda.h); ``rda_debug_set_wait_fault()`` turns it off."""
+    lib.rda_debug_set_wait_fault(int(drop_chunk), int(wait_limit_ns))
+
+
 def rda_read_device_error(workspace, stream=None) -> int:
     code = _i(0)
     _check(lib.rda_read_device_error(_ptr(workspace), ctypes.byref(code), _stream(stream)),
@@ -261,5 +269,5 @@ def rda_read_device_error(workspace, stream=None) -> int:
 
 __all__ = ["rda_prefill_chunked", "rda_prefill_varlen", "rda_decode_step", "rda_decode_tokens",
            "rda_prefill_chunked_noalloc",
-           "rda_read_device_error", "rda_prefill_workspace_bytes", "new_workspace", "version",
+           "rda_read_device_error", "rda_debug_set_wait_fault", "rda_prefill_workspace_bytes", "new_workspace", "version",
            "RdaError", "lib", "LIB_PATH"]

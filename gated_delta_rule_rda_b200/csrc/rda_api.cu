@@ -2,6 +2,7 @@
 // dispatch to the kernels on the caller's stream.  Nothing here allocates
 // device memory; nothing here computes any part of the recurrence.
 #include <algorithm>
+#include <atomic>
 #include <cstring>
 #include <numeric>
 #include <vector>
@@ -47,6 +48,38 @@ size_t workspace_bytes(int B, long T, int H, int Dk, int Dv, int num_seqs) {
 
 }  // namespace
 
+namespace rda {
+
+namespace {
+constexpr uint64_t kDefaultWaitNs = 4000000000ull;   // 4 s
+std::atomic<uint64_t> g_wait_ns{kDefaultWaitNs};
+std::atomic<int> g_drop_chunk{-1};
+}  // namespace
+
+WaitSettings wait_settings() { return WaitSettings{g_wait_ns.load(), g_drop_chunk.load()}; }
+
+rda_status_t validate_prefill_chunked(const void *q, const void *k, const void *v, const float *log_alpha,
+                                      const float *beta, const float *write_gate, const float *initial_state,
+                                      const float *final_state, const void *out, rda_dtype_t dtype, int B,
+                                      int T, int H, int Dk, int Dv, size_t *scratch_bytes) {
+    if (dtype != RDA_F32 && dtype != RDA_BF16) return RDA_ERR_UNSUPPORTED;
+    if (B < 0 || T < 0 || H <= 0) return RDA_ERR_INVALID_ARG;
+    if (!dims_ok(Dk, Dv)) return RDA_ERR_UNSUPPORTED;
+    if (!sizes_ok((long long)B * T, H, Dk, Dv)) return RDA_ERR_INVALID_ARG;
+    if ((long long)B * H * Dk * Dv >= (1LL << 31)) return RDA_ERR_INVALID_ARG;
+    if ((initial_state && !aligned(initial_state, 16)) || (final_state && !aligned(final_state, 16)))
+        return RDA_ERR_MISALIGNED;
+    if (write_gate && !aligned(write_gate, 4)) return RDA_ERR_MISALIGNED;
+    if (B > 0 && T > 0) {
+        rda_status_t st = check_io_ptrs(q, k, v, log_alpha, beta, out);
+        if (st != RDA_OK) return st;
+    }
+    *scratch_bytes = chunked_supported(dtype, Dk, Dv) ? workspace_bytes(B, T, H, Dk, Dv, 0) : kErrorWordBytes;
+    return RDA_OK;
+}
+
+}  // namespace rda
+
 extern "C" {
 
 const char *rda_status_string(rda_status_t s) {
@@ -76,25 +109,14 @@ rda_status_t rda_prefill_chunked(const void *q, const void *k, const void *v,
                                  void *out, rda_dtype_t dtype,
                                  int B, int T, int H, int Dk, int Dv, float scale,
                                  void *workspace, size_t workspace_bytes_given, void *stream) {
-    if (dtype != RDA_F32 && dtype != RDA_BF16) return RDA_ERR_UNSUPPORTED;
-    if (B < 0 || T < 0 || H <= 0) return RDA_ERR_INVALID_ARG;
-    if (!dims_ok(Dk, Dv)) return RDA_ERR_UNSUPPORTED;
-    if (!sizes_ok((long long)B * T, H, Dk, Dv)) return RDA_ERR_INVALID_ARG;
-    if ((long long)B * H * Dk * Dv >= (1LL << 31)) return RDA_ERR_INVALID_ARG;
-    const bool chunked = chunked_supported(dtype, Dk, Dv);
-    const size_t need = chunked ? workspace_bytes(B, T, H, Dk, Dv, 0) : kErrorWordBytes;
+    size_t need = 0;
+    rda_status_t st = validate_prefill_chunked(q, k, v, log_alpha, beta, write_gate, initial_state, final_state,
+                                               out, dtype, B, T, H, Dk, Dv, &need);
+    if (st != RDA_OK) return st;
     if (!workspace || workspace_bytes_given < need) return RDA_ERR_WORKSPACE;
     if (!aligned(workspace, 256)) return RDA_ERR_MISALIGNED;
-    if ((initial_state && !aligned(initial_state, 16)) || (final_state && !aligned(final_state, 16)))
-        return RDA_ERR_MISALIGNED;
-    if (write_gate && !aligned(write_gate, 4)) return RDA_ERR_MISALIGNED;
     cudaStream_t s = static_cast<cudaStream_t>(stream);
-    const bool empty = (B == 0 || T == 0);
-    if (!empty) {
-        rda_status_t st = check_io_ptrs(q, k, v, log_alpha, beta, out);
-        if (st != RDA_OK) return st;
-    }
-    if (empty) {
+    if (B == 0 || T == 0) {
         if (B > 0 && final_state) {
             const size_t bytes = sizeof(float) * (size_t)B * H * Dk * Dv;
             cudaError_t e = initial_state
@@ -113,8 +135,12 @@ rda_status_t rda_prefill_chunked(const void *q, const void *k, const void *v,
     a.num_seqs = B; a.T = T; a.total_T = B * T;
     a.H = H; a.Dk = Dk; a.Dv = Dv; a.scale = scale;
     a.err = static_cast<int32_t *>(workspace);
-    cudaError_t e = chunked ? launch_chunked(a, static_cast<char *>(workspace) + kErrorWordBytes, s)
-                            : launch_recurrent(a, dtype, s);
+    const WaitSettings ws = wait_settings();
+    a.wait_ns = ws.wait_ns;
+    a.debug_drop_chunk = ws.drop_chunk;
+    cudaError_t e = chunked_supported(dtype, Dk, Dv)
+                        ? launch_chunked(a, static_cast<char *>(workspace) + kErrorWordBytes, s)
+                        : launch_recurrent(a, dtype, s);
     return e == cudaSuccess ? RDA_OK : RDA_ERR_CUDA;
 }
 
@@ -173,6 +199,9 @@ rda_status_t rda_prefill_varlen(const void *q, const void *k, const void *v,
     a.num_seqs = num_seqs; a.T = 0; a.total_T = total_T;
     a.H = H; a.Dk = Dk; a.Dv = Dv; a.scale = scale;
     a.err = static_cast<int32_t *>(workspace);
+    const WaitSettings ws = wait_settings();
+    a.wait_ns = ws.wait_ns;
+    a.debug_drop_chunk = ws.drop_chunk;
     cudaError_t e = chunked
         ? launch_chunked(a, static_cast<char *>(workspace) + kErrorWordBytes + order_bytes(num_seqs), s)
         : launch_recurrent(a, dtype, s);
@@ -226,6 +255,11 @@ rda_status_t rda_decode_tokens(const void *q, const void *k, const void *v,
     a.B = B; a.T = T; a.H = H; a.Dk = Dk; a.Dv = Dv; a.scale = scale;
     return launch_decode_tokens(a, dtype, static_cast<cudaStream_t>(stream)) == cudaSuccess ? RDA_OK
                                                                                               : RDA_ERR_CUDA;
+}
+
+void rda_debug_set_wait_fault(int drop_chunk, unsigned long long wait_limit_ns) {
+    rda::g_drop_chunk.store(drop_chunk < 0 ? -1 : drop_chunk);
+    rda::g_wait_ns.store(wait_limit_ns ? (uint64_t)wait_limit_ns : rda::kDefaultWaitNs);
 }
 
 rda_status_t rda_read_device_error(void *workspace, int *code, void *stream) {

@@ -56,7 +56,6 @@ using namespace ptx;
 
 constexpr int kC = 64;            // chunk length
 constexpr int kDK = 128;          // key dimension handled here
-constexpr uint64_t kWaitNs = 4000000000ull;   // bounded waits: 4 s
 
 // Per (chunk, head) image in the workspace (bytes).
 constexpr uint32_t kImgW = 0;          // -W, bf16 K-major SW128, 2 halves of 8 KiB (64 rows x 64 cols)
@@ -77,13 +76,13 @@ __device__ __forceinline__ uint64_t globaltimer() {
 // a single-thread agent (TMA / MMA issue) passes its own `mine`, so that it
 // never changes a flag such threads read.
 __device__ __noinline__ bool wait_bar_slow(uint64_t *bar, uint32_t parity, volatile int *stop, volatile int *mine,
-                                           int32_t *err) {
+                                           int32_t *err, uint64_t limit_ns) {
     const uint64_t t0 = globaltimer();
     for (uint32_t i = 0;; ++i) {
         if (mbar_try_wait(bar, parity)) return true;
         if ((i & 63) == 63) {
             if (*stop || *mine) return false;
-            if (globaltimer() - t0 > kWaitNs) {
+            if (globaltimer() - t0 > limit_ns) {
                 *mine = 1;
                 atomicCAS(err, 0, (int32_t)RDA_ERR_TIMEOUT);
                 return false;
@@ -92,20 +91,21 @@ __device__ __noinline__ bool wait_bar_slow(uint64_t *bar, uint32_t parity, volat
     }
 }
 __device__ __forceinline__ bool wait_bar2(uint64_t *bar, uint32_t parity, volatile int *stop, volatile int *mine,
-                                          int32_t *err) {
+                                          int32_t *err, uint64_t limit_ns) {
     if (mbar_try_wait(bar, parity)) return true;
-    return wait_bar_slow(bar, parity, stop, mine, err);
+    return wait_bar_slow(bar, parity, stop, mine, err, limit_ns);
 }
-__device__ __forceinline__ bool wait_bar(uint64_t *bar, uint32_t parity, volatile int *flag, int32_t *err) {
-    return wait_bar2(bar, parity, flag, flag, err);
+__device__ __forceinline__ bool wait_bar(uint64_t *bar, uint32_t parity, volatile int *flag, int32_t *err,
+                                         uint64_t limit_ns) {
+    return wait_bar2(bar, parity, flag, flag, err, limit_ns);
 }
 
 // Bounded wait that ignores the abort flag: used only to let copies or MMAs
 // already in flight land before a CTA that gave up exits.
-__device__ __noinline__ void drain_bar(uint64_t *bar, uint32_t parity) {
+__device__ __noinline__ void drain_bar(uint64_t *bar, uint32_t parity, uint64_t limit_ns) {
     const uint64_t t0 = globaltimer();
     while (!mbar_try_wait(bar, parity))
-        if (globaltimer() - t0 > kWaitNs) return;
+        if (globaltimer() - t0 > limit_ns) return;
 }
 
 // Byte offset of 16-byte chunk `c` of row `row` in a tile whose rows are
@@ -500,7 +500,7 @@ prep_kernel(const __grid_constant__ PrepMaps maps, const PrefillArgs a) {
             constexpr uint32_t ID_KK = idesc_bf16(64, 64, 0, 0);
             constexpr uint32_t ID_W = idesc_bf16(64, 128, 0, 1);
             const uint32_t ID_U = Dv == 128 ? idesc_bf16(64, 128, 0, 1) : idesc_bf16(64, 64, 0, 1);
-            bool ok = wait_bar2(&bars[PB_FULL], 0, abort_flag, agent_flag, a.err);
+            bool ok = wait_bar2(&bars[PB_FULL], 0, abort_flag, agent_flag, a.err, a.wait_ns);
             if (ok) {
                 tc_fence_after();
 #pragma unroll
@@ -517,7 +517,7 @@ prep_kernel(const __grid_constant__ PrepMaps maps, const PrefillArgs a) {
                              smem_desc(kk_ + off, 16, 1024, kSw128), ID_KK, kk > 0);
                 }
                 mma_commit(&bars[PB_QK]);
-                ok = wait_bar2(&bars[PB_TREADY], 0, abort_flag, agent_flag, a.err);
+                ok = wait_bar2(&bars[PB_TREADY], 0, abort_flag, agent_flag, a.err, a.wait_ns);
             }
             if (ok) {
                 // the compute threads fenced their generic accesses to A's region
@@ -532,8 +532,8 @@ prep_kernel(const __grid_constant__ PrepMaps maps, const PrefillArgs a) {
                     mma_bf16(tmem + PT_W, smem_desc(tbg + kk * 32, 16, 1024, kSw128),
                              smem_desc(kk_ + kk * 2048, 8192, 1024, kSw128), ID_W, kk > 0);
                 mma_commit(&bars[PB_W]);
-                ok = wait_bar2(&bars[PB_WFREE], 0, abort_flag, agent_flag, a.err) &&
-                     wait_bar2(&bars[PB_VFULL], 0, abort_flag, agent_flag, a.err);
+                ok = wait_bar2(&bars[PB_WFREE], 0, abort_flag, agent_flag, a.err, a.wait_ns) &&
+                     wait_bar2(&bars[PB_VFULL], 0, abort_flag, agent_flag, a.err, a.wait_ns);
             }
             if (ok) {
                 tc_fence_after();
@@ -544,9 +544,9 @@ prep_kernel(const __grid_constant__ PrepMaps maps, const PrefillArgs a) {
                 mma_commit(&bars[PB_U]);
             }
             mma_commit(&bars[PB_DRAIN]);      // every MMA issued has completed before TMEM is freed
-            drain_bar(&bars[PB_DRAIN], 0);
-            drain_bar(&bars[PB_FULL], 0);     // the CTA may not exit with copies in flight
-            if (v_issued) drain_bar(&bars[PB_VFULL], 0);
+            drain_bar(&bars[PB_DRAIN], 0, a.wait_ns);
+            drain_bar(&bars[PB_FULL], 0, a.wait_ns);     // the CTA may not exit with copies in flight
+            if (v_issued) drain_bar(&bars[PB_VFULL], 0, a.wait_ns);
         }
     } else {
         const int cw = threadIdx.x - 32;
@@ -558,7 +558,7 @@ prep_kernel(const __grid_constant__ PrepMaps maps, const PrefillArgs a) {
         float *Xs = reinterpret_cast<float *>(sm + PS_XS);
 
         chunk_gates(gates, r, lane, g_s);
-        if (cw == 0 && !wait_bar(&bars[PB_KK], 0, abort_flag, a.err)) *abort_flag = 1;
+        if (cw == 0 && !wait_bar(&bars[PB_KK], 0, abort_flag, a.err, a.wait_ns)) *abort_flag = 1;
         named_bar_sync(1, 128);
         if (!*abort_flag) {
             tc_fence_after();
@@ -573,12 +573,12 @@ prep_kernel(const __grid_constant__ PrepMaps maps, const PrefillArgs a) {
             }
             tc_fence_before();
         }
-        if (cw == 0 && !*abort_flag && !wait_bar(&bars[PB_QK], 0, abort_flag, a.err)) *abort_flag = 1;
+        if (cw == 0 && !*abort_flag && !wait_bar(&bars[PB_QK], 0, abort_flag, a.err, a.wait_ns)) *abort_flag = 1;
         named_bar_sync(1, 128);
         if (!*abort_flag) {
             // the Q tile landed before the Q K^T product was issued; this wait (complete
             // already) makes the copy visible to these threads
-            wait_bar(&bars[PB_FULL], 0, abort_flag, a.err);
+            wait_bar(&bars[PB_FULL], 0, abort_flag, a.err, a.wait_ns);
             tc_fence_after();
             // P rows ta, ta + 8: (Q K^T)[t][s] e^{g_t - g_s}, s <= t -> bf16 K-major
             // SW128 image, stored from registers
@@ -627,7 +627,7 @@ prep_kernel(const __grid_constant__ PrepMaps maps, const PrefillArgs a) {
         named_bar_sync(1, 128);
         if (cw == 0 && !*abort_flag) {
             mbar_arrive(&bars[PB_TREADY]);
-            if (!wait_bar(&bars[PB_W], 0, abort_flag, a.err)) *abort_flag = 1;
+            if (!wait_bar(&bars[PB_W], 0, abort_flag, a.err, a.wait_ns)) *abort_flag = 1;
         }
         named_bar_sync(1, 128);
         if (!*abort_flag) {
@@ -655,7 +655,7 @@ prep_kernel(const __grid_constant__ PrepMaps maps, const PrefillArgs a) {
             mbar_arrive(&bars[PB_WFREE]);
             bulk_store(img + kImgW, sm + PS_WIMG, 16384);
             bulk_commit();
-            if (!wait_bar(&bars[PB_U], 0, abort_flag, a.err)) *abort_flag = 1;
+            if (!wait_bar(&bars[PB_U], 0, abort_flag, a.err, a.wait_ns)) *abort_flag = 1;
         }
         named_bar_sync(1, 128);
         if (!*abort_flag) {
@@ -847,11 +847,15 @@ scan_kernel(const __grid_constant__ ScanMaps maps, const PrefillArgs a) {
         // ------------------------------------------------------------ producer
         if (lane == 0) {
             pdl_wait_primary();      // the prep's images are complete and visible
+            int last[kScanStages];   // last chunk whose loads went out on each stage
+            for (int i = 0; i < kScanStages; ++i) last[i] = -1;
             for (int c = 0; c < nchunks; ++c) {
                 const int st = c % kScanStages;
                 if (c >= kScanStages &&
-                    !wait_bar2(&bars[SB_EMPTY + st], (c / kScanStages - 1) & 1, abort_flag, agent_flag, a.err))
+                    !wait_bar2(&bars[SB_EMPTY + st], (c / kScanStages - 1) & 1, abort_flag, agent_flag, a.err, a.wait_ns))
                     break;
+                if (c == a.debug_drop_chunk) continue;   // fault injection (tests only): never filled
+                last[st] = c;
                 uint64_t *full = &bars[SB_FULL + st];
                 uint8_t *stg = sm + st * SS_STAGE;
                 const uint8_t *img = a.workspace_chunks + ((size_t)(gc0 + c) * H + h) * a.chunk_bytes;
@@ -866,6 +870,10 @@ scan_kernel(const __grid_constant__ ScanMaps maps, const PrefillArgs a) {
                 bulk_load(stg + SS_U, img + kImgU + (size_t)slice * UBYTES, UBYTES, full);
                 bulk_load(stg + SS_G, img + kImgU + 64 * Dv * 2, 512, full);
             }
+            // the CTA may not exit with copies in flight: after an abort the scan
+            // warps stop consuming, so wait (bounded) for every stage's last fill
+            for (int i = 0; i < kScanStages; ++i)
+                if (last[i] >= 0) drain_bar(&bars[SB_FULL + i], (last[i] / kScanStages) & 1, a.wait_ns);
         }
         return;
     }
@@ -907,7 +915,7 @@ scan_kernel(const __grid_constant__ ScanMaps maps, const PrefillArgs a) {
                     const uint32_t v = pack_bf16(S[mt][nt][2 * hh], S[mt][nt][2 * hh + 1]);
                     *reinterpret_cast<uint32_t *>(sm + SC_SS + d * RS + j * 2) = v;
                 }
-        if (tid == 0 && !wait_bar(&bars[SB_FULL + st], (c / kScanStages) & 1, abort_flag, a.err)) *abort_flag = 1;
+        if (tid == 0 && !wait_bar(&bars[SB_FULL + st], (c / kScanStages) & 1, abort_flag, a.err, a.wait_ns)) *abort_flag = 1;
         named_bar_sync(1, NCW);
         if (*abort_flag) break;
         // ---- U = U' + (-W) S for rows t = 16rg .. 16rg+15 (accumulators start at U')

@@ -31,6 +31,8 @@ struct PrefillArgs {
     int H, Dk, Dv;
     float scale;
     int32_t *err;                // device error word
+    uint64_t wait_ns;            // bound of every device-side wait
+    int debug_drop_chunk;        // fault injection (tests only): the scan never fills this chunk; -1 = off
     // chunked path only (filled by launch_chunked)
     const int32_t *chunk_base;   // packed: first global chunk of each sequence [N+1]
     uint8_t *workspace_chunks;   // per (chunk, head) prep results
@@ -47,6 +49,14 @@ struct DecodeArgs {
     int T;                       // tokens per sequence (multi-token decode only)
 };
 
+// Bound of the device-side waits, and the test-only fault injection, as set by
+// rda_debug_set_wait_fault (defaults: 4 s, no fault).
+struct WaitSettings {
+    uint64_t wait_ns;
+    int drop_chunk;
+};
+WaitSettings wait_settings();
+
 // Most tokens one multi-token decode call takes per sequence.
 constexpr int kMaxDecodeTokens = 8;
 
@@ -59,5 +69,14 @@ cudaError_t launch_chunked(const PrefillArgs &a, void *scratch, cudaStream_t s);
 bool chunked_supported(rda_dtype_t dtype, int Dk, int Dv);
 // Scratch the chunked path needs: fixed-length batches pass num_seqs = 0.
 size_t chunked_workspace_bytes(long total_T, int T, int B, int H, int Dv, int num_seqs);
+
+// Host-side argument checks of rda_prefill_chunked except those of the
+// workspace; enqueues nothing.  On RDA_OK, *scratch_bytes is the workspace
+// that call needs for these arguments (the error word alone on the
+// token-sequential path).
+rda_status_t validate_prefill_chunked(const void *q, const void *k, const void *v, const float *log_alpha,
+                                      const float *beta, const float *write_gate, const float *initial_state,
+                                      const float *final_state, const void *out, rda_dtype_t dtype, int B,
+                                      int T, int H, int Dk, int Dv, size_t *scratch_bytes);
 
 }  // namespace rda

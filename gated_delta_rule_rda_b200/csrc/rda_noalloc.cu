@@ -10,40 +10,18 @@
 // The array is shared by every call on a device and keeps the last call's
 // contents; calls whose work overlaps on the GPU (for example on two streams
 // without ordering between them) race on it.  The device error word at its
-// start is cleared at the beginning of each call.
-#include <mutex>
-
+// start is cleared at the beginning of each call that passes the argument
+// checks; a call that fails them enqueues nothing.
 #include "rda_internal.h"
 
 namespace {
 
-// Largest scratch this entry point can use, bytes: enough for the chunked
-// path's per-chunk images of about 1,600 (chunk, head) pairs at Dv = 128,
-// e.g. B = 1, T = 4096, H = 16.
+// Largest scratch this entry point can use, bytes: the chunked path's
+// per-chunk images of about 1,600 (chunk, head) pairs at Dv = 128 (H = 16:
+// T up to about 6,400).
 constexpr size_t kNoAllocScratchBytes = size_t(64) << 20;
 
 static __device__ __align__(256) unsigned char g_noalloc_scratch[kNoAllocScratchBytes];
-
-// Host code may not use the array's name as a device address: it resolves the
-// address once per device, with that device current.
-std::mutex g_mu;
-void *g_scratch_addr[64] = {};
-
-cudaError_t scratch_for_current_device(void **out) {
-    int dev = 0;
-    cudaError_t e = cudaGetDevice(&dev);
-    if (e != cudaSuccess) return e;
-    if (dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
-    std::lock_guard<std::mutex> lk(g_mu);
-    if (!g_scratch_addr[dev]) {
-        void *p = nullptr;
-        e = cudaGetSymbolAddress(&p, g_noalloc_scratch);
-        if (e != cudaSuccess) return e;
-        g_scratch_addr[dev] = p;
-    }
-    *out = g_scratch_addr[dev];
-    return cudaSuccess;
-}
 
 }  // namespace
 
@@ -54,15 +32,19 @@ extern "C" rda_status_t rda_prefill_chunked_noalloc(const void *q, const void *k
                                                    void *out, rda_dtype_t dtype,
                                                    int B, int T, int H, int Dk, int Dv, float scale,
                                                    void *stream) {
-    if (B < 0 || T < 0 || H <= 0) return RDA_ERR_INVALID_ARG;
-    const size_t need = rda_prefill_workspace_bytes(B, T, H, Dk, Dv, 0);
-    if (need == 0) return (Dk == 64 || Dk == 128) && (Dv == 64 || Dv == 128) ? RDA_ERR_INVALID_ARG
-                                                                              : RDA_ERR_UNSUPPORTED;
+    size_t need = 0;
+    rda_status_t st = rda::validate_prefill_chunked(q, k, v, log_alpha, beta, write_gate, initial_state,
+                                                    final_state, out, dtype, B, T, H, Dk, Dv, &need);
+    if (st != RDA_OK) return st;
     if (need > kNoAllocScratchBytes) return RDA_ERR_WORKSPACE;
+    // The array's name is not a device address in host code.  Its address is
+    // looked up in the current context on every call, so a context created
+    // after a device reset (or another context on the same device) gets its
+    // own array's address, never a stale one.
     void *scratch = nullptr;
-    if (scratch_for_current_device(&scratch) != cudaSuccess) return RDA_ERR_CUDA;
-    if (cudaMemsetAsync(scratch, 0, sizeof(int32_t), static_cast<cudaStream_t>(stream)) != cudaSuccess)
-        return RDA_ERR_CUDA;
+    if (cudaGetSymbolAddress(&scratch, g_noalloc_scratch) != cudaSuccess || !scratch) return RDA_ERR_CUDA;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    if (cudaMemsetAsync(scratch, 0, sizeof(int32_t), s) != cudaSuccess) return RDA_ERR_CUDA;
     return rda_prefill_chunked(q, k, v, log_alpha, beta, write_gate, initial_state, final_state, out, dtype,
                                B, T, H, Dk, Dv, scale, scratch, kNoAllocScratchBytes, stream);
 }

@@ -35,7 +35,9 @@
  *
  * OWNERSHIP AND ORDERING
  *   Every pointer named "device" is device memory owned by the caller; the
- *   library allocates no device memory and keeps no per-call state.  Each call
+ *   library allocates no device memory and keeps no per-call state.  The one
+ *   exception is rda_prefill_chunked_noalloc's fixed scratch array, a static
+ *   device array of the library (described with that call).  Each call
  *   enqueues its work on `stream` (a cudaStream_t, passed as void*; NULL is the
  *   legacy default stream) and returns without synchronising.  Calls are
  *   thread-safe.  Input buffers must not be modified, and outputs not read,
@@ -207,20 +209,24 @@ rda_status_t rda_decode_tokens(const void *q, const void *k, const void *v,
  * library scratch memory: host programs that own all device memory themselves
  * (an inference server that sizes its memory pool once at start-up and allows
  * no cudaMalloc afterwards, a plug-in whose host framework passes tensors but
- * offers no way to ask for scratch).  Arguments, layouts, results and errors
- * are those of rda_prefill_chunked; it calls no cudaMalloc, cudaFree or other
- * allocating routine.
+ * offers no way to ask for scratch).  Arguments, layouts and argument errors
+ * are those of rda_prefill_chunked, and its results equal that call's bit for
+ * bit; it calls no cudaMalloc, cudaFree or other allocating routine.
  *
  * Its scratch is a fixed 64 MiB array in device memory that every GPU loading
- * this library holds until the process exits.  Problems whose
- * rda_prefill_workspace_bytes(B,T,H,Dk,Dv,0) exceeds 64 MiB are rejected with
- * RDA_ERR_WORKSPACE before anything is enqueued (at Dv = 128 the limit is
- * about 1,600 chunk-head pairs, e.g. B = 1, T = 4096, H = 16).  The first call on
- * a device looks up the array's device address; make that first call before
- * any stream capture.  All calls on a device share the array, which keeps the
- * last call's contents: calls whose work overlaps on the GPU (unordered
- * streams) race on it.  Each call clears the array's device error word before
- * launching; a device-side timeout is not reported back through this call.
+ * this library holds until the process exits.  A call that needs more scratch
+ * than that (rda_prefill_workspace_bytes for bf16 inputs with Dk = 128: about
+ * 1,600 chunk-head pairs at Dv = 128, i.e. H = 16 and T up to about 6,400; the
+ * nano shape T = 4096, H = 16 fits) is rejected with RDA_ERR_WORKSPACE.  The
+ * token-sequential path (fp32 inputs, or Dk = 64) needs only the error word and
+ * is never rejected for size.  Like every other argument error, a rejection
+ * enqueues nothing.  Each call looks up the array's device address in the
+ * current context; the first call in a context also loads the library's device
+ * code, so make it before any stream capture.  All calls on a device share the
+ * array, which keeps the last call's contents: calls whose work overlaps on the
+ * GPU (unordered streams) race on it.  Each accepted call clears the array's
+ * device error word before launching; a device-side timeout is not reported
+ * back through this call.
  */
 rda_status_t rda_prefill_chunked_noalloc(const void *q, const void *k, const void *v,
                                          const float *log_alpha, const float *beta,
@@ -229,6 +235,22 @@ rda_status_t rda_prefill_chunked_noalloc(const void *q, const void *k, const voi
                                          void *out, rda_dtype_t dtype,
                                          int B, int T, int H, int Dk, int Dv, float scale,
                                          void *stream);
+
+/*
+ * TESTING ONLY: fault injection for the device-side timeout path.
+ *
+ * Process-wide; affects the prefill calls made after it returns.  The bound of
+ * every device-side wait becomes `wait_limit_ns` (0 restores the default, 4 s),
+ * and, when drop_chunk >= 0, the state scan of the chunked path never fills
+ * the operands of chunk `drop_chunk` of each (sequence, head, value slice):
+ * the scan's wait for that chunk runs out, the kernel records RDA_ERR_TIMEOUT
+ * in the workspace error word, waits (bounded) for the copies it already has
+ * in flight and returns, leaving the outputs from that chunk on and the final
+ * state unwritten.  The context stays usable.  rda_debug_set_wait_fault(-1, 0)
+ * turns it off (the default).  Not for production use: no other argument is
+ * checked, and calls on other threads see the setting too.
+ */
+void rda_debug_set_wait_fault(int drop_chunk, unsigned long long wait_limit_ns);
 
 /*
  * Waits for `stream`, then reads and clears the device error word at the start

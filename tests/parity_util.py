@@ -33,13 +33,9 @@ def gpu_fixed(inp, scale=1.0, device="cuda"):
     return to_np(out), to_np(sf)
 
 
-def oracle_fixed(inp, scale=1.0, heads=None):
-    sel = (lambda t: t) if heads is None else (lambda t: None if t is None else t[:, :, heads])
-    s0 = inp.initial_state
-    if heads is not None and s0 is not None:
-        s0 = s0[:, heads]
-    return oracle.forward(sel(inp.q), sel(inp.k), sel(inp.v), sel(inp.log_alpha), sel(inp.beta),
-                          gamma=sel(inp.gamma), initial_state=s0, scale=scale)
+def oracle_fixed(inp, scale=1.0):
+    return oracle.forward(inp.q, inp.k, inp.v, inp.log_alpha, inp.beta, gamma=inp.gamma,
+                          initial_state=inp.initial_state, scale=scale)
 
 
 def gpu_varlen(vin, scale=1.0, host_schedule=True, device="cuda"):
@@ -51,19 +47,3 @@ def gpu_varlen(vin, scale=1.0, host_schedule=True, device="cuda"):
                                      cu_seqlens_host=vin.cu_seqlens if host_schedule else None)
     torch.cuda.synchronize()
     return to_np(out), to_np(sf)
-
-
-def oracle_varlen_subset(vin, seqs, heads, scale=1.0):
-    """Oracle over a subset of sequences and heads; returns per-sequence
-    (out [L, len(heads), Dv], state [len(heads), Dk, Dv]) lists."""
-    cu = vin.cu_seqlens.numpy()
-    outs, states = [], []
-    for n in seqs:
-        a, b = int(cu[n]), int(cu[n + 1])
-        sl = lambda t: None if t is None else t[a:b][:, heads][None]
-        s0 = None if vin.initial_states is None else vin.initial_states[n:n + 1, heads]
-        o, s = oracle.forward(sl(vin.q), sl(vin.k), sl(vin.v), sl(vin.log_alpha), sl(vin.beta),
-                              gamma=sl(vin.gamma), initial_state=s0, scale=scale)
-        outs.append(o[0])
-        states.append(s[0])
-    return outs, states
