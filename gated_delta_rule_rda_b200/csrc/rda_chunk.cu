@@ -108,6 +108,13 @@ __device__ __noinline__ void drain_bar(uint64_t *bar, uint32_t parity, uint64_t 
         if (globaltimer() - t0 > limit_ns) return;
 }
 
+// The dynamic shared memory rounded up to a 1024-byte boundary (what 128-byte
+// swizzled tiles need).  Derived from the __shared__ array by pointer
+// arithmetic, so that accesses through it stay shared-memory accesses.
+__device__ __forceinline__ uint8_t *smem_align_1024(uint8_t *raw) {
+    return raw + ((1024u - (smem_u32(raw) & 1023u)) & 1023u);
+}
+
 // Byte offset of 16-byte chunk `c` of row `row` in a tile whose rows are
 // `rowbytes` long, in the canonical swizzle of that width (rows contiguous;
 // address bits [4,7) XORed with bits [7,10)).
@@ -443,7 +450,7 @@ template <int NV>
 __global__ void __launch_bounds__(kPrepThreads, 4)
 prep_kernel(const __grid_constant__ PrepMaps maps, const PrefillArgs a) {
     extern __shared__ uint8_t smem_raw[];
-    uint8_t *sm = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    uint8_t *sm = smem_align_1024(smem_raw);
     // the scan may launch (and run its prologue) once every prep CTA has started;
     // it waits for this grid's completion before it reads the workspace
     if (threadIdx.x == 0) pdl_launch_dependents();
@@ -798,7 +805,7 @@ template <int NV>
 __global__ void __launch_bounds__(kScanThreads, 1)
 scan_kernel(const __grid_constant__ ScanMaps maps, const PrefillArgs a) {
     extern __shared__ uint8_t smem_raw[];
-    uint8_t *sm = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    uint8_t *sm = smem_align_1024(smem_raw);
     using L = ScanSmem<NV>;
     constexpr uint32_t SC_SS = L::SS, SC_UT = L::UT;
     uint64_t *bars = reinterpret_cast<uint64_t *>(sm + L::BAR);
