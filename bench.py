@@ -421,6 +421,36 @@ def other_workloads(device, stream, rank, world, reps=5):
                            "hbm_frac": nbytes / (ms * 1e-3) / 1e9 / load_peaks()[0]}
     del inp, ws, out, sf
 
+    # per-key-channel decay at the nano shape (token-sequential fp32 kernel)
+    inp = rda_gen.workload("nano_prefill_channel_b1_t4096_h16_d128").to(device)
+    B, T, H, Dk = inp.q.shape
+    ws = rda.new_workspace(rda.rda_prefill_workspace_bytes(B, T, H, Dk, Dk, 0), device)
+    out = torch.empty_like(inp.v)
+    sf = torch.empty((B, H, Dk, Dk), device=device)
+    ms = timed(lambda: rda.rda_prefill_chunked(inp.q, inp.k, inp.v, inp.log_alpha, inp.beta,
+                                               initial_state=inp.initial_state, out=out,
+                                               final_state=sf, workspace=ws))
+    nbytes = B * T * H * (prefill_bytes_per_token_head() + 4 * (Dk - 1)) + 2 * B * state_bytes(H, Dk, Dk)
+    res["channel_prefill"] = {"workload": "nano_prefill_channel_b1_t4096_h16_d128", "ms": ms,
+                              "tokens_per_s": world * B * T / (ms * 1e-3),
+                              "hbm_frac": nbytes / (ms * 1e-3) / 1e9 / load_peaks()[0]}
+    del inp, ws, out, sf
+
+    # per-key-channel decode step at the decode shape: one step's inputs, 128 calls
+    din = rda_gen.decode_inputs(B=256, H=16, Dk=128, Dv=128, steps=1, seed=8, channel=True).to(device)
+    st = din.state.clone()
+    dout = torch.empty((256, 16, 128), dtype=din.q.dtype, device=device)
+
+    def ch_rep():
+        for _ in range(128):
+            rda.rda_decode_step(din.q[0], din.k[0], din.v[0], din.log_alpha[0], din.beta[0], st, out=dout)
+    ms = timed(ch_rep) / 128
+    bytes_step = 256 * 16 * (decode_bytes_per_seq_head(128, 128, 2) + 4 * 127)
+    res["channel_decode"] = {"workload": "decode_b256_h16_d128, per-key-channel decay", "ms_per_step": ms,
+                             "state_gbs": world * bytes_step / (ms * 1e-3) / 1e9,
+                             "hbm_frac": bytes_step / (ms * 1e-3) / 1e9 / load_peaks()[0]}
+    del din, st, dout
+
     # multi-token decode: the decode workload's first 128 tokens as calls of T tokens
     din = rda_gen.workload("decode_b256_h16_d128_128steps")
     st = din.state.to(device)

@@ -51,6 +51,12 @@ lib.rda_decode_tokens.argtypes = [_vp] * 8 + [_i] * 6 + [_f, _vp]
 lib.rda_decode_tokens.restype = _i
 lib.rda_read_device_error.argtypes = [_vp, ctypes.POINTER(_i), _vp]
 lib.rda_read_device_error.restype = _i
+lib.rda_prefill_chunked_channel.argtypes = lib.rda_prefill_chunked.argtypes
+lib.rda_prefill_chunked_channel.restype = _i
+lib.rda_prefill_varlen_channel.argtypes = lib.rda_prefill_varlen.argtypes
+lib.rda_prefill_varlen_channel.restype = _i
+lib.rda_decode_step_channel.argtypes = lib.rda_decode_step.argtypes
+lib.rda_decode_step_channel.restype = _i
 lib.rda_prefill_chunked_noalloc.argtypes = [_vp] * 9 + [_i] * 6 + [_f, _vp]
 lib.rda_prefill_chunked_noalloc.restype = _i
 lib.rda_debug_set_wait_fault.argtypes = [_i, ctypes.c_ulonglong]
@@ -127,7 +133,8 @@ def rda_prefill_chunked(q, k, v, log_alpha, beta, write_gate=None, initial_state
                         scale=1.0, out=None, final_state=None, return_final_state=True,
                         workspace=None, stream=None):
     """Fixed-length prefill.  q, k ``[B,T,H,Dk]``; v ``[B,T,H,Dv]``; gates fp32
-    ``[B,T,H]``; initial_state fp32 ``[B,H,Dk,Dv]`` or None.
+    ``[B,T,H]`` (log_alpha ``[B,T,H,Dk]`` for per-key-channel decay, which calls
+    ``rda_prefill_chunked_channel``); initial_state fp32 ``[B,H,Dk,Dv]`` or None.
 
     Returns ``(out [B,T,H,Dv], final_state [B,H,Dk,Dv] or None)``.
     """
@@ -138,8 +145,9 @@ def rda_prefill_chunked(q, k, v, log_alpha, beta, write_gate=None, initial_state
     dt = _dtype_code(q)
     if k.dtype != q.dtype or v.dtype != q.dtype:
         raise TypeError("rda: q, k and v must share a dtype")
-    if k.shape != q.shape or v.shape[:3] != (B, T, H) or log_alpha.shape != (B, T, H) \
-            or beta.shape != (B, T, H):
+    channel = log_alpha.dim() == 4
+    if k.shape != q.shape or v.shape[:3] != (B, T, H) or beta.shape != (B, T, H) \
+            or log_alpha.shape != ((B, T, H, Dk) if channel else (B, T, H)):
         raise ValueError("rda: inconsistent shapes")
     if out is None:
         out = torch.empty((B, T, H, Dv), dtype=q.dtype, device=q.device)
@@ -147,11 +155,12 @@ def rda_prefill_chunked(q, k, v, log_alpha, beta, write_gate=None, initial_state
         final_state = torch.empty((B, H, Dk, Dv), dtype=torch.float32, device=q.device)
     if workspace is None:
         workspace = new_workspace(rda_prefill_workspace_bytes(B, T, H, Dk, Dv, 0), q.device)
-    code = lib.rda_prefill_chunked(_ptr(q), _ptr(k), _ptr(v), _ptr(log_alpha), _ptr(beta),
-                                   _ptr(write_gate), _ptr(initial_state), _ptr(final_state),
-                                   _ptr(out), dt, B, T, H, Dk, Dv, float(scale),
-                                   _ptr(workspace), workspace.numel(), _stream(stream))
-    _check(code, "rda_prefill_chunked")
+    fn = lib.rda_prefill_chunked_channel if channel else lib.rda_prefill_chunked
+    code = fn(_ptr(q), _ptr(k), _ptr(v), _ptr(log_alpha), _ptr(beta),
+              _ptr(write_gate), _ptr(initial_state), _ptr(final_state),
+              _ptr(out), dt, B, T, H, Dk, Dv, float(scale),
+              _ptr(workspace), workspace.numel(), _stream(stream))
+    _check(code, fn.__name__)
     return out, final_state
 
 
@@ -160,7 +169,8 @@ def rda_prefill_varlen(q, k, v, log_alpha, beta, cu_seqlens, write_gate=None,
                        return_final_states=True, cu_seqlens_host=None, workspace=None,
                        stream=None):
     """Packed prefill.  q, k ``[total,H,Dk]``; v ``[total,H,Dv]``; gates
-    ``[total,H]``; cu_seqlens int32 CUDA ``[N+1]``; cu_seqlens_host optional
+    ``[total,H]`` (log_alpha ``[total,H,Dk]`` for per-key-channel decay);
+    cu_seqlens int32 CUDA ``[N+1]``; cu_seqlens_host optional
     int32 CPU mirror (enables longest-first scheduling).
 
     Returns ``(out [total,H,Dv], final_states [N,H,Dk,Dv] or None)``.
@@ -186,18 +196,20 @@ def rda_prefill_varlen(q, k, v, log_alpha, beta, cu_seqlens, write_gate=None,
         if cu_seqlens_host.is_cuda:
             raise ValueError("rda: cu_seqlens_host must be a CPU tensor")
         host_ptr = ctypes.c_void_p(cu_seqlens_host.data_ptr())
-    code = lib.rda_prefill_varlen(_ptr(q), _ptr(k), _ptr(v), _ptr(log_alpha), _ptr(beta),
-                                  _ptr(write_gate), _ptr(cu_seqlens), host_ptr, N, total,
-                                  _ptr(initial_states), _ptr(final_states), _ptr(out), dt, H, Dk,
-                                  Dv, float(scale), _ptr(workspace), workspace.numel(),
-                                  _stream(stream))
-    _check(code, "rda_prefill_varlen")
+    fn = lib.rda_prefill_varlen_channel if log_alpha.dim() == 3 else lib.rda_prefill_varlen
+    code = fn(_ptr(q), _ptr(k), _ptr(v), _ptr(log_alpha), _ptr(beta),
+              _ptr(write_gate), _ptr(cu_seqlens), host_ptr, N, total,
+              _ptr(initial_states), _ptr(final_states), _ptr(out), dt, H, Dk,
+              Dv, float(scale), _ptr(workspace), workspace.numel(),
+              _stream(stream))
+    _check(code, fn.__name__)
     return out, final_states
 
 
 def rda_decode_step(q, k, v, log_alpha, beta, state, write_gate=None, scale=1.0, out=None,
                     stream=None):
-    """One decode step.  q, k ``[B,H,Dk]``; v ``[B,H,Dv]``; gates fp32 ``[B,H]``;
+    """One decode step.  q, k ``[B,H,Dk]``; v ``[B,H,Dv]``; gates fp32 ``[B,H]``
+    (log_alpha ``[B,H,Dk]`` for per-key-channel decay);
     state fp32 ``[B,H,Dk,Dv]`` updated in place.  Returns ``out [B,H,Dv]``."""
     B, H, Dk = q.shape
     Dv = v.shape[-1]
@@ -206,10 +218,11 @@ def rda_decode_step(q, k, v, log_alpha, beta, state, write_gate=None, scale=1.0,
     dt = _dtype_code(q)
     if out is None:
         out = torch.empty((B, H, Dv), dtype=q.dtype, device=q.device)
-    code = lib.rda_decode_step(_ptr(q), _ptr(k), _ptr(v), _ptr(log_alpha), _ptr(beta),
-                               _ptr(write_gate), _ptr(state), _ptr(out), dt, B, H, Dk, Dv,
-                               float(scale), _stream(stream))
-    _check(code, "rda_decode_step")
+    fn = lib.rda_decode_step_channel if log_alpha.dim() == 3 else lib.rda_decode_step
+    code = fn(_ptr(q), _ptr(k), _ptr(v), _ptr(log_alpha), _ptr(beta),
+              _ptr(write_gate), _ptr(state), _ptr(out), dt, B, H, Dk, Dv,
+              float(scale), _stream(stream))
+    _check(code, fn.__name__)
     return out
 
 

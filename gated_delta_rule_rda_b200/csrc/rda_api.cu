@@ -61,7 +61,7 @@ WaitSettings wait_settings() { return WaitSettings{g_wait_ns.load(), g_drop_chun
 rda_status_t validate_prefill_chunked(const void *q, const void *k, const void *v, const float *log_alpha,
                                       const float *beta, const float *write_gate, const float *initial_state,
                                       const float *final_state, const void *out, rda_dtype_t dtype, int B,
-                                      int T, int H, int Dk, int Dv, size_t *scratch_bytes) {
+                                      int T, int H, int Dk, int Dv, size_t *scratch_bytes, bool channel) {
     if (dtype != RDA_F32 && dtype != RDA_BF16) return RDA_ERR_UNSUPPORTED;
     if (B < 0 || T < 0 || H <= 0) return RDA_ERR_INVALID_ARG;
     if (!dims_ok(Dk, Dv)) return RDA_ERR_UNSUPPORTED;
@@ -74,7 +74,8 @@ rda_status_t validate_prefill_chunked(const void *q, const void *k, const void *
         rda_status_t st = check_io_ptrs(q, k, v, log_alpha, beta, out);
         if (st != RDA_OK) return st;
     }
-    *scratch_bytes = chunked_supported(dtype, Dk, Dv) ? workspace_bytes(B, T, H, Dk, Dv, 0) : kErrorWordBytes;
+    *scratch_bytes = (chunked_supported(dtype, Dk, Dv) && !channel) ? workspace_bytes(B, T, H, Dk, Dv, 0)
+                                                                   : kErrorWordBytes;
     return RDA_OK;
 }
 
@@ -102,7 +103,7 @@ size_t rda_prefill_workspace_bytes(int B, int T, int H, int Dk, int Dv, int num_
     return workspace_bytes(B, T, H, Dk, Dv, num_seqs);
 }
 
-rda_status_t rda_prefill_chunked(const void *q, const void *k, const void *v,
+static rda_status_t prefill_chunked_impl(bool channel, const void *q, const void *k, const void *v,
                                  const float *log_alpha, const float *beta,
                                  const float *write_gate,
                                  const float *initial_state, float *final_state,
@@ -111,7 +112,7 @@ rda_status_t rda_prefill_chunked(const void *q, const void *k, const void *v,
                                  void *workspace, size_t workspace_bytes_given, void *stream) {
     size_t need = 0;
     rda_status_t st = validate_prefill_chunked(q, k, v, log_alpha, beta, write_gate, initial_state, final_state,
-                                               out, dtype, B, T, H, Dk, Dv, &need);
+                                               out, dtype, B, T, H, Dk, Dv, &need, channel);
     if (st != RDA_OK) return st;
     if (!workspace || workspace_bytes_given < need) return RDA_ERR_WORKSPACE;
     if (!aligned(workspace, 256)) return RDA_ERR_MISALIGNED;
@@ -138,13 +139,36 @@ rda_status_t rda_prefill_chunked(const void *q, const void *k, const void *v,
     const WaitSettings ws = wait_settings();
     a.wait_ns = ws.wait_ns;
     a.debug_drop_chunk = ws.drop_chunk;
-    cudaError_t e = chunked_supported(dtype, Dk, Dv)
+    a.channel_decay = channel;
+    cudaError_t e = (chunked_supported(dtype, Dk, Dv) && !channel)
                         ? launch_chunked(a, static_cast<char *>(workspace) + kErrorWordBytes, s)
                         : launch_recurrent(a, dtype, s);
     return e == cudaSuccess ? RDA_OK : RDA_ERR_CUDA;
 }
 
-rda_status_t rda_prefill_varlen(const void *q, const void *k, const void *v,
+rda_status_t rda_prefill_chunked(const void *q, const void *k, const void *v,
+                                 const float *log_alpha, const float *beta,
+                                 const float *write_gate,
+                                 const float *initial_state, float *final_state,
+                                 void *out, rda_dtype_t dtype,
+                                 int B, int T, int H, int Dk, int Dv, float scale,
+                                 void *workspace, size_t workspace_bytes_given, void *stream) {
+    return prefill_chunked_impl(false, q, k, v, log_alpha, beta, write_gate, initial_state, final_state, out,
+                                dtype, B, T, H, Dk, Dv, scale, workspace, workspace_bytes_given, stream);
+}
+
+rda_status_t rda_prefill_chunked_channel(const void *q, const void *k, const void *v,
+                                         const float *log_alpha, const float *beta,
+                                         const float *write_gate,
+                                         const float *initial_state, float *final_state,
+                                         void *out, rda_dtype_t dtype,
+                                         int B, int T, int H, int Dk, int Dv, float scale,
+                                         void *workspace, size_t workspace_bytes_given, void *stream) {
+    return prefill_chunked_impl(true, q, k, v, log_alpha, beta, write_gate, initial_state, final_state, out,
+                                dtype, B, T, H, Dk, Dv, scale, workspace, workspace_bytes_given, stream);
+}
+
+static rda_status_t prefill_varlen_impl(bool channel, const void *q, const void *k, const void *v,
                                 const float *log_alpha, const float *beta,
                                 const float *write_gate,
                                 const int32_t *cu_seqlens, const int32_t *cu_seqlens_host,
@@ -159,7 +183,7 @@ rda_status_t rda_prefill_varlen(const void *q, const void *k, const void *v,
     if (!sizes_ok(total_T, H, Dk, Dv)) return RDA_ERR_INVALID_ARG;
     if ((long long)num_seqs * H * Dk * Dv >= (1LL << 31)) return RDA_ERR_INVALID_ARG;
     if (num_seqs > 0 && !cu_seqlens) return RDA_ERR_INVALID_ARG;
-    const bool chunked = chunked_supported(dtype, Dk, Dv);
+    const bool chunked = chunked_supported(dtype, Dk, Dv) && !channel;
     const size_t need = chunked ? workspace_bytes(1, total_T, H, Dk, Dv, num_seqs)
                                 : kErrorWordBytes + order_bytes(num_seqs);
     if (!workspace || workspace_bytes_given < need) return RDA_ERR_WORKSPACE;
@@ -202,13 +226,42 @@ rda_status_t rda_prefill_varlen(const void *q, const void *k, const void *v,
     const WaitSettings ws = wait_settings();
     a.wait_ns = ws.wait_ns;
     a.debug_drop_chunk = ws.drop_chunk;
+    a.channel_decay = channel;
     cudaError_t e = chunked
         ? launch_chunked(a, static_cast<char *>(workspace) + kErrorWordBytes + order_bytes(num_seqs), s)
         : launch_recurrent(a, dtype, s);
     return e == cudaSuccess ? RDA_OK : RDA_ERR_CUDA;
 }
 
-rda_status_t rda_decode_step(const void *q, const void *k, const void *v,
+rda_status_t rda_prefill_varlen(const void *q, const void *k, const void *v,
+                                const float *log_alpha, const float *beta,
+                                const float *write_gate,
+                                const int32_t *cu_seqlens, const int32_t *cu_seqlens_host,
+                                int num_seqs, int total_T,
+                                const float *initial_states, float *final_states,
+                                void *out, rda_dtype_t dtype,
+                                int H, int Dk, int Dv, float scale,
+                                void *workspace, size_t workspace_bytes_given, void *stream) {
+    return prefill_varlen_impl(false, q, k, v, log_alpha, beta, write_gate, cu_seqlens, cu_seqlens_host, num_seqs,
+                               total_T, initial_states, final_states, out, dtype, H, Dk, Dv, scale, workspace,
+                               workspace_bytes_given, stream);
+}
+
+rda_status_t rda_prefill_varlen_channel(const void *q, const void *k, const void *v,
+                                        const float *log_alpha, const float *beta,
+                                        const float *write_gate,
+                                        const int32_t *cu_seqlens, const int32_t *cu_seqlens_host,
+                                        int num_seqs, int total_T,
+                                        const float *initial_states, float *final_states,
+                                        void *out, rda_dtype_t dtype,
+                                        int H, int Dk, int Dv, float scale,
+                                        void *workspace, size_t workspace_bytes_given, void *stream) {
+    return prefill_varlen_impl(true, q, k, v, log_alpha, beta, write_gate, cu_seqlens, cu_seqlens_host, num_seqs,
+                               total_T, initial_states, final_states, out, dtype, H, Dk, Dv, scale, workspace,
+                               workspace_bytes_given, stream);
+}
+
+static rda_status_t decode_step_impl(bool channel, const void *q, const void *k, const void *v,
                              const float *log_alpha, const float *beta,
                              const float *write_gate,
                              float *state, void *out, rda_dtype_t dtype,
@@ -228,7 +281,26 @@ rda_status_t rda_decode_step(const void *q, const void *k, const void *v,
     a.log_alpha = log_alpha; a.beta = beta; a.gamma = write_gate;
     a.state = state; a.out = out;
     a.B = B; a.H = H; a.Dk = Dk; a.Dv = Dv; a.scale = scale;
+    a.channel_decay = channel;
     return launch_decode(a, dtype, static_cast<cudaStream_t>(stream)) == cudaSuccess ? RDA_OK : RDA_ERR_CUDA;
+}
+
+rda_status_t rda_decode_step(const void *q, const void *k, const void *v,
+                             const float *log_alpha, const float *beta,
+                             const float *write_gate,
+                             float *state, void *out, rda_dtype_t dtype,
+                             int B, int H, int Dk, int Dv, float scale, void *stream) {
+    return decode_step_impl(false, q, k, v, log_alpha, beta, write_gate, state, out, dtype, B, H, Dk, Dv, scale,
+                            stream);
+}
+
+rda_status_t rda_decode_step_channel(const void *q, const void *k, const void *v,
+                                     const float *log_alpha, const float *beta,
+                                     const float *write_gate,
+                                     float *state, void *out, rda_dtype_t dtype,
+                                     int B, int H, int Dk, int Dv, float scale, void *stream) {
+    return decode_step_impl(true, q, k, v, log_alpha, beta, write_gate, state, out, dtype, B, H, Dk, Dv, scale,
+                            stream);
 }
 
 rda_status_t rda_decode_tokens(const void *q, const void *k, const void *v,

@@ -11,6 +11,11 @@
 // The step is bound by HBM: 2 * Dk * Dv * 4 bytes of state per (sequence,
 // head) against a few hundred bytes of token data.
 //
+// Per-key-channel decay (log alpha [B, H, Dk]): the decayed state is
+// S_old diag(alpha) in the math orientation, i.e. row i of the [Dk][Dv]
+// storage scales by alpha_i; with a = S_old (alpha o k), b = S_old (alpha o q):
+//     e = gamma v - a,  o = scale (b + beta (k.q) e),  S_new = S_old diag(alpha) + beta e k^T.
+//
 // Layout of the work: one CTA per (sequence, head).  The state block
 // [Dk][Dv] is row-major, so a warp reads whole rows with 16-byte loads
 // (perfectly coalesced); each thread owns 4 value columns of DK/RG rows and
@@ -24,7 +29,7 @@ namespace {
 
 constexpr int kThreads = 256;
 
-template <typename Tio, int DK, int DV>
+template <typename Tio, int DK, int DV, bool CH>
 __global__ void __launch_bounds__(kThreads, 2)
 decode_kernel(DecodeArgs a) {
     constexpr int TPR = DV / 4;              // threads across one state row
@@ -32,6 +37,7 @@ decode_kernel(DecodeArgs a) {
     constexpr int R = DK / RG;               // rows per thread
     __shared__ float k_s[DK];
     __shared__ float q_s[DK];
+    __shared__ float a_s[CH ? DK : 1];       // per-channel alpha
     __shared__ float4 red_a[RG][TPR];
     __shared__ float4 red_b[RG][TPR];
     __shared__ float kq_s;
@@ -52,9 +58,10 @@ decode_kernel(DecodeArgs a) {
     for (int i = threadIdx.x; i < DK; i += kThreads) {
         k_s[i] = Io<Tio>::ld(k + i);
         q_s[i] = Io<Tio>::ld(q + i);
+        if constexpr (CH) a_s[i] = expf(a.log_alpha[(size_t)bh * DK + i]);
     }
     const float4 vv = Io<Tio>::ld4(static_cast<const Tio *>(a.v) + (size_t)bh * DV + 4 * col4);
-    const float al = expf(a.log_alpha[bh]);
+    const float al = CH ? 1.f : expf(a.log_alpha[bh]);
     const float be = a.beta[bh];
     const float ga = a.gamma ? a.gamma[bh] : 1.f;
     __syncthreads();
@@ -70,7 +77,8 @@ decode_kernel(DecodeArgs a) {
     float4 pa = make_float4(0.f, 0.f, 0.f, 0.f), pb = pa;
 #pragma unroll
     for (int r = 0; r < R; ++r) {
-        const float kr = k_s[rg + RG * r], qr = q_s[rg + RG * r];
+        const float ar = CH ? a_s[rg + RG * r] : 1.f;
+        const float kr = ar * k_s[rg + RG * r], qr = ar * q_s[rg + RG * r];
         pa.x = fmaf(S[r].x, kr, pa.x); pa.y = fmaf(S[r].y, kr, pa.y);
         pa.z = fmaf(S[r].z, kr, pa.z); pa.w = fmaf(S[r].w, kr, pa.w);
         pb.x = fmaf(S[r].x, qr, pb.x); pb.y = fmaf(S[r].y, qr, pb.y);
@@ -107,22 +115,23 @@ decode_kernel(DecodeArgs a) {
 #pragma unroll
     for (int r = 0; r < R; ++r) {
         const float kr = k_s[rg + RG * r];
+        const float ar = CH ? a_s[rg + RG * r] : al;
         float4 s = S[r];
-        s.x = fmaf(al, s.x, be4.x * kr);
-        s.y = fmaf(al, s.y, be4.y * kr);
-        s.z = fmaf(al, s.z, be4.z * kr);
-        s.w = fmaf(al, s.w, be4.w * kr);
+        s.x = fmaf(ar, s.x, be4.x * kr);
+        s.y = fmaf(ar, s.y, be4.y * kr);
+        s.z = fmaf(ar, s.z, be4.z * kr);
+        s.w = fmaf(ar, s.w, be4.w * kr);
         __stcs(reinterpret_cast<float4 *>(st + (size_t)(rg + RG * r) * DV) + col4, s);
     }
 }
 
-template <typename Tio>
+template <typename Tio, bool CH>
 cudaError_t launch_t(const DecodeArgs &a, cudaStream_t s) {
     const unsigned grid = (unsigned)(a.B * a.H);
-    if (a.Dk == 128 && a.Dv == 128) decode_kernel<Tio, 128, 128><<<grid, kThreads, 0, s>>>(a);
-    else if (a.Dk == 128 && a.Dv == 64) decode_kernel<Tio, 128, 64><<<grid, kThreads, 0, s>>>(a);
-    else if (a.Dk == 64 && a.Dv == 128) decode_kernel<Tio, 64, 128><<<grid, kThreads, 0, s>>>(a);
-    else decode_kernel<Tio, 64, 64><<<grid, kThreads, 0, s>>>(a);
+    if (a.Dk == 128 && a.Dv == 128) decode_kernel<Tio, 128, 128, CH><<<grid, kThreads, 0, s>>>(a);
+    else if (a.Dk == 128 && a.Dv == 64) decode_kernel<Tio, 128, 64, CH><<<grid, kThreads, 0, s>>>(a);
+    else if (a.Dk == 64 && a.Dv == 128) decode_kernel<Tio, 64, 128, CH><<<grid, kThreads, 0, s>>>(a);
+    else decode_kernel<Tio, 64, 64, CH><<<grid, kThreads, 0, s>>>(a);
     return cudaGetLastError();
 }
 
@@ -130,7 +139,9 @@ cudaError_t launch_t(const DecodeArgs &a, cudaStream_t s) {
 
 cudaError_t launch_decode(const DecodeArgs &a, rda_dtype_t dtype, cudaStream_t s) {
     if (a.B == 0) return cudaSuccess;
-    return dtype == RDA_F32 ? launch_t<float>(a, s) : launch_t<__nv_bfloat16>(a, s);
+    if (a.channel_decay)
+        return dtype == RDA_F32 ? launch_t<float, true>(a, s) : launch_t<__nv_bfloat16, true>(a, s);
+    return dtype == RDA_F32 ? launch_t<float, false>(a, s) : launch_t<__nv_bfloat16, false>(a, s);
 }
 
 }  // namespace rda

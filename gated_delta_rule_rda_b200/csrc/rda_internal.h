@@ -33,6 +33,7 @@ struct PrefillArgs {
     int32_t *err;                // device error word
     uint64_t wait_ns;            // bound of every device-side wait
     int debug_drop_chunk;        // fault injection (tests only): the scan never fills this chunk; -1 = off
+    bool channel_decay;          // log_alpha is per key channel: [tokens, H, Dk]
     // chunked path only (filled by launch_chunked)
     const int32_t *chunk_base;   // packed: first global chunk of each sequence [N+1]
     uint8_t *workspace_chunks;   // per (chunk, head) prep results
@@ -47,6 +48,7 @@ struct DecodeArgs {
     int B, H, Dk, Dv;
     float scale;
     int T;                       // tokens per sequence (multi-token decode only)
+    bool channel_decay;          // log_alpha is per key channel: [B, H, Dk]
 };
 
 // Bound of the device-side waits, and the test-only fault injection, as set by
@@ -73,10 +75,10 @@ size_t chunked_workspace_bytes(long total_T, int T, int B, int H, int Dv, int nu
 // Host-side argument checks of rda_prefill_chunked except those of the
 // workspace; enqueues nothing.  On RDA_OK, *scratch_bytes is the workspace
 // that call needs for these arguments (the error word alone on the
-// token-sequential path).
+// token-sequential path).  `channel`: per-key-channel log alpha [.., T, H, Dk].
 rda_status_t validate_prefill_chunked(const void *q, const void *k, const void *v, const float *log_alpha,
                                       const float *beta, const float *write_gate, const float *initial_state,
                                       const float *final_state, const void *out, rda_dtype_t dtype, int B,
-                                      int T, int H, int Dk, int Dv, size_t *scratch_bytes);
+                                      int T, int H, int Dk, int Dv, size_t *scratch_bytes, bool channel = false);
 
 }  // namespace rda

@@ -14,7 +14,15 @@
 // columns each and split the key rows across lanes; the two reductions over
 // the key dimension are warp butterflies.
 //
-// This path serves fp32 inputs (held to fp32 accuracy) and bf16 with Dk = 64.
+// With per-key-channel decay (log alpha [.., T, H, Dk]; key dim i of the state
+// decays by alpha_i) the decayed state is S diag(alpha), so the same identity
+// holds with the two reductions taken against alpha o k and alpha o q, the
+// key-query product k.q unchanged, and each key row decayed by its own alpha:
+//     e = gamma v - S (alpha o k),  o = scale (S (alpha o q) + beta (k.q) e),
+//     S <- S diag(alpha) + beta e k^T
+//
+// This path serves fp32 inputs (held to fp32 accuracy), bf16 with Dk = 64, and
+// every per-key-channel call.
 #include "rda_internal.h"
 #include "rda_io.cuh"
 
@@ -26,12 +34,13 @@ constexpr int kCols = 32;          // value columns per CTA
 constexpr int kColsPerWarp = 4;
 constexpr int kTile = 16;          // tokens staged in shared memory at a time
 
-template <typename Tio, int DK>
+template <typename Tio, int DK, bool CH>
 __global__ void __launch_bounds__(kThreads)
 recurrent_kernel(PrefillArgs a) {
     constexpr int R = DK / 32;     // key rows per lane
     __shared__ float k_s[kTile][DK];
     __shared__ float q_s[kTile][DK];
+    __shared__ float a_s[CH ? kTile : 1][DK];   // per-channel alpha
     __shared__ float v_s[kTile][kCols];
     __shared__ float o_s[kTile][kCols];
     __shared__ float g_s[kTile][3];    // alpha, beta, gamma
@@ -73,6 +82,7 @@ recurrent_kernel(PrefillArgs a) {
             const size_t row = (size_t)(t0 + tb + tt) * H + h;
             k_s[tt][d] = Io<Tio>::ld(k + row * DK + d);
             q_s[tt][d] = Io<Tio>::ld(q + row * DK + d);
+            if constexpr (CH) a_s[tt][d] = expf(a.log_alpha[row * DK + d]);
         }
         for (int idx = threadIdx.x; idx < nt * kCols; idx += kThreads) {
             const int tt = idx / kCols, c = idx % kCols;
@@ -81,18 +91,21 @@ recurrent_kernel(PrefillArgs a) {
         }
         if (threadIdx.x < nt) {
             const size_t row = (size_t)(t0 + tb + threadIdx.x) * H + h;
-            g_s[threadIdx.x][0] = expf(a.log_alpha[row]);
+            g_s[threadIdx.x][0] = CH ? 1.f : expf(a.log_alpha[row]);
             g_s[threadIdx.x][1] = a.beta[row];
             g_s[threadIdx.x][2] = a.gamma ? a.gamma[row] : 1.f;
         }
         __syncthreads();
 
         for (int tt = 0; tt < nt; ++tt) {
-            float kk[R], qq[R];
+            float kk[R], qq[R], ka[R], qa[R], ar[R];
 #pragma unroll
             for (int r = 0; r < R; ++r) {
                 kk[r] = k_s[tt][lane + 32 * r];
                 qq[r] = q_s[tt][lane + 32 * r];
+                ar[r] = CH ? a_s[tt][lane + 32 * r] : 1.f;
+                ka[r] = CH ? ar[r] * kk[r] : kk[r];
+                qa[r] = CH ? ar[r] * qq[r] : qq[r];
             }
             float red[9];
 #pragma unroll
@@ -100,8 +113,8 @@ recurrent_kernel(PrefillArgs a) {
                 float sa = 0.f, sb = 0.f;
 #pragma unroll
                 for (int r = 0; r < R; ++r) {
-                    sa = fmaf(S[r][c], kk[r], sa);
-                    sb = fmaf(S[r][c], qq[r], sb);
+                    sa = fmaf(S[r][c], ka[r], sa);
+                    sb = fmaf(S[r][c], qa[r], sb);
                 }
                 red[c] = sa;
                 red[4 + c] = sb;
@@ -124,7 +137,7 @@ recurrent_kernel(PrefillArgs a) {
                 if (lane == c) o_mine = o;
                 const float bee = be * e;
 #pragma unroll
-                for (int r = 0; r < R; ++r) S[r][c] = fmaf(al, S[r][c], bee * kk[r]);
+                for (int r = 0; r < R; ++r) S[r][c] = fmaf(CH ? ar[r] : al, S[r][c], bee * kk[r]);
             }
             if (lane < 4) o_s[tt][jw + lane] = o_mine;
         }
@@ -144,13 +157,13 @@ recurrent_kernel(PrefillArgs a) {
     }
 }
 
-template <typename Tio>
+template <typename Tio, bool CH>
 cudaError_t launch_t(const PrefillArgs &a, cudaStream_t s) {
     dim3 grid(a.Dv / kCols, a.H, a.num_seqs);
     if (a.Dk == 128)
-        recurrent_kernel<Tio, 128><<<grid, kThreads, 0, s>>>(a);
+        recurrent_kernel<Tio, 128, CH><<<grid, kThreads, 0, s>>>(a);
     else
-        recurrent_kernel<Tio, 64><<<grid, kThreads, 0, s>>>(a);
+        recurrent_kernel<Tio, 64, CH><<<grid, kThreads, 0, s>>>(a);
     return cudaGetLastError();
 }
 
@@ -158,7 +171,9 @@ cudaError_t launch_t(const PrefillArgs &a, cudaStream_t s) {
 
 cudaError_t launch_recurrent(const PrefillArgs &a, rda_dtype_t dtype, cudaStream_t s) {
     if (a.num_seqs == 0) return cudaSuccess;
-    return dtype == RDA_F32 ? launch_t<float>(a, s) : launch_t<__nv_bfloat16>(a, s);
+    if (a.channel_decay)
+        return dtype == RDA_F32 ? launch_t<float, true>(a, s) : launch_t<__nv_bfloat16, true>(a, s);
+    return dtype == RDA_F32 ? launch_t<float, false>(a, s) : launch_t<__nv_bfloat16, false>(a, s);
 }
 
 }  // namespace rda

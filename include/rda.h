@@ -203,6 +203,53 @@ rda_status_t rda_decode_tokens(const void *q, const void *k, const void *v,
                                int B, int T, int H, int Dk, int Dv, float scale, void *stream);
 
 /*
+ * PER-KEY-CHANNEL DECAY
+ *
+ * The model printout in the "tiny-random/raon-1-mini" README (section
+ * "Printing the model") gives the RDA layer decay projections f_a_proj /
+ * f_b_proj whose output is as wide as heads x key dims, and the blog post on
+ * Raon-1 mini (architecture section) and the nano article (section "The other
+ * 1.5B") describe RDA as a modification of Kimi Delta Attention, whose decay is
+ * per key channel.  These three calls take that form: log_alpha holds one
+ * decay per key dimension, and key dimension i of the state decays by alpha_i
+ * (the same order: decay, error against the decayed state, write, read):
+ *
+ *     S_t = S_{t-1} diag(alpha_t) (I - beta_t k_t k_t^T) + beta_t (gamma_t v_t) k_t^T
+ *     o_t = scale * S_t q_t
+ *
+ * With every alpha_t[i] equal this is the scalar rule above.  Arguments,
+ * layouts, results and errors are those of the scalar calls except:
+ *   log_alpha  device fp32 [B,T,H,Dk] (varlen: [total_T,H,Dk]; decode: [B,H,Dk]),
+ *              each value in [-5, 0] (precondition, not checked)
+ * The prefill calls evaluate the rule token by token in fp32 (any dtype,
+ * Dk and Dv in {64, 128}); they need only the error word of the workspace
+ * but accept any workspace of at least rda_prefill_workspace_bytes(...).
+ */
+rda_status_t rda_prefill_chunked_channel(const void *q, const void *k, const void *v,
+                                         const float *log_alpha, const float *beta,
+                                         const float *write_gate,
+                                         const float *initial_state, float *final_state,
+                                         void *out, rda_dtype_t dtype,
+                                         int B, int T, int H, int Dk, int Dv, float scale,
+                                         void *workspace, size_t workspace_bytes, void *stream);
+
+rda_status_t rda_prefill_varlen_channel(const void *q, const void *k, const void *v,
+                                        const float *log_alpha, const float *beta,
+                                        const float *write_gate,
+                                        const int32_t *cu_seqlens, const int32_t *cu_seqlens_host,
+                                        int num_seqs, int total_T,
+                                        const float *initial_states, float *final_states,
+                                        void *out, rda_dtype_t dtype,
+                                        int H, int Dk, int Dv, float scale,
+                                        void *workspace, size_t workspace_bytes, void *stream);
+
+rda_status_t rda_decode_step_channel(const void *q, const void *k, const void *v,
+                                     const float *log_alpha, const float *beta,
+                                     const float *write_gate,
+                                     float *state, void *out, rda_dtype_t dtype,
+                                     int B, int H, int Dk, int Dv, float scale, void *stream);
+
+/*
  * Fixed-length prefill that allocates nothing and takes no workspace.
  *
  * The pages describe no such call; it exists for callers that cannot give the

@@ -55,6 +55,8 @@ def draw_log_alpha(rng, shape, decay: str):
         return -_softplus(_normal(rng, shape) + 2.0) * 0.1
     if decay == "uniform":
         return np.log(rng.uniform(0.90, 0.9999, size=shape))
+    if decay == "strong":   # the decay's lower bound region: log alpha in [-5, -4]
+        return rng.uniform(-5.0, -4.0, size=shape)
     raise ValueError(f"unknown decay distribution {decay!r}")
 
 
@@ -77,14 +79,15 @@ class Inputs:
 
 
 def fixed_inputs(B, T, H, Dk, Dv, dtype=torch.bfloat16, seed=0, s0=True, decay="softplus",
-                 gamma=False) -> Inputs:
-    """Draws one fixed-length batch (see module docstring for the recipe)."""
+                 gamma=False, channel=False) -> Inputs:
+    """Draws one fixed-length batch (see module docstring for the recipe).
+    With ``channel`` log_alpha is drawn per key channel, ``[B,T,H,Dk]``."""
     rng = np.random.Generator(np.random.PCG64(seed))
     q = _l2norm_last(_normal(rng, (B, T, H, Dk)))
     k = _l2norm_last(_normal(rng, (B, T, H, Dk)))
     v = _normal(rng, (B, T, H, Dv))
     beta = _sigmoid(_normal(rng, (B, T, H)))
-    la = draw_log_alpha(rng, (B, T, H), decay)
+    la = draw_log_alpha(rng, (B, T, H, Dk) if channel else (B, T, H), decay)
     st = _normal(rng, (B, H, Dk, Dv)) * S0_STD if s0 else None
     ga = None
     if gamma:
@@ -94,7 +97,8 @@ def fixed_inputs(B, T, H, Dk, Dv, dtype=torch.bfloat16, seed=0, s0=True, decay="
         ga = _to(_sigmoid(braw + d) / _sigmoid(braw), torch.float32)
     return Inputs(_to(q, dtype), _to(k, dtype), _to(v, dtype), _to(la, torch.float32),
                   _to(beta, torch.float32), None if st is None else _to(st, torch.float32), ga,
-                  dict(B=B, T=T, H=H, Dk=Dk, Dv=Dv, dtype=dtype, seed=seed, decay=decay))
+                  dict(B=B, T=T, H=H, Dk=Dk, Dv=Dv, dtype=dtype, seed=seed, decay=decay,
+                       channel=channel))
 
 
 @dataclass
@@ -119,7 +123,7 @@ class VarlenInputs:
 
 def varlen_inputs(lengths=None, H=16, Dk=128, Dv=128, dtype=torch.bfloat16, seed=5,
                   num_seqs=64, min_len=128, max_len=8192, s0=True, decay="softplus",
-                  gamma=False) -> VarlenInputs:
+                  gamma=False, channel=False) -> VarlenInputs:
     """Draws packed sequences.  Lengths are drawn first (integers, both ends
     inclusive) unless given; then per-token tensors are drawn sequence by
     sequence in the module's order, so peak host memory stays bounded."""
@@ -134,7 +138,7 @@ def varlen_inputs(lengths=None, H=16, Dk=128, Dv=128, dtype=torch.bfloat16, seed
     q = torch.empty((total, H, Dk), dtype=dtype)
     k = torch.empty((total, H, Dk), dtype=dtype)
     v = torch.empty((total, H, Dv), dtype=dtype)
-    la = torch.empty((total, H), dtype=torch.float32)
+    la = torch.empty((total, H, Dk) if channel else (total, H), dtype=torch.float32)
     be = torch.empty((total, H), dtype=torch.float32)
     for n in range(N):
         a, b = int(cu[n]), int(cu[n + 1])
@@ -143,7 +147,7 @@ def varlen_inputs(lengths=None, H=16, Dk=128, Dv=128, dtype=torch.bfloat16, seed
         k[a:b] = _to(_l2norm_last(_normal(rng, (L, H, Dk))), dtype)
         v[a:b] = _to(_normal(rng, (L, H, Dv)), dtype)
         be[a:b] = _to(_sigmoid(_normal(rng, (L, H))), torch.float32)
-        la[a:b] = _to(draw_log_alpha(rng, (L, H), decay), torch.float32)
+        la[a:b] = _to(draw_log_alpha(rng, (L, H, Dk) if channel else (L, H), decay), torch.float32)
     st = _to(_normal(rng, (N, H, Dk, Dv)) * S0_STD, torch.float32) if s0 else None
     ga = None
     if gamma:
@@ -174,13 +178,13 @@ class DecodeInputs:
 
 
 def decode_inputs(B=256, H=16, Dk=128, Dv=128, steps=128, dtype=torch.bfloat16, seed=4,
-                  decay="softplus") -> DecodeInputs:
+                  decay="softplus", channel=False) -> DecodeInputs:
     rng = np.random.Generator(np.random.PCG64(seed))
     q = _l2norm_last(_normal(rng, (steps, B, H, Dk)))
     k = _l2norm_last(_normal(rng, (steps, B, H, Dk)))
     v = _normal(rng, (steps, B, H, Dv))
     beta = _sigmoid(_normal(rng, (steps, B, H)))
-    la = draw_log_alpha(rng, (steps, B, H), decay)
+    la = draw_log_alpha(rng, (steps, B, H, Dk) if channel else (steps, B, H), decay)
     st = _normal(rng, (B, H, Dk, Dv)) * S0_STD
     return DecodeInputs(_to(q, dtype), _to(k, dtype), _to(v, dtype), _to(la, torch.float32),
                         _to(beta, torch.float32), _to(st, torch.float32),
@@ -205,6 +209,11 @@ WORKLOADS = {
     "varlen_64seqs_128to8192_h16_d128": dict(kind="varlen", num_seqs=64, min_len=128,
                                              max_len=8192, H=16, Dk=128, Dv=128,
                                              dtype=torch.bfloat16, seed=5, s0=True),
+    # per-key-channel decay at the nano shape: log alpha [B,T,H,Dk], each element
+    # drawn like the scalar decay
+    "nano_prefill_channel_b1_t4096_h16_d128": dict(kind="fixed", B=1, T=4096, H=16, Dk=128,
+                                                   Dv=128, dtype=torch.bfloat16, seed=7, s0=True,
+                                                   decay="softplus", channel=True),
 }
 
 

@@ -24,6 +24,8 @@ def _declared_functions():
 def test_header_declares_the_entry_points():
     names = _declared_functions()
     for want in ["rda_prefill_chunked", "rda_prefill_varlen", "rda_decode_step", "rda_decode_tokens",
+                 "rda_prefill_chunked_channel", "rda_prefill_varlen_channel", "rda_decode_step_channel",
+                 "rda_prefill_chunked_noalloc", "rda_debug_set_wait_fault",
                  "rda_prefill_workspace_bytes", "rda_read_device_error", "rda_status_string",
                  "rda_version"]:
         assert want in names
