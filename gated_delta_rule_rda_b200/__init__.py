@@ -59,12 +59,18 @@ lib.rda_decode_step_channel.argtypes = lib.rda_decode_step.argtypes
 lib.rda_decode_step_channel.restype = _i
 lib.rda_prefill_chunked_noalloc.argtypes = [_vp] * 9 + [_i] * 6 + [_f, _vp]
 lib.rda_prefill_chunked_noalloc.restype = _i
+lib.rda_prep_inputs.argtypes = [_vp] * 8 + [_vp, _vp, _vp, _i, _vp, _i, _i, _i, _i] + [_vp] * 6 + \
+    [_i, _i, _i, _i, _i, _vp]
+lib.rda_prep_inputs.restype = _i
+lib.rda_output_gate_norm.argtypes = [_vp, _vp, _vp, _f, _i, _vp, _i, ctypes.c_longlong, _i, _i, _vp]
+lib.rda_output_gate_norm.restype = _i
 lib.rda_debug_set_wait_fault.argtypes = [_i, ctypes.c_ulonglong]
 lib.rda_debug_set_wait_fault.restype = None
 
 RDA_OK = 0
 RDA_F32 = 0
 RDA_BF16 = 1
+RDA_ACT_NONE, RDA_ACT_SILU, RDA_ACT_SIGMOID = 0, 1, 2
 STATUS_NAMES = {0: "RDA_OK", 1: "RDA_ERR_INVALID_ARG", 2: "RDA_ERR_UNSUPPORTED",
                 3: "RDA_ERR_MISALIGNED", 4: "RDA_ERR_WORKSPACE", 5: "RDA_ERR_CUDA",
                 6: "RDA_ERR_TIMEOUT"}
@@ -267,6 +273,70 @@ def rda_prefill_chunked_noalloc(q, k, v, log_alpha, beta, write_gate=None, initi
     return out, final_state
 
 
+def rda_prep_inputs(q_raw, k_raw, v_raw, conv_w_q, conv_w_k, conv_w_v, beta_raw, log_alpha_raw,
+                    cu_seqlens=None, delta=None, conv_window_in=None, conv_window_out=None,
+                    conv_act=RDA_ACT_SILU, max_seqlen=None, stream=None):
+    """The steps before the core (short conv, q/k L2 norm, gates, log-decay clamp).
+
+    Fixed length: q_raw, k_raw ``[B,T,H,Dk]``, v_raw ``[B,T,H,Dv]``, beta_raw, delta
+    ``[B,T,H]``, log_alpha_raw ``[B,T,H]`` or ``[B,T,H,Dk]``.  Packed: the same
+    without B, plus ``cu_seqlens`` (int32 CUDA) and ``max_seqlen``.  Conv
+    windows are bf16 ``[N,3,H*(2Dk+Dv)]``.  Returns a dict with q, k, v, beta,
+    write_gate (None without delta) and log_alpha.
+    """
+    packed = cu_seqlens is not None
+    H, Dk = q_raw.shape[-2:]
+    Dv = v_raw.shape[-1]
+    if packed:
+        total = q_raw.shape[0]
+        N = cu_seqlens.numel() - 1
+        T = 0
+        if max_seqlen is None:
+            raise ValueError("rda: packed sequences need max_seqlen")
+    else:
+        N, T = q_raw.shape[:2]
+        total = N * T
+        max_seqlen = T
+    channel = log_alpha_raw.dim() == q_raw.dim()
+    _need_cuda(q_raw, k_raw, v_raw, conv_w_q, conv_w_k, conv_w_v, beta_raw, log_alpha_raw,
+               cu_seqlens, delta, conv_window_in, conv_window_out)
+    _need_f32(conv_w_q, conv_w_k, conv_w_v, beta_raw, log_alpha_raw, delta)
+    for w in (conv_window_in, conv_window_out):
+        if w is not None and w.dtype != torch.bfloat16:
+            raise TypeError("rda: the conv window is bfloat16")
+    dt = _dtype_code(q_raw)
+    q, k, v = torch.empty_like(q_raw), torch.empty_like(k_raw), torch.empty_like(v_raw)
+    beta = torch.empty_like(beta_raw)
+    gamma = None if delta is None else torch.empty_like(beta_raw)
+    la = torch.empty_like(log_alpha_raw)
+    code = lib.rda_prep_inputs(_ptr(q_raw), _ptr(k_raw), _ptr(v_raw), _ptr(conv_w_q), _ptr(conv_w_k),
+                               _ptr(conv_w_v), _ptr(conv_window_in), _ptr(conv_window_out),
+                               _ptr(beta_raw), _ptr(delta), _ptr(log_alpha_raw), int(channel),
+                               _ptr(cu_seqlens), N, T, int(max_seqlen), total,
+                               _ptr(q), _ptr(k), _ptr(v), _ptr(beta), _ptr(gamma), _ptr(la),
+                               dt, H, Dk, Dv, int(conv_act), _stream(stream))
+    _check(code, "rda_prep_inputs")
+    return dict(q=q, k=k, v=v, beta=beta, write_gate=gamma, log_alpha=la)
+
+
+def rda_output_gate_norm(o, g, norm_weight, eps=1e-5, gate_act=RDA_ACT_SIGMOID, out=None,
+                         stream=None):
+    """RMSNorm of the core's output over the head dimension times act(g).
+    o, g ``[..., H, Dv]`` (same dtype); norm_weight fp32 ``[Dv]``."""
+    _need_cuda(o, g, norm_weight, out)
+    _need_f32(norm_weight)
+    if g.shape != o.shape or g.dtype != o.dtype:
+        raise ValueError("rda: o and g must match")
+    H, Dv = o.shape[-2:]
+    tokens = o.numel() // (H * Dv)
+    if out is None:
+        out = torch.empty_like(o)
+    code = lib.rda_output_gate_norm(_ptr(o), _ptr(g), _ptr(norm_weight), float(eps), int(gate_act),
+                                    _ptr(out), _dtype_code(o), tokens, H, Dv, _stream(stream))
+    _check(code, "rda_output_gate_norm")
+    return out
+
+
 def rda_debug_set_wait_fault(drop_chunk=-1, wait_limit_ns=0):
     """Testing only: bound of the device-side waits and an injected stall of the
     scan (see include/rda.h); ``rda_debug_set_wait_fault()`` turns it off."""
@@ -281,6 +351,7 @@ def rda_read_device_error(workspace, stream=None) -> int:
 
 
 __all__ = ["rda_prefill_chunked", "rda_prefill_varlen", "rda_decode_step", "rda_decode_tokens",
+           "rda_prep_inputs", "rda_output_gate_norm",
            "rda_prefill_chunked_noalloc",
            "rda_read_device_error", "rda_debug_set_wait_fault", "rda_prefill_workspace_bytes", "new_workspace", "version",
            "RdaError", "lib", "LIB_PATH"]

@@ -329,6 +329,64 @@ rda_status_t rda_decode_tokens(const void *q, const void *k, const void *v,
                                                                                               : RDA_ERR_CUDA;
 }
 
+rda_status_t rda_prep_inputs(const void *q_raw, const void *k_raw, const void *v_raw,
+                             const float *conv_w_q, const float *conv_w_k, const float *conv_w_v,
+                             const void *conv_window_in, void *conv_window_out,
+                             const float *beta_raw, const float *delta,
+                             const float *log_alpha_raw, int channel_decay,
+                             const int32_t *cu_seqlens, int num_seqs, int seq_len, int max_seqlen, int total_T,
+                             void *q, void *k, void *v, float *beta, float *write_gate, float *log_alpha,
+                             rda_dtype_t dtype, int H, int Dk, int Dv, rda_act_t conv_act, void *stream) {
+    if (dtype != RDA_F32 && dtype != RDA_BF16) return RDA_ERR_UNSUPPORTED;
+    if (!dims_ok(Dk, Dv)) return RDA_ERR_UNSUPPORTED;
+    if (conv_act != RDA_ACT_NONE && conv_act != RDA_ACT_SILU) return RDA_ERR_UNSUPPORTED;
+    if (num_seqs < 0 || total_T < 0 || H <= 0 || max_seqlen < 0) return RDA_ERR_INVALID_ARG;
+    if (!cu_seqlens && (seq_len < 0 || (long long)num_seqs * seq_len != total_T)) return RDA_ERR_INVALID_ARG;
+    if (!sizes_ok(total_T, H, Dk, Dv)) return RDA_ERR_INVALID_ARG;
+    if ((long long)num_seqs * 3 * H * (2 * Dk + Dv) >= (1LL << 31)) return RDA_ERR_INVALID_ARG;
+    if ((delta == nullptr) != (write_gate == nullptr)) return RDA_ERR_INVALID_ARG;
+    if (num_seqs == 0) return RDA_OK;
+    if (!conv_w_q || !conv_w_k || !conv_w_v || !beta_raw || !log_alpha_raw || !beta || !log_alpha)
+        return RDA_ERR_INVALID_ARG;
+    if (total_T > 0) {
+        rda_status_t st = check_io_ptrs(q_raw, k_raw, v_raw, beta_raw, log_alpha_raw, q);
+        if (st != RDA_OK) return st;
+        if (!k || !v) return RDA_ERR_INVALID_ARG;
+        if (!aligned(k, 16) || !aligned(v, 16)) return RDA_ERR_MISALIGNED;
+    }
+    if ((conv_window_in && !aligned(conv_window_in, 2)) || (conv_window_out && !aligned(conv_window_out, 2)))
+        return RDA_ERR_MISALIGNED;
+    PrepLaunch l{};
+    l.raw[0] = q_raw; l.raw[1] = k_raw; l.raw[2] = v_raw;
+    l.w[0] = conv_w_q; l.w[1] = conv_w_k; l.w[2] = conv_w_v;
+    l.win_in = conv_window_in; l.win_out = conv_window_out;
+    l.beta_raw = beta_raw; l.delta = delta; l.la_raw = log_alpha_raw;
+    l.cu_seqlens = cu_seqlens;
+    l.num_seqs = num_seqs; l.seq_len = seq_len; l.max_seqlen = cu_seqlens ? max_seqlen : seq_len;
+    l.H = H; l.Dk = Dk; l.Dv = Dv;
+    l.channel = channel_decay != 0; l.act = conv_act; l.dtype = dtype;
+    l.out[0] = q; l.out[1] = k; l.out[2] = v;
+    l.beta = beta; l.gamma = write_gate; l.log_alpha = log_alpha;
+    return launch_prep_inputs(l, static_cast<cudaStream_t>(stream)) == cudaSuccess ? RDA_OK : RDA_ERR_CUDA;
+}
+
+rda_status_t rda_output_gate_norm(const void *o, const void *g, const float *norm_weight, float eps,
+                                  rda_act_t gate_act, void *out, rda_dtype_t dtype,
+                                  long long tokens, int H, int Dv, void *stream) {
+    if (dtype != RDA_F32 && dtype != RDA_BF16) return RDA_ERR_UNSUPPORTED;
+    if (Dv != 64 && Dv != 128) return RDA_ERR_UNSUPPORTED;
+    if (gate_act != RDA_ACT_SIGMOID && gate_act != RDA_ACT_SILU && gate_act != RDA_ACT_NONE)
+        return RDA_ERR_UNSUPPORTED;
+    if (tokens < 0 || H <= 0 || !(eps >= 0.f)) return RDA_ERR_INVALID_ARG;
+    if (tokens * H * Dv >= (1LL << 31)) return RDA_ERR_INVALID_ARG;
+    if (tokens == 0) return RDA_OK;
+    if (!o || !g || !norm_weight || !out) return RDA_ERR_INVALID_ARG;
+    if (!aligned(o, 16) || !aligned(g, 16) || !aligned(out, 16) || !aligned(norm_weight, 4))
+        return RDA_ERR_MISALIGNED;
+    return launch_output_gate_norm(o, g, norm_weight, out, (long)tokens * H, Dv, eps, gate_act, dtype,
+                                   static_cast<cudaStream_t>(stream)) == cudaSuccess ? RDA_OK : RDA_ERR_CUDA;
+}
+
 void rda_debug_set_wait_fault(int drop_chunk, unsigned long long wait_limit_ns) {
     rda::g_drop_chunk.store(drop_chunk < 0 ? -1 : drop_chunk);
     rda::g_wait_ns.store(wait_limit_ns ? (uint64_t)wait_limit_ns : rda::kDefaultWaitNs);

@@ -59,6 +59,25 @@ struct WaitSettings {
 };
 WaitSettings wait_settings();
 
+// The steps around the core (rda_prep_inputs, rda_output_gate_norm).
+struct PrepLaunch {
+    const void *raw[3];          // q, k, v projections
+    const float *w[3];           // conv taps [H*D, 3]
+    const void *win_in;          // bf16 [N, 3, C] or null (zeros)
+    void *win_out;               // bf16 [N, 3, C] or null
+    const float *beta_raw, *delta, *la_raw;
+    const int32_t *cu_seqlens;   // null: num_seqs sequences of seq_len tokens
+    int num_seqs, seq_len, max_seqlen, H, Dk, Dv;
+    bool channel;
+    int act;
+    rda_dtype_t dtype;
+    void *out[3];
+    float *beta, *gamma, *log_alpha;
+};
+cudaError_t launch_prep_inputs(const PrepLaunch &l, cudaStream_t s);
+cudaError_t launch_output_gate_norm(const void *o, const void *g, const float *w, void *out, long rows, int Dv,
+                                    float eps, int act, rda_dtype_t dtype, cudaStream_t s);
+
 // Most tokens one multi-token decode call takes per sequence.
 constexpr int kMaxDecodeTokens = 8;
 

@@ -44,7 +44,11 @@
  *   until the stream has reached the call.  The first call of an entry point
  *   in a process sets kernel attributes (host-side, once); make it outside
  *   stream capture.  Later calls only enqueue kernels, so a CUDA graph
- *   captured from `stream` replays them.
+ *   captured from `stream` replays them; the exception is rda_prefill_varlen
+ *   (and its per-channel form) with a non-NULL cu_seqlens_host, which copies a
+ *   schedule from temporary host memory and must not be captured (pass NULL
+ *   under capture).  This paragraph's capture statement does not cover
+ *   rda_prefill_chunked_noalloc, which is described with that call.
  *
  * ALIASING
  *   final_state may equal initial_state (updated in place).  No other output
@@ -85,6 +89,12 @@ typedef enum {
     RDA_F32 = 0,               /* q, k, v, out are float                             */
     RDA_BF16 = 1               /* q, k, v, out are bfloat16 (raw 16-bit words)       */
 } rda_dtype_t;
+
+typedef enum {
+    RDA_ACT_NONE = 0,          /* identity                                           */
+    RDA_ACT_SILU = 1,          /* x * sigmoid(x)                                     */
+    RDA_ACT_SIGMOID = 2        /* 1 / (1 + exp(-x))                                  */
+} rda_act_t;
 
 /* Static, human-readable name of a status code.  Never NULL. */
 const char *rda_status_string(rda_status_t status);
@@ -248,6 +258,74 @@ rda_status_t rda_decode_step_channel(const void *q, const void *k, const void *v
                                      const float *write_gate,
                                      float *state, void *out, rda_dtype_t dtype,
                                      int B, int H, int Dk, int Dv, float scale, void *stream);
+
+/*
+ * THE STEPS AROUND THE CORE
+ *
+ * The model printout in the "tiny-random/raon-1-mini" README (section
+ * "Printing the model") shows what the RDA layer does before and after the
+ * recurrence: q, k and v pass through short convolutions (q_conv1d, k_conv1d,
+ * v_conv1d) after their projections; b_proj and rda_w_proj give the write
+ * strength and the write gate; g_proj gives an output gate and o_norm, an
+ * RMSNorm over the head dimension (eps 1e-5), normalises the core's output.
+ * The nano article sizes the per-layer convolution window at three tokens
+ * (section "The cache is small if the runtime keeps it small") and gives the
+ * write gate sigma(beta_raw + delta) / sigma(beta_raw) and the decay's lower
+ * bound of -5 in log space (section "The other 1.5B"); the blog post on Raon-1
+ * mini keeps the convolution history in BF16.  Where the pages are silent the
+ * reading taken is stated with the argument.
+ *
+ * rda_prep_inputs: from the projections' outputs to the core's inputs, one
+ * pass, per sequence n and token t:
+ *   y_t = act(w[c][0] x_{t-2} + w[c][1] x_{t-1} + w[c][2] x_t)  per channel c of
+ *         q, k and v (a causal depthwise 3-tap convolution; x_{-1}, x_{-2} come
+ *         from the carried window)
+ *   q_t, k_t = y_t / ||y_t||_2 per head;  v_t = y_t
+ *   beta = sigmoid(beta_raw);  write_gate = sigmoid(beta_raw + delta) / beta
+ *   log_alpha = min(max(log_alpha_raw, -5), 0)
+ *
+ *   q_raw, k_raw   device, dtype, [total_T,H,Dk];  v_raw device, dtype, [total_T,H,Dv]
+ *   conv_w_q, conv_w_k  device fp32 [H*Dk, 3];  conv_w_v device fp32 [H*Dv, 3]
+ *                  (taps for t-2, t-1, t; channel c = head * D + d)
+ *   conv_window_in   device bf16 [num_seqs, 3, H*Dk + H*Dk + H*Dv] or NULL
+ *                  (zeros): the last three raw inputs of each sequence before
+ *                  this call, oldest first, channels of q, k, v concatenated
+ *   conv_window_out  device bf16, same layout, or NULL: the last three raw
+ *                  inputs after this call (may equal conv_window_in)
+ *   beta_raw       device fp32 [total_T,H];  delta device fp32 [total_T,H] or NULL
+ *   log_alpha_raw  device fp32 [total_T,H], or [total_T,H,Dk] with channel_decay != 0
+ *   cu_seqlens     device int32 [num_seqs+1] (packed sequences; max_seqlen must
+ *                  be at least the longest one), or NULL: num_seqs sequences of
+ *                  seq_len tokens (total_T = num_seqs * seq_len)
+ *   q, k, v        device, dtype, outputs in the core's layouts
+ *   beta, log_alpha  device fp32 outputs like beta_raw, log_alpha_raw
+ *   write_gate     device fp32 [total_T,H] output; NULL exactly when delta is NULL
+ *   conv_act       RDA_ACT_NONE or RDA_ACT_SILU (the pages do not name the
+ *                  convolution's activation; Kimi Delta Attention, which the
+ *                  pages say RDA modifies, uses SiLU)
+ * q_raw, k_raw, v_raw, q, k, v must be 16-byte aligned.
+ */
+rda_status_t rda_prep_inputs(const void *q_raw, const void *k_raw, const void *v_raw,
+                             const float *conv_w_q, const float *conv_w_k, const float *conv_w_v,
+                             const void *conv_window_in, void *conv_window_out,
+                             const float *beta_raw, const float *delta,
+                             const float *log_alpha_raw, int channel_decay,
+                             const int32_t *cu_seqlens, int num_seqs, int seq_len, int max_seqlen, int total_T,
+                             void *q, void *k, void *v, float *beta, float *write_gate, float *log_alpha,
+                             rda_dtype_t dtype, int H, int Dk, int Dv, rda_act_t conv_act, void *stream);
+
+/*
+ * rda_output_gate_norm: after the core, per token and head,
+ *   out = o / sqrt(mean_d(o^2) + eps) * norm_weight * act(g)
+ *
+ *   o, g, out      device, dtype, [tokens,H,Dv], 16-byte aligned (out may equal o)
+ *   norm_weight    device fp32 [Dv] (o_norm's weight, shared by the heads)
+ *   gate_act       RDA_ACT_SIGMOID, RDA_ACT_SILU or RDA_ACT_NONE (the pages do
+ *                  not name the output gate's activation)
+ */
+rda_status_t rda_output_gate_norm(const void *o, const void *g, const float *norm_weight, float eps,
+                                  rda_act_t gate_act, void *out, rda_dtype_t dtype,
+                                  long long tokens, int H, int Dv, void *stream);
 
 /*
  * Fixed-length prefill that allocates nothing and takes no workspace.

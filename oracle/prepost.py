@@ -109,7 +109,7 @@ def prep_inputs(q_raw, k_raw, v_raw, w_q, w_k, w_v, beta_raw, log_alpha_raw, cu_
         parts = []
         for raw, w, lo, hi, D in ((q_raw, w_q, 0, cq, Dk), (k_raw, w_k, cq, cq + ck, Dk),
                                   (v_raw, w_v, cq + ck, cq + ck + cv, Dv)):
-            y, nw = short_conv(raw[a:b].reshape(b - a, -1), w, None if wn is None else wn[:, lo:hi], act)
+            y, nw = short_conv(raw[a:b].reshape(b - a, hi - lo), w, None if wn is None else wn[:, lo:hi], act)
             parts.append(y.reshape(b - a, H, D))
             new_win[n, :, lo:hi] = nw
         q[a:b] = l2_normalize(parts[0])

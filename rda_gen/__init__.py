@@ -191,6 +191,69 @@ def decode_inputs(B=256, H=16, Dk=128, Dv=128, steps=128, dtype=torch.bfloat16, 
                         dict(B=B, H=H, Dk=Dk, Dv=Dv, steps=steps, dtype=dtype, seed=seed))
 
 
+@dataclass
+class RawLayerInputs:
+    """The projections' outputs an RDA layer hands to the steps before the core,
+    and the parameters of those steps: q_raw, k_raw [.., H, Dk]; v_raw [.., H, Dv]
+    (fixed length ``[B,T,..]`` or packed ``[total,..]`` with cu_seqlens); conv
+    taps [H*D, 3]; beta_raw, delta [.., H]; log_alpha_raw [.., H] or [.., H, Dk];
+    conv_window [N, 3, H*(2Dk+Dv)] (bf16); and, for the step after the core, an
+    output gate g [.., H, Dv] and the norm weight [Dv]."""
+    q_raw: torch.Tensor
+    k_raw: torch.Tensor
+    v_raw: torch.Tensor
+    w_q: torch.Tensor
+    w_k: torch.Tensor
+    w_v: torch.Tensor
+    beta_raw: torch.Tensor
+    delta: torch.Tensor
+    log_alpha_raw: torch.Tensor
+    conv_window: torch.Tensor
+    g: torch.Tensor
+    norm_weight: torch.Tensor
+    cu_seqlens: Optional[torch.Tensor] = None
+    meta: dict = field(default_factory=dict)
+
+    def to(self, device):
+        f = lambda t: None if t is None else t.to(device)
+        return RawLayerInputs(*(f(getattr(self, k)) for k in (
+            "q_raw", "k_raw", "v_raw", "w_q", "w_k", "w_v", "beta_raw", "delta", "log_alpha_raw",
+            "conv_window", "g", "norm_weight", "cu_seqlens")), dict(self.meta))
+
+
+def raw_layer_inputs(B=None, T=None, H=2, Dk=128, Dv=128, dtype=torch.bfloat16, seed=0,
+                     lengths=None, channel=False) -> RawLayerInputs:
+    """Fixed length (B, T) or packed (``lengths``).  q/k/v projections, beta_raw
+    and g ~ N(0, 1); delta ~ N(0, 0.25); conv taps ~ N(0, 1/3); the log decay
+    before its clamp ~ U(-6, 0.2) (both ends of the clamp are reached); the
+    carried window ~ N(0, 1); the norm weight ~ 1 + N(0, 0.01)."""
+    rng = np.random.Generator(np.random.PCG64(seed))
+    if lengths is not None:
+        lengths = np.asarray(lengths, np.int64)
+        cu = np.concatenate([[0], np.cumsum(lengths)])
+        lead, N = (int(cu[-1]),), len(lengths)
+    else:
+        cu, lead, N = None, (B, T), B
+    q = _normal(rng, lead + (H, Dk))
+    k = _normal(rng, lead + (H, Dk))
+    v = _normal(rng, lead + (H, Dv))
+    w_q = _normal(rng, (H * Dk, 3)) / np.sqrt(3.0)
+    w_k = _normal(rng, (H * Dk, 3)) / np.sqrt(3.0)
+    w_v = _normal(rng, (H * Dv, 3)) / np.sqrt(3.0)
+    br = _normal(rng, lead + (H,))
+    de = _normal(rng, lead + (H,)) * 0.5
+    la = rng.uniform(-6.0, 0.2, size=lead + ((H, Dk) if channel else (H,)))
+    win = _normal(rng, (N, 3, H * (2 * Dk + Dv)))
+    g = _normal(rng, lead + (H, Dv))
+    nw = 1.0 + _normal(rng, (Dv,)) * 0.1
+    f32 = lambda x: _to(x, torch.float32)
+    return RawLayerInputs(_to(q, dtype), _to(k, dtype), _to(v, dtype), f32(w_q), f32(w_k), f32(w_v),
+                          f32(br), f32(de), f32(la), _to(win, torch.bfloat16), _to(g, dtype), f32(nw),
+                          None if cu is None else torch.from_numpy(cu.astype(np.int32)),
+                          dict(B=B, T=T, H=H, Dk=Dk, Dv=Dv, dtype=dtype, seed=seed, channel=channel,
+                               lengths=None if lengths is None else lengths.tolist()))
+
+
 # The measured workloads.  Seeds are the workload numbers (the mini shape, H = 40, is 6).
 WORKLOADS = {
     "fp32_parity_b1_t256_h2_d64": dict(kind="fixed", B=1, T=256, H=2, Dk=64, Dv=64,

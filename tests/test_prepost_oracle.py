@@ -106,6 +106,16 @@ def test_prep_norms_and_directions():
     assert np.array_equal(r["conv_window"][2, :, :H * Dk], case["q_raw"][-3:].reshape(3, -1))
 
 
+def test_prep_empty_sequence_passes_window_through():
+    case = _prep_case(lengths=(4, 0, 2))
+    r = pp.prep_inputs(**case)
+    assert np.array_equal(r["conv_window"][1], case["conv_window"][1])
+    # a 2-token sequence keeps the newest old row and its two inputs
+    H, Dk = 2, 4
+    assert np.array_equal(r["conv_window"][2, 0, :H * Dk], case["conv_window"][2, 2, :H * Dk])
+    assert np.array_equal(r["conv_window"][2, 1:, :H * Dk], case["q_raw"][4:6].reshape(2, -1))
+
+
 def test_prep_sequences_do_not_leak():
     """A sequence's outputs depend only on its own tokens and its own window."""
     case = _prep_case()
