@@ -624,6 +624,47 @@ def profile_decode_tokens(T, steps, warmup):
     print(json.dumps({"decode_tokens_T": T, "ms_per_call": s.elapsed_time(e) / steps}), flush=True)
 
 
+def profile_prefill(steps, warmup):
+    """Only the nano prefill: `warmup` + `steps` eager calls, L2 flushed before
+    each (a short, self-contained run for a profiler)."""
+    import torch
+    import gated_delta_rule_rda_b200 as rda
+    import rda_gen
+    inp = rda_gen.workload(WORKLOAD).to("cuda")
+    B, T, H, Dk = inp.q.shape
+    Dv = inp.v.shape[-1]
+    ws = rda.new_workspace(rda.rda_prefill_workspace_bytes(B, T, H, Dk, Dv, 0), "cuda")
+    out = torch.empty_like(inp.v)
+    sf = torch.empty(B, H, Dk, Dv, device="cuda")
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device="cuda")
+    for _ in range(warmup + steps):
+        flush.zero_()
+        rda.rda_prefill_chunked(inp.q, inp.k, inp.v, inp.log_alpha, inp.beta, initial_state=inp.initial_state,
+                                out=out, final_state=sf, workspace=ws)
+    torch.cuda.synchronize()
+    assert rda.rda_read_device_error(ws) == 0
+    print(json.dumps({"profile_prefill_calls": warmup + steps}), flush=True)
+
+
+def profile_prepost(steps, warmup):
+    """Only the steps around the core at the nano shape (bf16 B1 T4096 H16 D128):
+    `warmup` + `steps` calls of each, L2 flushed before each pair."""
+    import torch
+    import gated_delta_rule_rda_b200 as rda
+    import rda_gen
+    raw = rda_gen.raw_layer_inputs(B=1, T=4096, H=16, Dk=128, Dv=128, dtype=torch.bfloat16, seed=9).to("cuda")
+    win_out = torch.empty_like(raw.conv_window)
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device="cuda")
+    for _ in range(warmup + steps):
+        flush.zero_()
+        rda.rda_prep_inputs(raw.q_raw, raw.k_raw, raw.v_raw, raw.w_q, raw.w_k, raw.w_v, raw.beta_raw,
+                            raw.log_alpha_raw, delta=raw.delta, conv_window_in=raw.conv_window,
+                            conv_window_out=win_out)
+        rda.rda_output_gate_norm(raw.v_raw, raw.g, raw.norm_weight)
+    torch.cuda.synchronize()
+    print(json.dumps({"profile_prepost_calls": warmup + steps}), flush=True)
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -636,11 +677,21 @@ def main():
                     help="also time the long-context and packed (varlen) prefill workloads")
     ap.add_argument("--profile-decode-tokens", type=int, default=0, metavar="T",
                     help="run only the multi-token decode with T tokens per call (for a profiler)")
+    ap.add_argument("--profile-prefill", action="store_true",
+                    help="run only warmup + steps nano prefill calls, L2 flushed (for a profiler)")
+    ap.add_argument("--profile-prepost", action="store_true",
+                    help="run only warmup + steps calls of the steps around the core (for a profiler)")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
     if args.profile_decode_tokens:
         profile_decode_tokens(args.profile_decode_tokens, args.steps, args.warmup)
+        return
+    if args.profile_prefill:
+        profile_prefill(args.steps, args.warmup)
+        return
+    if args.profile_prepost:
+        profile_prepost(args.steps, args.warmup)
         return
 
     world = int(os.environ.get("WORLD_SIZE", "1"))

@@ -226,6 +226,54 @@ __device__ __forceinline__ void mma_f32_split(float *acc, const float *a, uint32
     if (!EXACT_B) mma_tf32_m16n8k8(acc, ah[0], ah[1], ah[2], ah[3], bl0, bl1);
 }
 
+// Persistent form: each CTA loops over (sequence, head) units.  A unit's state
+// (64 KiB) is copied into shared memory with 16-byte asynchronous copies
+// (cp.async, completed by a hardware wait, no spin) and from there into the
+// registers; the copy of the CTA's next unit is issued as soon as the buffer is
+// free, so every SM always has state bytes in flight while it computes.
+constexpr int kTcRow = kTcD + 4;    // padded smem row (528 B): conflict-free 8-byte fragment reads
+constexpr uint32_t kTcStateBytes = kTcD * kTcRow * 4;
+constexpr uint32_t kTcRawBytes = 3 * kMaxT * kTcD * 4;                    // k, q, v rows (fp32 at most)
+constexpr uint32_t kTcSmem = kTcStateBytes + kTcRawBytes + 3 * kMaxT * 4; // + the gates
+
+__device__ __forceinline__ void cp_async16(uint32_t dst, const void *src) {
+    asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(dst), "l"(src) : "memory");
+}
+__device__ __forceinline__ void cp_async4(uint32_t dst, const void *src) {
+    asm volatile("cp.async.ca.shared.global [%0], [%1], 4;" ::"r"(dst), "l"(src) : "memory");
+}
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+__device__ __forceinline__ void cp_async_wait_all() { asm volatile("cp.async.wait_group 0;" ::: "memory"); }
+
+// Everything unit bh needs, copied into shared memory: its state (4,096
+// 16-byte pieces into the padded buffer), the raw rows of its T keys, queries
+// and values, and its gates (log alpha, beta, gamma).
+template <typename Tio>
+__device__ __forceinline__ void issue_unit_copy(const DecodeArgs &a, int bh, uint32_t smem) {
+    const float *st = a.state + (size_t)bh * kTcD * kTcD;
+#pragma unroll
+    for (int i = 0; i < 16; ++i) {
+        const int id = i * kThreads + threadIdx.x;
+        const int row = id >> 5, c16 = id & 31;
+        cp_async16(smem + (row * kTcRow + c16 * 4) * 4, st + row * kTcD + c16 * 4);
+    }
+    const int T = a.T, H = a.H, b = bh / H, h = bh % H;
+    constexpr int PR = kTcD * (int)sizeof(Tio) / 16;      // 16-byte pieces per row
+    const uint32_t raw = smem + kTcStateBytes;
+    for (int id = threadIdx.x; id < 3 * T * PR; id += kThreads) {
+        const int which = id / (T * PR), t = (id / PR) % T, c = id % PR;
+        const Tio *src = static_cast<const Tio *>(which == 0 ? a.k : (which == 1 ? a.q : a.v)) +
+                         (((size_t)b * T + t) * H + h) * kTcD;
+        cp_async16(raw + ((which * kMaxT + t) * kTcD) * (uint32_t)sizeof(Tio) + c * 16, reinterpret_cast<const char *>(src) + c * 16);
+    }
+    if (threadIdx.x < 3 * T) {
+        const int which = threadIdx.x / T, t = threadIdx.x % T;
+        const float *src = which == 0 ? a.log_alpha : (which == 1 ? a.beta : a.gamma);
+        if (src) cp_async4(raw + kTcRawBytes + (which * kMaxT + t) * 4, src + ((size_t)b * T + t) * H + h);
+    }
+    cp_async_commit();
+}
+
 template <typename Tio>
 __global__ void __launch_bounds__(kThreads, 2)
 decode_tokens_tc_kernel(DecodeArgs a) {
@@ -242,143 +290,159 @@ decode_tokens_tc_kernel(DecodeArgs a) {
     __shared__ float g_s[3][kMaxT];                        // alpha, beta, gamma
     __shared__ float c_s;
 
+    extern __shared__ __align__(16) float sbuf[];         // [kTcD][kTcRow] state of the current unit
+
     const int T = a.T, H = a.H;
-    const int bh = blockIdx.x, b = bh / H, h = bh % H;
+    const int units = a.B * H;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int g = lane >> 2, tg = lane & 3;
     const int jc = 16 * warp + 2 * g;                      // this thread's column pair
-    float *st = a.state + (size_t)bh * D * D;
-    auto tok = [&](int t) { return ((size_t)b * T + t) * H + h; };
-
-    // the state reads first (each instruction: 4 rows x 64 contiguous bytes)
-    float s[16][4];
-#pragma unroll
-    for (int nb = 0; nb < 16; ++nb) {
-        const float *p = st + (size_t)(8 * nb + 2 * tg) * D + jc;
-        const float2 r0 = __ldcs(reinterpret_cast<const float2 *>(p));
-        const float2 r1 = __ldcs(reinterpret_cast<const float2 *>(p + D));
-        s[nb][0] = r0.x;
-        s[nb][2] = r0.y;
-        s[nb][1] = r1.x;
-        s[nb][3] = r1.y;
-    }
-    if (threadIdx.x < kMaxT) {
-        const int t = threadIdx.x;
-        const bool live = t < T;
-        g_s[0][t] = live ? expf(a.log_alpha[tok(t)]) : 1.f;
-        g_s[1][t] = live ? a.beta[tok(t)] : 0.f;
-        g_s[2][t] = live && a.gamma ? a.gamma[tok(t)] : 1.f;
-    }
-    for (int i = threadIdx.x; i < kMaxT * D; i += kThreads) {
-        const int t = i / D, d = i % D;
-        const bool live = t < T;
-        k_s[t][d] = live ? Io<Tio>::ld(static_cast<const Tio *>(a.k) + tok(t) * D + d) : 0.f;
-        q_s[t][d] = live ? Io<Tio>::ld(static_cast<const Tio *>(a.q) + tok(t) * D + d) : 0.f;
-        if (live) v_s[t][d] = Io<Tio>::ld(static_cast<const Tio *>(a.v) + tok(t) * D + d);
-    }
-    __syncthreads();
-
-    {
-        // a_t and b_t for this warp's 16 columns: S^T [k q] over the 128 key dims
-        // (B column n = token g; rows of block nb in the order of the A columns)
-        float pk[4] = {0.f, 0.f, 0.f, 0.f}, pq[4] = {0.f, 0.f, 0.f, 0.f};
+    const uint32_t buf = static_cast<uint32_t>(__cvta_generic_to_shared(sbuf));
+    const Tio *raw_s = reinterpret_cast<const Tio *>(reinterpret_cast<const char *>(sbuf) + kTcStateBytes);
+    const float *graw_s = reinterpret_cast<const float *>(reinterpret_cast<const char *>(sbuf) + kTcStateBytes +
+                                                          kTcRawBytes);
+    if ((int)blockIdx.x < units) issue_unit_copy<Tio>(a, blockIdx.x, buf);
+    for (int bh = blockIdx.x; bh < units; bh += gridDim.x) {
+        const int b = bh / H, h = bh % H;
+        float *st = a.state + (size_t)bh * D * D;
+        auto tok = [&](int t) { return ((size_t)b * T + t) * H + h; };
+        // this unit's copies have landed: state -> registers, rows and gates ->
+        // the fp32 work arrays; then the next unit's copy
+        cp_async_wait_all();
+        __syncthreads();
+        float s[16][4];
 #pragma unroll
         for (int nb = 0; nb < 16; ++nb) {
-            const float af[4] = {s[nb][0], s[nb][2], s[nb][1], s[nb][3]};
-            const float2 kb = *reinterpret_cast<const float2 *>(&k_s[g][8 * nb + 2 * tg]);
-            const float2 qb = *reinterpret_cast<const float2 *>(&q_s[g][8 * nb + 2 * tg]);
-            uint32_t kh0, kl0, kh1, kl1, qh0, ql0, qh1, ql1;
-            split_tf32(kb.x, kh0, kl0);
-            split_tf32(kb.y, kh1, kl1);
-            split_tf32(qb.x, qh0, ql0);
-            split_tf32(qb.y, qh1, ql1);
-            mma_f32_split<kExact>(pk, af, kh0, kh1, kl0, kl1);
-            mma_f32_split<kExact>(pq, af, qh0, qh1, ql0, ql1);
+            const float *p = sbuf + (8 * nb + 2 * tg) * kTcRow + jc;
+            const float2 r0 = *reinterpret_cast<const float2 *>(p);
+            const float2 r1 = *reinterpret_cast<const float2 *>(p + kTcRow);
+            s[nb][0] = r0.x;
+            s[nb][2] = r0.y;
+            s[nb][1] = r1.x;
+            s[nb][3] = r1.y;
         }
-        // accumulator: column jc (+1), token 2tg (+1)
-        if (2 * tg < T) {
-            ab_s[0][2 * tg][jc] = pk[0];
-            ab_s[0][2 * tg][jc + 1] = pk[2];
-            ab_s[1][2 * tg][jc] = pq[0];
-            ab_s[1][2 * tg][jc + 1] = pq[2];
+        if (threadIdx.x < kMaxT) {
+            const int t = threadIdx.x;
+            const bool live = t < T;
+            g_s[0][t] = live ? expf(graw_s[t]) : 1.f;
+            g_s[1][t] = live ? graw_s[kMaxT + t] : 0.f;
+            g_s[2][t] = live && a.gamma ? graw_s[2 * kMaxT + t] : 1.f;
         }
-        if (2 * tg + 1 < T) {
-            ab_s[0][2 * tg + 1][jc] = pk[1];
-            ab_s[0][2 * tg + 1][jc + 1] = pk[3];
-            ab_s[1][2 * tg + 1][jc] = pq[1];
-            ab_s[1][2 * tg + 1][jc + 1] = pq[3];
+        for (int i = threadIdx.x; i < kMaxT * D; i += kThreads) {
+            const int t = i / D, d = i % D;
+            const bool live = t < T;
+            k_s[t][d] = live ? Io<Tio>::ld(raw_s + (0 * kMaxT + t) * D + d) : 0.f;
+            q_s[t][d] = live ? Io<Tio>::ld(raw_s + (1 * kMaxT + t) * D + d) : 0.f;
+            if (live) v_s[t][d] = Io<Tio>::ld(raw_s + (2 * kMaxT + t) * D + d);
         }
-        // token Gram values over this warp's 16 key dims: K [K Q]^T (A rows = tokens
-        // g; rows g + 8 zero)
-        float gk[4] = {0.f, 0.f, 0.f, 0.f}, gq[4] = {0.f, 0.f, 0.f, 0.f};
-#pragma unroll
-        for (int ks = 2 * warp; ks < 2 * warp + 2; ++ks) {
-            const float af[4] = {k_s[g][8 * ks + tg], 0.f, k_s[g][8 * ks + tg + 4], 0.f};
-            uint32_t kh0, kl0, kh1, kl1, qh0, ql0, qh1, ql1;
-            split_tf32(k_s[g][8 * ks + tg], kh0, kl0);
-            split_tf32(k_s[g][8 * ks + tg + 4], kh1, kl1);
-            split_tf32(q_s[g][8 * ks + tg], qh0, ql0);
-            split_tf32(q_s[g][8 * ks + tg + 4], qh1, ql1);
-            mma_f32_split<kExact>(gk, af, kh0, kh1, kl0, kl1);
-            mma_f32_split<kExact>(gq, af, qh0, qh1, ql0, ql1);
-        }
-        gp_s[warp][0][g][2 * tg] = gk[0];
-        gp_s[warp][0][g][2 * tg + 1] = gk[1];
-        gp_s[warp][1][g][2 * tg] = gq[0];
-        gp_s[warp][1][g][2 * tg + 1] = gq[1];
-    }
-    __syncthreads();
-    if (threadIdx.x < 2 * kMaxT * kMaxT) {
-        const int which = threadIdx.x >> 6, i = (threadIdx.x >> 3) & 7, t = threadIdx.x & 7;
-        float x = 0.f;
-#pragma unroll
-        for (int w = 0; w < kThreads / 32; ++w) x += gp_s[w][which][i][t];
-        (which ? kq_s : kk_s)[i][t] = x;
-    }
-    __syncthreads();
+        __syncthreads();
+        if (bh + (int)gridDim.x < units) issue_unit_copy<Tio>(a, bh + gridDim.x, buf);
+        __syncthreads();
 
-    // the token recurrence, one value column per thread
-    if (threadIdx.x < D) {
-        const int j = threadIdx.x;
-        float c = 1.f;
-        float w[kMaxT];
+        {
+            // a_t and b_t for this warp's 16 columns: S^T [k q] over the 128 key dims
+            // (B column n = token g; rows of block nb in the order of the A columns)
+            float pk[4] = {0.f, 0.f, 0.f, 0.f}, pq[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
-        for (int t = 0; t < kMaxT; ++t) {
-            if (t >= T) break;
-            float p = c * ab_s[0][t][j];
+            for (int nb = 0; nb < 16; ++nb) {
+                const float af[4] = {s[nb][0], s[nb][2], s[nb][1], s[nb][3]};
+                const float2 kb = *reinterpret_cast<const float2 *>(&k_s[g][8 * nb + 2 * tg]);
+                const float2 qb = *reinterpret_cast<const float2 *>(&q_s[g][8 * nb + 2 * tg]);
+                uint32_t kh0, kl0, kh1, kl1, qh0, ql0, qh1, ql1;
+                split_tf32(kb.x, kh0, kl0);
+                split_tf32(kb.y, kh1, kl1);
+                split_tf32(qb.x, qh0, ql0);
+                split_tf32(qb.y, qh1, ql1);
+                mma_f32_split<kExact>(pk, af, kh0, kh1, kl0, kl1);
+                mma_f32_split<kExact>(pq, af, qh0, qh1, ql0, ql1);
+            }
+            // accumulator: column jc (+1), token 2tg (+1)
+            if (2 * tg < T) {
+                ab_s[0][2 * tg][jc] = pk[0];
+                ab_s[0][2 * tg][jc + 1] = pk[2];
+                ab_s[1][2 * tg][jc] = pq[0];
+                ab_s[1][2 * tg][jc + 1] = pq[2];
+            }
+            if (2 * tg + 1 < T) {
+                ab_s[0][2 * tg + 1][jc] = pk[1];
+                ab_s[0][2 * tg + 1][jc + 1] = pk[3];
+                ab_s[1][2 * tg + 1][jc] = pq[1];
+                ab_s[1][2 * tg + 1][jc + 1] = pq[3];
+            }
+            // token Gram values over this warp's 16 key dims: K [K Q]^T (A rows = tokens
+            // g; rows g + 8 zero)
+            float gk[4] = {0.f, 0.f, 0.f, 0.f}, gq[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
-            for (int i = 0; i < t; ++i) p = fmaf(w[i], kk_s[i][t], p);
-            const float al = g_s[0][t];
-#pragma unroll
-            for (int i = 0; i < t; ++i) w[i] *= al;
-            w[t] = g_s[1][t] * (g_s[2][t] * v_s[t][j] - al * p);
-            c *= al;
-            float o = c * ab_s[1][t][j];
-#pragma unroll
-            for (int i = 0; i <= t; ++i) o = fmaf(w[i], kq_s[i][t], o);
-            Io<Tio>::st(static_cast<Tio *>(a.out) + tok(t) * D + j, a.scale * o);
+            for (int ks = 2 * warp; ks < 2 * warp + 2; ++ks) {
+                const float af[4] = {k_s[g][8 * ks + tg], 0.f, k_s[g][8 * ks + tg + 4], 0.f};
+                uint32_t kh0, kl0, kh1, kl1, qh0, ql0, qh1, ql1;
+                split_tf32(k_s[g][8 * ks + tg], kh0, kl0);
+                split_tf32(k_s[g][8 * ks + tg + 4], kh1, kl1);
+                split_tf32(q_s[g][8 * ks + tg], qh0, ql0);
+                split_tf32(q_s[g][8 * ks + tg + 4], qh1, ql1);
+                mma_f32_split<kExact>(gk, af, kh0, kh1, kl0, kl1);
+                mma_f32_split<kExact>(gq, af, qh0, qh1, ql0, ql1);
+            }
+            gp_s[warp][0][g][2 * tg] = gk[0];
+            gp_s[warp][0][g][2 * tg + 1] = gk[1];
+            gp_s[warp][1][g][2 * tg] = gq[0];
+            gp_s[warp][1][g][2 * tg + 1] = gq[1];
         }
+        __syncthreads();
+        if (threadIdx.x < 2 * kMaxT * kMaxT) {
+            const int which = threadIdx.x >> 6, i = (threadIdx.x >> 3) & 7, t = threadIdx.x & 7;
+            float x = 0.f;
 #pragma unroll
-        for (int t = 0; t < kMaxT; ++t) w_s[t][j] = t < T ? w[t] : 0.f;
-        if (j == 0) c_s = c;
-    }
-    __syncthreads();
+            for (int w = 0; w < kThreads / 32; ++w) x += gp_s[w][which][i][t];
+            (which ? kq_s : kk_s)[i][t] = x;
+        }
+        __syncthreads();
 
-    // S_new^T = c S^T + W K: A = W (value columns x tokens), B = K (tokens x key
-    // dims), accumulated into the state registers
-    const float c = c_s;
-    const float wf[4] = {w_s[tg][jc], w_s[tg][jc + 1], w_s[tg + 4][jc], w_s[tg + 4][jc + 1]};
+        // the token recurrence, one value column per thread
+        if (threadIdx.x < D) {
+            const int j = threadIdx.x;
+            float c = 1.f;
+            float w[kMaxT];
 #pragma unroll
-    for (int nb = 0; nb < 16; ++nb) {
-        uint32_t bh0, bl0, bh1, bl1;
-        split_tf32(k_s[tg][8 * nb + g], bh0, bl0);
-        split_tf32(k_s[tg + 4][8 * nb + g], bh1, bl1);
+            for (int t = 0; t < kMaxT; ++t) {
+                if (t >= T) break;
+                float p = c * ab_s[0][t][j];
 #pragma unroll
-        for (int i = 0; i < 4; ++i) s[nb][i] *= c;
-        mma_f32_split<kExact>(s[nb], wf, bh0, bh1, bl0, bl1);
-        float *p = st + (size_t)(8 * nb + 2 * tg) * D + jc;
-        __stcs(reinterpret_cast<float2 *>(p), make_float2(s[nb][0], s[nb][2]));
-        __stcs(reinterpret_cast<float2 *>(p + D), make_float2(s[nb][1], s[nb][3]));
+                for (int i = 0; i < t; ++i) p = fmaf(w[i], kk_s[i][t], p);
+                const float al = g_s[0][t];
+#pragma unroll
+                for (int i = 0; i < t; ++i) w[i] *= al;
+                w[t] = g_s[1][t] * (g_s[2][t] * v_s[t][j] - al * p);
+                c *= al;
+                float o = c * ab_s[1][t][j];
+#pragma unroll
+                for (int i = 0; i <= t; ++i) o = fmaf(w[i], kq_s[i][t], o);
+                Io<Tio>::st(static_cast<Tio *>(a.out) + tok(t) * D + j, a.scale * o);
+            }
+#pragma unroll
+            for (int t = 0; t < kMaxT; ++t) w_s[t][j] = t < T ? w[t] : 0.f;
+            if (j == 0) c_s = c;
+        }
+        __syncthreads();
+
+        // S_new^T = c S^T + W K: A = W (value columns x tokens), B = K (tokens x key
+        // dims), accumulated into the state registers
+        const float c = c_s;
+        const float wf[4] = {w_s[tg][jc], w_s[tg][jc + 1], w_s[tg + 4][jc], w_s[tg + 4][jc + 1]};
+#pragma unroll
+        for (int nb = 0; nb < 16; ++nb) {
+            uint32_t bh0, bl0, bh1, bl1;
+            split_tf32(k_s[tg][8 * nb + g], bh0, bl0);
+            split_tf32(k_s[tg + 4][8 * nb + g], bh1, bl1);
+#pragma unroll
+            for (int i = 0; i < 4; ++i) s[nb][i] *= c;
+            mma_f32_split<kExact>(s[nb], wf, bh0, bh1, bl0, bl1);
+            float *p = st + (size_t)(8 * nb + 2 * tg) * D + jc;
+            __stcs(reinterpret_cast<float2 *>(p), make_float2(s[nb][0], s[nb][2]));
+            __stcs(reinterpret_cast<float2 *>(p + D), make_float2(s[nb][1], s[nb][3]));
+        }
+
+        __syncthreads();      // the shared arrays are reused by the next unit
     }
 }
 
@@ -400,7 +464,17 @@ cudaError_t launch_t(const DecodeArgs &a, cudaStream_t s) {
         // one or two tokens: the paired-FMA kernel streams the state in 16-byte
         // pieces and is faster; from three tokens the products dominate
         if (a.T <= 2) return launch_shape<Tio, 128, 128>(a, s);
-        decode_tokens_tc_kernel<Tio><<<(unsigned)(a.B * a.H), kThreads, 0, s>>>(a);
+        static cudaError_t attr = cudaFuncSetAttribute(decode_tokens_tc_kernel<Tio>,
+                                                       cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                                       (int)kTcSmem);
+        if (attr != cudaSuccess) return attr;
+        int dev = 0, sms = 0;
+        cudaError_t e = cudaGetDevice(&dev);
+        if (e == cudaSuccess) e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+        if (e != cudaSuccess) return e;
+        const long units = (long)a.B * a.H;
+        const unsigned grid = (unsigned)(units < 2L * sms ? units : 2L * sms);   // two CTAs per SM
+        decode_tokens_tc_kernel<Tio><<<grid, kThreads, kTcSmem, s>>>(a);
         return cudaGetLastError();
     }
     if (a.Dk == 128 && a.Dv == 64) return launch_shape<Tio, 128, 64>(a, s);
