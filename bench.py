@@ -475,6 +475,19 @@ def other_workloads(device, stream, rank, world, reps=5):
                              "hbm_frac": bytes_step / (ms * 1e-3) / 1e9 / load_peaks()[0]}
     del din, st, dout
 
+    # backward pass at the nano shape (token-sequential fp32, checkpoints every 16 tokens)
+    inp = rda_gen.workload(WORKLOAD).to(device)
+    B, T, H, Dk = inp.q.shape
+    gen = torch.Generator(device="cpu").manual_seed(11)
+    d_out = torch.randn(inp.v.shape, generator=gen).to(device=device, dtype=inp.v.dtype)
+    d_sf = torch.randn((B, H, Dk, Dk), generator=gen).to(device)
+    bws = rda.new_workspace(int(rda.lib.rda_backward_workspace_bytes(B, T, H, Dk, Dk)), device)
+    ms = timed(lambda: rda.rda_backward(inp.q, inp.k, inp.v, inp.log_alpha, inp.beta, d_out,
+                                        initial_state=inp.initial_state, d_final_state=d_sf, workspace=bws))
+    res["backward"] = {"workload": WORKLOAD + ", gradients of <d_out, out> + <d_final_state, final_state>",
+                       "ms": ms, "tokens_per_s": world * B * T / (ms * 1e-3)}
+    del inp, d_out, d_sf, bws
+
     # the steps around the core at the nano shape: short conv + norms + gates, and
     # the output norm x gate
     raw = rda_gen.raw_layer_inputs(B=1, T=4096, H=16, Dk=128, Dv=128, dtype=torch.bfloat16, seed=9).to(device)

@@ -64,6 +64,10 @@ lib.rda_prep_inputs.argtypes = [_vp] * 8 + [_vp, _vp, _vp, _i, _vp, _i, _i, _i, 
 lib.rda_prep_inputs.restype = _i
 lib.rda_output_gate_norm.argtypes = [_vp, _vp, _vp, _f, _i, _vp, _i, ctypes.c_longlong, _i, _i, _vp]
 lib.rda_output_gate_norm.restype = _i
+lib.rda_backward_workspace_bytes.argtypes = [_i] * 5
+lib.rda_backward_workspace_bytes.restype = _sz
+lib.rda_backward.argtypes = [_vp] * 16 + [_i] * 6 + [_f, _vp, _sz, _vp]
+lib.rda_backward.restype = _i
 lib.rda_debug_set_wait_fault.argtypes = [_i, ctypes.c_ulonglong]
 lib.rda_debug_set_wait_fault.restype = None
 
@@ -337,6 +341,34 @@ def rda_output_gate_norm(o, g, norm_weight, eps=1e-5, gate_act=RDA_ACT_SIGMOID, 
     return out
 
 
+def rda_backward(q, k, v, log_alpha, beta, d_out, write_gate=None, initial_state=None,
+                 d_final_state=None, scale=1.0, workspace=None, stream=None):
+    """Gradients of ``<d_out, out> + <d_final_state, final_state>`` for a
+    fixed-length prefill (shapes as :func:`rda_prefill_chunked`).  Returns a
+    dict of fp32 tensors dq, dk, dv, d_log_alpha, d_beta, d_write_gate (None
+    without a write gate) and d_initial_state."""
+    B, T, H, Dk = q.shape
+    Dv = v.shape[-1]
+    _need_cuda(q, k, v, log_alpha, beta, d_out, write_gate, initial_state, d_final_state, workspace)
+    _need_f32(log_alpha, beta, write_gate, initial_state, d_final_state)
+    dt = _dtype_code(q)
+    if d_out.dtype != q.dtype or d_out.shape != v.shape:
+        raise ValueError("rda: d_out must match out")
+    f = lambda *shape: torch.empty(shape, dtype=torch.float32, device=q.device)
+    g = dict(dq=f(B, T, H, Dk), dk=f(B, T, H, Dk), dv=f(B, T, H, Dv), d_log_alpha=f(B, T, H),
+             d_beta=f(B, T, H), d_write_gate=None if write_gate is None else f(B, T, H),
+             d_initial_state=f(B, H, Dk, Dv))
+    if workspace is None:
+        workspace = new_workspace(int(lib.rda_backward_workspace_bytes(B, T, H, Dk, Dv)), q.device)
+    code = lib.rda_backward(_ptr(q), _ptr(k), _ptr(v), _ptr(log_alpha), _ptr(beta), _ptr(write_gate),
+                            _ptr(initial_state), _ptr(d_out), _ptr(d_final_state), _ptr(g["dq"]),
+                            _ptr(g["dk"]), _ptr(g["dv"]), _ptr(g["d_log_alpha"]), _ptr(g["d_beta"]),
+                            _ptr(g["d_write_gate"]), _ptr(g["d_initial_state"]), dt, B, T, H, Dk, Dv,
+                            float(scale), _ptr(workspace), workspace.numel(), _stream(stream))
+    _check(code, "rda_backward")
+    return g
+
+
 def rda_debug_set_wait_fault(drop_chunk=-1, wait_limit_ns=0):
     """Testing only: bound of the device-side waits and an injected stall of the
     scan (see include/rda.h); ``rda_debug_set_wait_fault()`` turns it off."""
@@ -351,7 +383,7 @@ def rda_read_device_error(workspace, stream=None) -> int:
 
 
 __all__ = ["rda_prefill_chunked", "rda_prefill_varlen", "rda_decode_step", "rda_decode_tokens",
-           "rda_prep_inputs", "rda_output_gate_norm",
+           "rda_prep_inputs", "rda_output_gate_norm", "rda_backward",
            "rda_prefill_chunked_noalloc",
            "rda_read_device_error", "rda_debug_set_wait_fault", "rda_prefill_workspace_bytes", "new_workspace", "version",
            "RdaError", "lib", "LIB_PATH"]

@@ -387,6 +387,75 @@ rda_status_t rda_output_gate_norm(const void *o, const void *g, const float *nor
                                    static_cast<cudaStream_t>(stream)) == cudaSuccess ? RDA_OK : RDA_ERR_CUDA;
 }
 
+size_t rda_backward_workspace_bytes(int B, int T, int H, int Dk, int Dv) {
+    if (B < 0 || T < 0 || H <= 0 || !dims_ok(Dk, Dv)) return 0;
+    return kErrorWordBytes + align_up(backward_ckpt_bytes(B, T, H, Dk, Dv), 256);
+}
+
+rda_status_t rda_backward(const void *q, const void *k, const void *v,
+                          const float *log_alpha, const float *beta, const float *write_gate,
+                          const float *initial_state, const void *d_out, const float *d_final_state,
+                          float *dq, float *dk, float *dv, float *d_log_alpha, float *d_beta,
+                          float *d_write_gate, float *d_initial_state,
+                          rda_dtype_t dtype, int B, int T, int H, int Dk, int Dv, float scale,
+                          void *workspace, size_t workspace_bytes_given, void *stream) {
+    if (dtype != RDA_F32 && dtype != RDA_BF16) return RDA_ERR_UNSUPPORTED;
+    if (B < 0 || T < 0 || H <= 0) return RDA_ERR_INVALID_ARG;
+    if (!dims_ok(Dk, Dv)) return RDA_ERR_UNSUPPORTED;
+    if (!sizes_ok((long long)B * T, H, Dk, Dv)) return RDA_ERR_INVALID_ARG;
+    if ((long long)B * H * Dk * Dv >= (1LL << 31)) return RDA_ERR_INVALID_ARG;
+    if ((write_gate == nullptr) != (d_write_gate == nullptr)) return RDA_ERR_INVALID_ARG;
+    if ((initial_state && !aligned(initial_state, 16)) || (d_final_state && !aligned(d_final_state, 16)) ||
+        (d_initial_state && !aligned(d_initial_state, 16)))
+        return RDA_ERR_MISALIGNED;
+    const size_t need = rda_backward_workspace_bytes(B, T, H, Dk, Dv);
+    if (!workspace || workspace_bytes_given < need) return RDA_ERR_WORKSPACE;
+    if (!aligned(workspace, 256)) return RDA_ERR_MISALIGNED;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    if (B == 0) return RDA_OK;
+    if (T == 0) {
+        if (d_initial_state) {
+            const size_t bytes = sizeof(float) * (size_t)B * H * Dk * Dv;
+            cudaError_t e = d_final_state ? cudaMemcpyAsync(d_initial_state, d_final_state, bytes,
+                                                            cudaMemcpyDeviceToDevice, s)
+                                          : cudaMemsetAsync(d_initial_state, 0, bytes, s);
+            if (e != cudaSuccess) return RDA_ERR_CUDA;
+        }
+        return RDA_OK;
+    }
+    rda_status_t st = check_io_ptrs(q, k, v, log_alpha, beta, d_out);
+    if (st != RDA_OK) return st;
+    if (!dq || !dk || !dv || !d_log_alpha || !d_beta) return RDA_ERR_INVALID_ARG;
+    if (!aligned(dq, 16) || !aligned(dk, 16) || !aligned(dv, 16)) return RDA_ERR_MISALIGNED;
+    // the outputs that collect sums over CTAs start at zero
+    const size_t tok = (size_t)B * T * H;
+    if (cudaMemsetAsync(dq, 0, tok * Dk * sizeof(float), s) != cudaSuccess ||
+        cudaMemsetAsync(dk, 0, tok * Dk * sizeof(float), s) != cudaSuccess ||
+        cudaMemsetAsync(d_log_alpha, 0, tok * sizeof(float), s) != cudaSuccess ||
+        cudaMemsetAsync(d_beta, 0, tok * sizeof(float), s) != cudaSuccess ||
+        (d_write_gate && cudaMemsetAsync(d_write_gate, 0, tok * sizeof(float), s) != cudaSuccess))
+        return RDA_ERR_CUDA;
+    float *ckpt = reinterpret_cast<float *>(static_cast<char *>(workspace) + kErrorWordBytes);
+    // forward pass: the checkpoints (outputs and final state not written)
+    PrefillArgs f{};
+    f.q = q; f.k = k; f.v = v;
+    f.log_alpha = log_alpha; f.beta = beta; f.gamma = write_gate;
+    f.s0 = initial_state; f.sf = nullptr; f.out = nullptr;
+    f.num_seqs = B; f.T = T; f.total_T = B * T;
+    f.H = H; f.Dk = Dk; f.Dv = Dv; f.scale = scale;
+    f.err = static_cast<int32_t *>(workspace);
+    f.ckpt = ckpt;
+    if (launch_recurrent(f, dtype, s) != cudaSuccess) return RDA_ERR_CUDA;
+    BackwardArgs b{};
+    b.q = q; b.k = k; b.v = v; b.d_out = d_out;
+    b.log_alpha = log_alpha; b.beta = beta; b.gamma = write_gate; b.d_sf = d_final_state;
+    b.ckpt = ckpt;
+    b.dq = dq; b.dk = dk; b.dv = dv; b.d_log_alpha = d_log_alpha; b.d_beta = d_beta;
+    b.d_gamma = d_write_gate; b.d_s0 = d_initial_state;
+    b.B = B; b.T = T; b.H = H; b.Dk = Dk; b.Dv = Dv; b.scale = scale;
+    return launch_backward(b, dtype, s) == cudaSuccess ? RDA_OK : RDA_ERR_CUDA;
+}
+
 void rda_debug_set_wait_fault(int drop_chunk, unsigned long long wait_limit_ns) {
     rda::g_drop_chunk.store(drop_chunk < 0 ? -1 : drop_chunk);
     rda::g_wait_ns.store(wait_limit_ns ? (uint64_t)wait_limit_ns : rda::kDefaultWaitNs);

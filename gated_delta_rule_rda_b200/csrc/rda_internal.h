@@ -34,6 +34,7 @@ struct PrefillArgs {
     uint64_t wait_ns;            // bound of every device-side wait
     int debug_drop_chunk;        // fault injection (tests only): the scan never fills this chunk; -1 = off
     bool channel_decay;          // log_alpha is per key channel: [tokens, H, Dk]
+    float *ckpt;                 // token-sequential path: the state entering every 16-token tile, or null
     // chunked path only (filled by launch_chunked)
     const int32_t *chunk_base;   // packed: first global chunk of each sequence [N+1]
     uint8_t *workspace_chunks;   // per (chunk, head) prep results
@@ -77,6 +78,18 @@ struct PrepLaunch {
 cudaError_t launch_prep_inputs(const PrepLaunch &l, cudaStream_t s);
 cudaError_t launch_output_gate_norm(const void *o, const void *g, const float *w, void *out, long rows, int Dv,
                                     float eps, int act, rda_dtype_t dtype, cudaStream_t s);
+
+// Backward pass (rda_backward): gradients of <d_out, out> + <d_sf, final state>.
+struct BackwardArgs {
+    const void *q, *k, *v, *d_out;
+    const float *log_alpha, *beta, *gamma, *d_sf;
+    const float *ckpt;           // states entering every 16-token tile, [B][H][tiles][Dk][Dv]
+    float *dq, *dk, *dv, *d_log_alpha, *d_beta, *d_gamma, *d_s0;
+    int B, T, H, Dk, Dv;
+    float scale;
+};
+cudaError_t launch_backward(const BackwardArgs &a, rda_dtype_t dtype, cudaStream_t s);
+size_t backward_ckpt_bytes(int B, int T, int H, int Dk, int Dv);
 
 // Most tokens one multi-token decode call takes per sequence.
 constexpr int kMaxDecodeTokens = 8;

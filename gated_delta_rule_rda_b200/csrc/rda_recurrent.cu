@@ -76,6 +76,15 @@ recurrent_kernel(PrefillArgs a) {
 
     for (long tb = 0; tb < len; tb += kTile) {
         const int nt = (int)min((long)kTile, len - tb);
+        if (a.ckpt) {
+            // the state entering this tile, for the backward pass: [seq][H][tile][Dk][Dv]
+            const long ntile = (len + kTile - 1) / kTile;
+            float *ck = a.ckpt + (((size_t)n * H + h) * ntile + tb / kTile) * DK * Dv;
+#pragma unroll
+            for (int r = 0; r < R; ++r)
+                *reinterpret_cast<float4 *>(ck + (size_t)(lane + 32 * r) * Dv + j0 + jw) =
+                    make_float4(S[r][0], S[r][1], S[r][2], S[r][3]);
+        }
         __syncthreads();
         for (int idx = threadIdx.x; idx < nt * DK; idx += kThreads) {
             const int tt = idx / DK, d = idx % DK;
@@ -142,10 +151,12 @@ recurrent_kernel(PrefillArgs a) {
             if (lane < 4) o_s[tt][jw + lane] = o_mine;
         }
         __syncthreads();
-        for (int idx = threadIdx.x; idx < nt * kCols; idx += kThreads) {
-            const int tt = idx / kCols, c = idx % kCols;
-            const size_t row = (size_t)(t0 + tb + tt) * H + h;
-            Io<Tio>::st(out + row * Dv + j0 + c, o_s[tt][c]);
+        if (out) {
+            for (int idx = threadIdx.x; idx < nt * kCols; idx += kThreads) {
+                const int tt = idx / kCols, c = idx % kCols;
+                const size_t row = (size_t)(t0 + tb + tt) * H + h;
+                Io<Tio>::st(out + row * Dv + j0 + c, o_s[tt][c]);
+            }
         }
     }
 

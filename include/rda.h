@@ -328,6 +328,43 @@ rda_status_t rda_output_gate_norm(const void *o, const void *g, const float *nor
                                   long long tokens, int H, int Dv, void *stream);
 
 /*
+ * BACKWARD PASS
+ *
+ * The pages never discuss training; this is the reverse-mode derivative of
+ * the rule above (the order of the nano article's section "The other 1.5B":
+ * decay, error against the decayed state, write, read), for the loss
+ *     L = <d_out, out> + <d_final_state, final_state>
+ * of a fixed-length prefill.  Evaluated token by token in fp32: a forward pass
+ * stores the state entering every 16-token tile in the workspace, and the
+ * backward pass walks the tiles in reverse, recomputing each tile's states from
+ * its checkpoint.  Scalar decay per (token, head).
+ *
+ *   q, k, v, log_alpha, beta, write_gate, initial_state, dtype, B..Dv, scale:
+ *                  as rda_prefill_chunked (write_gate and initial_state nullable)
+ *   d_out          device, dtype, [B,T,H,Dv]
+ *   d_final_state  device fp32 [B,H,Dk,Dv] or NULL (zero)
+ *   dq, dk         device fp32 [B,T,H,Dk];  dv device fp32 [B,T,H,Dv]
+ *   d_log_alpha, d_beta  device fp32 [B,T,H]
+ *   d_write_gate   device fp32 [B,T,H]; NULL exactly when write_gate is NULL
+ *   d_initial_state  device fp32 [B,H,Dk,Dv] or NULL (not returned); it is
+ *                  also the gradient of a zero initial state when that is NULL
+ *   workspace      device, >= rda_backward_workspace_bytes(B,T,H,Dk,Dv)
+ *                  (B H ceil(T/16) Dk Dv fp32 checkpoints plus 256 bytes:
+ *                  256 MiB for B=1, T=4096, H=16, D=128)
+ * Outputs are overwritten (the call clears the summed ones first); none may
+ * alias an input.
+ */
+size_t rda_backward_workspace_bytes(int B, int T, int H, int Dk, int Dv);
+
+rda_status_t rda_backward(const void *q, const void *k, const void *v,
+                          const float *log_alpha, const float *beta, const float *write_gate,
+                          const float *initial_state, const void *d_out, const float *d_final_state,
+                          float *dq, float *dk, float *dv, float *d_log_alpha, float *d_beta,
+                          float *d_write_gate, float *d_initial_state,
+                          rda_dtype_t dtype, int B, int T, int H, int Dk, int Dv, float scale,
+                          void *workspace, size_t workspace_bytes, void *stream);
+
+/*
  * Fixed-length prefill that allocates nothing and takes no workspace.
  *
  * The pages describe no such call; it exists for callers that cannot give the

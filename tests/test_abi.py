@@ -26,7 +26,8 @@ def test_header_declares_the_entry_points():
     for want in ["rda_prefill_chunked", "rda_prefill_varlen", "rda_decode_step", "rda_decode_tokens",
                  "rda_prefill_chunked_channel", "rda_prefill_varlen_channel", "rda_decode_step_channel",
                  "rda_prefill_chunked_noalloc", "rda_debug_set_wait_fault",
-                 "rda_prep_inputs", "rda_output_gate_norm",
+                 "rda_prep_inputs", "rda_output_gate_norm", "rda_backward",
+                 "rda_backward_workspace_bytes",
                  "rda_prefill_workspace_bytes", "rda_read_device_error", "rda_status_string",
                  "rda_version"]:
         assert want in names
