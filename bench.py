@@ -445,10 +445,10 @@ def other_workloads(device, stream, rank, world, reps=5):
                            "hbm_frac": nbytes / (ms * 1e-3) / 1e9 / load_peaks()[0]}
     del inp, ws, out, sf
 
-    # per-key-channel decay at the nano shape (token-sequential fp32 kernel)
+    # per-key-channel decay at the nano shape (chunked tensor-core path)
     inp = rda_gen.workload("nano_prefill_channel_b1_t4096_h16_d128").to(device)
     B, T, H, Dk = inp.q.shape
-    ws = rda.new_workspace(rda.rda_prefill_workspace_bytes(B, T, H, Dk, Dk, 0), device)
+    ws = rda.new_workspace(rda.rda_prefill_channel_workspace_bytes(B, T, H, Dk, Dk, 0), device)
     out = torch.empty_like(inp.v)
     sf = torch.empty((B, H, Dk, Dk), device=device)
     ms = timed(lambda: rda.rda_prefill_chunked(inp.q, inp.k, inp.v, inp.log_alpha, inp.beta,

@@ -41,6 +41,8 @@ lib.rda_version.argtypes = []
 lib.rda_version.restype = ctypes.c_char_p
 lib.rda_prefill_workspace_bytes.argtypes = [_i] * 6
 lib.rda_prefill_workspace_bytes.restype = _sz
+lib.rda_prefill_channel_workspace_bytes.argtypes = [_i] * 6
+lib.rda_prefill_channel_workspace_bytes.restype = _sz
 lib.rda_prefill_chunked.argtypes = [_vp] * 9 + [_i] * 6 + [_f, _vp, _sz, _vp]
 lib.rda_prefill_chunked.restype = _i
 lib.rda_prefill_varlen.argtypes = [_vp] * 8 + [_i, _i, _vp, _vp, _vp, _i, _i, _i, _i, _f, _vp, _sz, _vp]
@@ -131,6 +133,10 @@ def rda_prefill_workspace_bytes(B, T, H, Dk, Dv, num_seqs=0) -> int:
     return int(lib.rda_prefill_workspace_bytes(B, T, H, Dk, Dv, num_seqs))
 
 
+def rda_prefill_channel_workspace_bytes(B, T, H, Dk, Dv, num_seqs=0) -> int:
+    return int(lib.rda_prefill_channel_workspace_bytes(B, T, H, Dk, Dv, num_seqs))
+
+
 def new_workspace(nbytes, device) -> torch.Tensor:
     """A workspace of ``nbytes`` (256-byte aligned by the caching allocator)
     whose device error word (first 256 bytes) starts cleared."""
@@ -164,7 +170,8 @@ def rda_prefill_chunked(q, k, v, log_alpha, beta, write_gate=None, initial_state
     if final_state is None and return_final_state:
         final_state = torch.empty((B, H, Dk, Dv), dtype=torch.float32, device=q.device)
     if workspace is None:
-        workspace = new_workspace(rda_prefill_workspace_bytes(B, T, H, Dk, Dv, 0), q.device)
+        wb = rda_prefill_channel_workspace_bytes if channel else rda_prefill_workspace_bytes
+        workspace = new_workspace(wb(B, T, H, Dk, Dv, 0), q.device)
     fn = lib.rda_prefill_chunked_channel if channel else lib.rda_prefill_chunked
     code = fn(_ptr(q), _ptr(k), _ptr(v), _ptr(log_alpha), _ptr(beta),
               _ptr(write_gate), _ptr(initial_state), _ptr(final_state),
@@ -199,7 +206,8 @@ def rda_prefill_varlen(q, k, v, log_alpha, beta, cu_seqlens, write_gate=None,
     if final_states is None and return_final_states:
         final_states = torch.empty((N, H, Dk, Dv), dtype=torch.float32, device=q.device)
     if workspace is None:
-        workspace = new_workspace(rda_prefill_workspace_bytes(1, total, H, Dk, Dv, N), q.device)
+        wb = rda_prefill_channel_workspace_bytes if log_alpha.dim() == 3 else rda_prefill_workspace_bytes
+        workspace = new_workspace(wb(1, total, H, Dk, Dv, N), q.device)
     host_ptr = None
     if cu_seqlens_host is not None:
         cu_seqlens_host = cu_seqlens_host.to(torch.int32).contiguous()
@@ -385,5 +393,6 @@ def rda_read_device_error(workspace, stream=None) -> int:
 __all__ = ["rda_prefill_chunked", "rda_prefill_varlen", "rda_decode_step", "rda_decode_tokens",
            "rda_prep_inputs", "rda_output_gate_norm", "rda_backward",
            "rda_prefill_chunked_noalloc",
-           "rda_read_device_error", "rda_debug_set_wait_fault", "rda_prefill_workspace_bytes", "new_workspace", "version",
+           "rda_read_device_error", "rda_debug_set_wait_fault", "rda_prefill_workspace_bytes",
+           "rda_prefill_channel_workspace_bytes", "new_workspace", "version",
            "RdaError", "lib", "LIB_PATH"]

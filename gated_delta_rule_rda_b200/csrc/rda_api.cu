@@ -36,13 +36,15 @@ size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
 
 // Workspace layout: [0, 256) error word; then, for packed batches, the
 // longest-first schedule (int32 per sequence); then, when the chunked
-// tensor-core path can run (Dk = 128), its per-chunk prep scratch.
+// tensor-core path can run (Dk = 128), its per-chunk prep scratch (larger
+// with a decay per key dim: the decayed K and Q images go there too).
 size_t order_bytes(int num_seqs) { return num_seqs > 0 ? align_up(sizeof(int32_t) * (size_t)num_seqs, 256) : 0; }
 
-size_t workspace_bytes(int B, long T, int H, int Dk, int Dv, int num_seqs) {
+size_t workspace_bytes(int B, long T, int H, int Dk, int Dv, int num_seqs, bool channel = false) {
     size_t b = kErrorWordBytes + order_bytes(num_seqs);
     if (chunked_supported(RDA_BF16, Dk, Dv))
-        b += align_up(chunked_workspace_bytes(num_seqs > 0 ? T : (long)B * T, (int)T, B, H, Dv, num_seqs), 256);
+        b += align_up(chunked_workspace_bytes(num_seqs > 0 ? T : (long)B * T, (int)T, B, H, Dv, num_seqs, channel),
+                      256);
     return b;
 }
 
@@ -74,8 +76,8 @@ rda_status_t validate_prefill_chunked(const void *q, const void *k, const void *
         rda_status_t st = check_io_ptrs(q, k, v, log_alpha, beta, out);
         if (st != RDA_OK) return st;
     }
-    *scratch_bytes = (chunked_supported(dtype, Dk, Dv) && !channel) ? workspace_bytes(B, T, H, Dk, Dv, 0)
-                                                                   : kErrorWordBytes;
+    *scratch_bytes = chunked_supported(dtype, Dk, Dv) ? workspace_bytes(B, T, H, Dk, Dv, 0, channel)
+                                                      : kErrorWordBytes;
     return RDA_OK;
 }
 
@@ -101,6 +103,11 @@ const char *rda_version(void) { return "0.1.0"; }
 size_t rda_prefill_workspace_bytes(int B, int T, int H, int Dk, int Dv, int num_seqs) {
     if (B < 0 || T < 0 || H <= 0 || num_seqs < 0 || !dims_ok(Dk, Dv)) return 0;
     return workspace_bytes(B, T, H, Dk, Dv, num_seqs);
+}
+
+size_t rda_prefill_channel_workspace_bytes(int B, int T, int H, int Dk, int Dv, int num_seqs) {
+    if (B < 0 || T < 0 || H <= 0 || num_seqs < 0 || !dims_ok(Dk, Dv)) return 0;
+    return workspace_bytes(B, T, H, Dk, Dv, num_seqs, true);
 }
 
 static rda_status_t prefill_chunked_impl(bool channel, const void *q, const void *k, const void *v,
@@ -140,7 +147,7 @@ static rda_status_t prefill_chunked_impl(bool channel, const void *q, const void
     a.wait_ns = ws.wait_ns;
     a.debug_drop_chunk = ws.drop_chunk;
     a.channel_decay = channel;
-    cudaError_t e = (chunked_supported(dtype, Dk, Dv) && !channel)
+    cudaError_t e = chunked_supported(dtype, Dk, Dv)
                         ? launch_chunked(a, static_cast<char *>(workspace) + kErrorWordBytes, s)
                         : launch_recurrent(a, dtype, s);
     return e == cudaSuccess ? RDA_OK : RDA_ERR_CUDA;
@@ -183,8 +190,8 @@ static rda_status_t prefill_varlen_impl(bool channel, const void *q, const void 
     if (!sizes_ok(total_T, H, Dk, Dv)) return RDA_ERR_INVALID_ARG;
     if ((long long)num_seqs * H * Dk * Dv >= (1LL << 31)) return RDA_ERR_INVALID_ARG;
     if (num_seqs > 0 && !cu_seqlens) return RDA_ERR_INVALID_ARG;
-    const bool chunked = chunked_supported(dtype, Dk, Dv) && !channel;
-    const size_t need = chunked ? workspace_bytes(1, total_T, H, Dk, Dv, num_seqs)
+    const bool chunked = chunked_supported(dtype, Dk, Dv);
+    const size_t need = chunked ? workspace_bytes(1, total_T, H, Dk, Dv, num_seqs, channel)
                                 : kErrorWordBytes + order_bytes(num_seqs);
     if (!workspace || workspace_bytes_given < need) return RDA_ERR_WORKSPACE;
     if (!aligned(workspace, 256)) return RDA_ERR_MISALIGNED;

@@ -62,6 +62,12 @@ constexpr uint32_t kImgW = 0;          // -W, bf16 K-major SW128, 2 halves of 8 
 constexpr uint32_t kImgP = 16384;      // P, bf16 K-major SW128, 8 KiB
 constexpr uint32_t kImgU = 24576;      // U', bf16, value slices of width NV, each [64][NV];
                                        // then e^{g_t} and e^{g_C - g_t}: 2 x 64 fp32
+                                       // (per-key-channel decay: both 1, then e^{G_C} per key dim,
+                                       // 128 fp32, then K~ = K o e^{G_C - G} and Q~ = Q o e^{G},
+                                       // bf16 K-major SW128 like the K and Q tiles)
+__host__ __device__ constexpr uint32_t img_decay(int Dv) { return kImgU + 64 * Dv * 2; }
+__host__ __device__ constexpr uint32_t img_kt(int Dv) { return img_decay(Dv) + 1024; }
+__host__ __device__ constexpr uint32_t img_qt(int Dv) { return img_kt(Dv) + 16384; }
 
 __device__ __forceinline__ uint64_t globaltimer() {
     uint64_t t;
@@ -310,8 +316,9 @@ constexpr uint32_t PS_AF = 16384;      // A fp32 [64][kLd]; after the solve V [6
 constexpr uint32_t PS_TF = PS_AF + 64 * kLd * 4;     // Q [64 x 128] (halves of 8 KiB, SW128) until the
                                                      // solve; T fp32 [64][kLd]; then the two T images
 constexpr uint32_t PS_XS = PS_TF + 64 * kLd * 4;     // 4 x 16x8 fp32
-constexpr uint32_t PS_G = PS_XS + 4 * 128 * 4;       // g, beta, beta*gamma, e^{ref-g}, e^g, e^{g_C-g}: 6 x 64 fp32
-constexpr uint32_t PS_BAR = PS_G + 6 * 64 * 4;
+constexpr uint32_t PS_G = PS_XS + 4 * 128 * 4;       // g, beta, beta*gamma, e^{ref-g}, e^g, e^{g_C-g}: 6 x 64 fp32,
+                                                     // then (per-channel decay) e^{G_C} per key dim: 128 fp32
+constexpr uint32_t PS_BAR = PS_G + 8 * 64 * 4;
 constexpr uint32_t PS_TMEMPTR = PS_BAR + 10 * 8;
 constexpr uint32_t PS_FLAGS = PS_TMEMPTR + 4;
 constexpr uint32_t kPrepSmem = PS_FLAGS + 8 + 1024;   // flags: compute threads', TMA / MMA thread's
@@ -323,6 +330,11 @@ constexpr uint32_t PS_WIMG = PS_K;            // -W image, over K (after the W M
 constexpr uint32_t PS_UIMG = PS_V;            // U' slices, over V (after the U' MMA)
 static_assert(PS_AF % 1024 == 0 && PS_TF % 1024 == 0, "SW128 tiles need 1024-byte alignment");
 static_assert(4 * (kPrepSmem + 1024) <= 233472, "four prep CTAs per SM");
+// per-key-channel decay: the cumulative log decay G[t][d] of the chunk, fp32 [64][kGld]
+constexpr int kGld = 132;
+constexpr uint32_t PS_GCH = (kPrepSmem - 1024 + 15) / 16 * 16;
+constexpr uint32_t kPrepSmemCh = PS_GCH + 64 * kGld * 4 + 1024;
+static_assert(2 * (kPrepSmemCh + 1024) <= 233472, "two per-channel prep CTAs per SM");
 // TMEM columns: K K^T and Q K^T side by side, then W, then U' (one at a time)
 constexpr uint32_t PT_KK = 0, PT_QK = 64, PT_W = 0, PT_U = 0;
 enum PrepBar { PB_FULL = 0, PB_VFULL, PB_KK, PB_QK, PB_TREADY, PB_W, PB_WFREE, PB_U, PB_DRAIN, kPrepBars };
@@ -375,7 +387,7 @@ __device__ __forceinline__ RowGates load_gates(const PrefillArgs &a, long row0, 
     RowGates x{0.f, 0.f, 1.f};
     if (r < 64 && r < lenc) {
         const size_t row = (size_t)(row0 + r) * a.H + h;
-        x.la = a.log_alpha[row];
+        if (!a.channel_decay) x.la = a.log_alpha[row];
         x.be = a.beta[row];
         if (a.gamma) x.ga = a.gamma[row];
     }
@@ -446,8 +458,170 @@ __device__ __forceinline__ void gram_rows(uint32_t taddr, int ta, int lane, cons
     }
 }
 
-template <int NV>
-__global__ void __launch_bounds__(kPrepThreads, 4)
+// ---------------------------------------------------------------------------
+// Per-key-channel decay: the decayed Grams.
+//
+// With one decay per key dim, the chunk's Gram entries are
+//     X[t] . (K[s] o e^{G[t] - G[s]})   (X = K for A, Q for P),
+// not a plain product times a mask.  Split the factor around a reference token
+// r of the column block, e^{G[t] - G[r]} on the row operand and e^{G[r] - G[s]}
+// on the column operand, and each 16 x 16 block is an ordinary product of
+// scaled operands.  References: for an off-diagonal block the last token of the
+// column block (both factors <= 1), for a diagonal block its first token (row
+// factors <= 1, column factors at most e^{15 x 5}, well inside the range of
+// bf16 and fp32).  A factor that underflows belongs to an entry far below
+// every other one in the row.  The operands are scaled in fp32 and rounded to
+// bf16 in the MMA fragments (mma.sync m16n8k16, fp32 accumulation).
+// ---------------------------------------------------------------------------
+__device__ __forceinline__ void mma16816_g(float *d, const uint32_t *a, uint32_t b0, uint32_t b1) {
+    asm volatile(
+        "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
+        "{%0,%1,%2,%3};"
+        : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+        : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
+}
+// Two consecutive key dims d, d + 1 of row t of a bf16 K-major SW128 tile
+// (64-column halves of 8 KiB), scaled by e^{s (G[t][d] - G[ref][d])} (s = +-1),
+// packed as a bf16 pair.
+__device__ __forceinline__ uint32_t scaled_pair(const uint8_t *tile, const float *Gm, int t, int d, int ref,
+                                                float sgn) {
+    const uint32_t raw = *reinterpret_cast<const uint32_t *>(tile + (d >> 6) * 8192 + swz(t, (d & 63) >> 3, 128) +
+                                                             (d & 7) * 2);
+    const float2 x = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(&raw));
+    const float2 gt = *reinterpret_cast<const float2 *>(Gm + t * kGld + d);
+    const float2 gr = *reinterpret_cast<const float2 *>(Gm + ref * kGld + d);
+    return pack_bf16(x.x * __expf(sgn * (gt.x - gr.x)), x.y * __expf(sgn * (gt.y - gr.y)));
+}
+// acc[nt] (n-tiles of 8 columns) += the 16 x 16 block (rows 16 rb.., columns
+// 16 cb..) of sum_d X[t][d] K[s][d] e^{G[t][d] - G[s][d]}, split around `ref`.
+__device__ __forceinline__ void gram_block_ch(const uint8_t *xt, const uint8_t *kt, const float *Gm, int rb, int cb,
+                                              int ref, int lane, float (&acc)[2][4]) {
+    const int g = lane >> 2, tg = lane & 3;
+    const int t0 = 16 * rb + g, t1 = t0 + 8;
+#pragma unroll 2
+    for (int ks = 0; ks < 8; ++ks) {
+        const int d = 16 * ks + 2 * tg;
+        uint32_t af[4];
+        af[0] = scaled_pair(xt, Gm, t0, d, ref, 1.f);
+        af[1] = scaled_pair(xt, Gm, t1, d, ref, 1.f);
+        af[2] = scaled_pair(xt, Gm, t0, d + 8, ref, 1.f);
+        af[3] = scaled_pair(xt, Gm, t1, d + 8, ref, 1.f);
+#pragma unroll
+        for (int nt = 0; nt < 2; ++nt) {
+            const int sc = 16 * cb + 8 * nt + g;
+            const uint32_t b0 = scaled_pair(kt, Gm, sc, d, ref, -1.f);
+            const uint32_t b1 = scaled_pair(kt, Gm, sc, d + 8, ref, -1.f);
+            mma16816_g(acc[nt], af, b0, b1);
+        }
+    }
+}
+
+// The per-channel prep's work up to the UT solve, by the 128 compute threads
+// (cw = 0..127; r = the thread's TMEM lane, the token whose gates it loaded):
+// the cumulative log decay G[t][d] of every key dim, beta and beta*gamma; the
+// decayed Grams A (strictly lower, rows times beta_t) into the fp32 work matrix
+// and P (lower, diagonal kept) as its image; the images K~ = K o e^{G_C - G} and
+// Q~ = Q o e^{G}; and K o e^{G} in place of the K tile (the B operand of W).
+// The scalar decay factors of the image are set to 1 and e^{G_C} per key dim
+// follows them.
+__device__ __forceinline__ void prep_channel_front(const PrefillArgs &a, uint8_t *sm, float *g_s, RowGates gates,
+                                                   int cw, int r, int lenc, long row0, int h, uint8_t *img,
+                                                   uint64_t *bars, volatile int *abort_flag) {
+    const int lane = cw & 31, wq = cw >> 5;
+    float *b_s = g_s + 64, *bg_s = g_s + 128, *eg_s = g_s + 256, *ed_s = g_s + 320, *dc_s = g_s + 384;
+    float *Gm = reinterpret_cast<float *>(sm + PS_GCH);
+    const int H = a.H;
+    {
+        // key dim cw: G[t] = sum of log alpha over the chunk's tokens up to t (0 past the end)
+        const float *la = a.log_alpha + ((size_t)row0 * H + h) * kDK + cw;
+        const size_t step = (size_t)H * kDK;
+        float x[64];
+#pragma unroll
+        for (int t = 0; t < 64; ++t) x[t] = t < lenc ? la[t * step] : 0.f;
+        float acc = 0.f;
+#pragma unroll
+        for (int t = 0; t < 64; ++t) {
+            acc += x[t];
+            Gm[t * kGld + cw] = acc;
+        }
+        dc_s[cw] = __expf(acc);
+    }
+    if (r < 64) {
+        b_s[r] = gates.be;
+        bg_s[r] = gates.be * gates.ga;
+        eg_s[r] = 1.f;
+        ed_s[r] = 1.f;
+    }
+    if (cw == 0 && !wait_bar(&bars[PB_FULL], 0, abort_flag, a.err, a.wait_ns)) *abort_flag = 1;
+    named_bar_sync(1, 128);
+    // only compute thread 0 writes the flag, and only before the barrier: uniform
+    const bool go = !*abort_flag;
+    // the tiles have landed (complete already); this wait makes the copies visible here
+    if (go) wait_bar(&bars[PB_FULL], 0, abort_flag, a.err, a.wait_ns);
+    float *Af = reinterpret_cast<float *>(sm + PS_AF);
+    const uint8_t *kt = sm + PS_K, *qt = sm + PS_Q;
+    const int g = lane >> 2, tg = lane & 3;
+    for (int task = wq; go && task < 20; task += 4) {
+        const bool isP = task >= 10;
+        int idx = isP ? task - 10 : task, rb = 0;            // block pairs (rb, cb), cb <= rb, in order
+        while (idx > rb) {
+            idx -= rb + 1;
+            ++rb;
+        }
+        const int cb = idx;
+        const int ref = rb == cb ? 16 * cb : 16 * cb + 15;
+        float acc[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
+        gram_block_ch(isP ? qt : kt, kt, Gm, rb, cb, ref, lane, acc);
+#pragma unroll
+        for (int nt = 0; nt < 2; ++nt)
+#pragma unroll
+            for (int hh = 0; hh < 2; ++hh) {
+                const int t = 16 * rb + g + 8 * hh, s0 = 16 * cb + 8 * nt + 2 * tg;
+                float v0 = acc[nt][2 * hh], v1 = acc[nt][2 * hh + 1];
+                if (isP) {
+                    v0 = s0 <= t ? v0 : 0.f;
+                    v1 = s0 + 1 <= t ? v1 : 0.f;
+                    *reinterpret_cast<uint32_t *>(img + kImgP + swz(t, s0 >> 3, 128) + (s0 & 7) * 2) =
+                        pack_bf16(v0, v1);
+                } else {
+                    const float be = b_s[t];
+                    *reinterpret_cast<float2 *>(Af + t * kLd + s0) =
+                        make_float2(s0 < t ? be * v0 : 0.f, s0 + 1 < t ? be * v1 : 0.f);
+                }
+            }
+    }
+    // the blocks of P's image above the diagonal are zero (the scan multiplies by all 64 columns)
+    for (int i = cw; go && i < 6 * 16 * 8; i += 128) {
+        const int blk = i >> 7, t = (i >> 3) & 15, pr = i & 7;
+        const int rb = blk < 3 ? 0 : (blk < 5 ? 1 : 2);
+        const int cb = blk < 3 ? blk + 1 : (blk < 5 ? blk - 1 : 3);
+        const int tt = 16 * rb + t, s0 = 16 * cb + 2 * pr;
+        *reinterpret_cast<uint32_t *>(img + kImgP + swz(tt, s0 >> 3, 128) + (s0 & 7) * 2) = 0u;
+    }
+    named_bar_sync(1, 128);
+    if (go) {
+        // key dims dp, dp + 1 of rows 32 th .. 32 th + 31
+        const int dp = 2 * (cw & 63), th = cw >> 6;
+        const float2 gC = *reinterpret_cast<const float2 *>(Gm + 63 * kGld + dp);
+        uint8_t *kimg = img + img_kt(a.Dv), *qimg = img + img_qt(a.Dv);
+        for (int t = 32 * th; t < 32 * th + 32; ++t) {
+            const uint32_t off = (dp >> 6) * 8192 + swz(t, (dp & 63) >> 3, 128) + (dp & 7) * 2;
+            const float2 gt = *reinterpret_cast<const float2 *>(Gm + t * kGld + dp);
+            const uint32_t kr = *reinterpret_cast<const uint32_t *>(sm + PS_K + off);
+            const uint32_t qr = *reinterpret_cast<const uint32_t *>(sm + PS_Q + off);
+            const float2 kx = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(&kr));
+            const float2 qx = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(&qr));
+            const float e0 = __expf(gt.x), e1 = __expf(gt.y);
+            *reinterpret_cast<uint32_t *>(kimg + off) =
+                pack_bf16(kx.x * __expf(gC.x - gt.x), kx.y * __expf(gC.y - gt.y));
+            *reinterpret_cast<uint32_t *>(qimg + off) = pack_bf16(qx.x * e0, qx.y * e1);
+            *reinterpret_cast<uint32_t *>(sm + PS_K + off) = pack_bf16(kx.x * e0, kx.y * e1);
+        }
+    }
+}
+
+template <int NV, bool CH>
+__global__ void __launch_bounds__(kPrepThreads, CH ? 2 : 4)
 prep_kernel(const __grid_constant__ PrepMaps maps, const PrefillArgs a) {
     extern __shared__ uint8_t smem_raw[];
     uint8_t *sm = smem_align_1024(smem_raw);
@@ -508,7 +682,8 @@ prep_kernel(const __grid_constant__ PrepMaps maps, const PrefillArgs a) {
             constexpr uint32_t ID_W = idesc_bf16(64, 128, 0, 1);
             const uint32_t ID_U = Dv == 128 ? idesc_bf16(64, 128, 0, 1) : idesc_bf16(64, 64, 0, 1);
             bool ok = wait_bar2(&bars[PB_FULL], 0, abort_flag, agent_flag, a.err, a.wait_ns);
-            if (ok) {
+            if (ok && CH) ok = wait_bar2(&bars[PB_TREADY], 0, abort_flag, agent_flag, a.err, a.wait_ns);
+            if (ok && !CH) {
                 tc_fence_after();
 #pragma unroll
                 for (int kk = 0; kk < 8; ++kk) {     // K K^T: A = B = the K tile (K-major)
@@ -564,6 +739,9 @@ prep_kernel(const __grid_constant__ PrepMaps maps, const PrefillArgs a) {
         float *Tf = reinterpret_cast<float *>(sm + PS_TF);
         float *Xs = reinterpret_cast<float *>(sm + PS_XS);
 
+        if constexpr (CH) {
+            prep_channel_front(a, sm, g_s, gates, cw, r, lenc, row0, h, img, bars, abort_flag);
+        } else {
         chunk_gates(gates, r, lane, g_s);
         if (cw == 0 && !wait_bar(&bars[PB_KK], 0, abort_flag, a.err, a.wait_ns)) *abort_flag = 1;
         named_bar_sync(1, 128);
@@ -599,6 +777,7 @@ prep_kernel(const __grid_constant__ PrepMaps maps, const PrefillArgs a) {
             }
             tc_fence_before();
         }
+        }
         named_bar_sync(1, 128);      // Q is dead: T goes there
         if (!*abort_flag) {
             ut_solve(Af, Tf, Xs, cw);      // ends with a barrier: A is dead from here
@@ -615,7 +794,7 @@ prep_kernel(const __grid_constant__ PrepMaps maps, const PrefillArgs a) {
                 float z1[8], z2[8];
 #pragma unroll
                 for (int e = 0; e < 8; ++e) {
-                    z1[e] = tv[e] * b_s[s0 + e] * eg_s[s0 + e];
+                    z1[e] = CH ? tv[e] * b_s[s0 + e] : tv[e] * b_s[s0 + e] * eg_s[s0 + e];
                     z2[e] = tv[e] * bg_s[s0 + e];
                 }
                 y1[cc] = pack8(z1);
@@ -687,7 +866,7 @@ prep_kernel(const __grid_constant__ PrepMaps maps, const PrefillArgs a) {
         if (cw == 0) {
             if (!*abort_flag) {
                 bulk_store(img + kImgU, sm + PS_UIMG, 64 * Dv * 2);
-                bulk_store(img + kImgU + 64 * Dv * 2, eg_s, 512);     // e^g, e^{g_C - g}
+                bulk_store(img + img_decay(Dv), eg_s, CH ? 1024 : 512);     // e^g, e^{g_C - g} (, e^{G_C})
                 bulk_commit();
             }
             bulk_wait_reads();
@@ -801,7 +980,7 @@ __device__ __forceinline__ void ld_b(uint32_t base, int k0, int n0, int lane, ui
     }
 }
 
-template <int NV>
+template <int NV, bool CH>
 __global__ void __launch_bounds__(kScanThreads, 1)
 scan_kernel(const __grid_constant__ ScanMaps maps, const PrefillArgs a) {
     extern __shared__ uint8_t smem_raw[];
@@ -866,16 +1045,23 @@ scan_kernel(const __grid_constant__ ScanMaps maps, const PrefillArgs a) {
                 uint64_t *full = &bars[SB_FULL + st];
                 uint8_t *stg = sm + st * SS_STAGE;
                 const uint8_t *img = a.workspace_chunks + ((size_t)(gc0 + c) * H + h) * a.chunk_bytes;
-                mbar_arrive_expect_tx(full, 16384 * 3 + 8192 + UBYTES + 512);
-                const int r0 = (int)(t0 + (long)c * kC);
-                tma_load_3d(stg + SS_K, &maps.k, full, 0, h, r0);
-                tma_load_3d(stg + SS_K + 8192, &maps.k, full, 64, h, r0);
+                constexpr uint32_t GBYTES = CH ? 1024 : 512;
+                mbar_arrive_expect_tx(full, 16384 * 3 + 8192 + UBYTES + GBYTES);
+                if constexpr (CH) {
+                    // per-channel decay: the prep's K o e^{G_C - G} and Q o e^{G} images
+                    bulk_load(stg + SS_K, img + img_kt(Dv), 16384, full);
+                    bulk_load(stg + SS_Q, img + img_qt(Dv), 16384, full);
+                } else {
+                    const int r0 = (int)(t0 + (long)c * kC);
+                    tma_load_3d(stg + SS_K, &maps.k, full, 0, h, r0);
+                    tma_load_3d(stg + SS_K + 8192, &maps.k, full, 64, h, r0);
+                    tma_load_3d(stg + SS_Q, &maps.q, full, 0, h, r0);
+                    tma_load_3d(stg + SS_Q + 8192, &maps.q, full, 64, h, r0);
+                }
                 bulk_load(stg + SS_W, img + kImgW, 16384, full);
-                tma_load_3d(stg + SS_Q, &maps.q, full, 0, h, r0);
-                tma_load_3d(stg + SS_Q + 8192, &maps.q, full, 64, h, r0);
                 bulk_load(stg + SS_P, img + kImgP, 8192, full);
                 bulk_load(stg + SS_U, img + kImgU + (size_t)slice * UBYTES, UBYTES, full);
-                bulk_load(stg + SS_G, img + kImgU + 64 * Dv * 2, 512, full);
+                bulk_load(stg + SS_G, img + img_decay(Dv), GBYTES, full);
             }
             // the CTA may not exit with copies in flight: after an abort the scan
             // warps stop consuming, so wait (bounded) for every stage's last fill
@@ -962,8 +1148,8 @@ scan_kernel(const __grid_constant__ ScanMaps maps, const PrefillArgs a) {
                     mma16816(ao[nt], aq[kk], bf[kk][2 * nt], bf[kk][2 * nt + 1]);
                 }
         }
-        {
-            const float ea = eg_s[ta], eb = eg_s[tb];     // e^{g_t}
+        if constexpr (!CH) {
+            const float ea = eg_s[ta], eb = eg_s[tb];     // e^{g_t} (per-channel: inside Q's image)
 #pragma unroll
             for (int nt = 0; nt < NT; ++nt) {
                 ao[nt][0] *= ea;
@@ -972,8 +1158,9 @@ scan_kernel(const __grid_constant__ ScanMaps maps, const PrefillArgs a) {
                 ao[nt][3] *= eb;
             }
         }
-        // ---- U and U~ = e^{g_C - g_t} U -> shared memory (B operands of P U and K^T U~)
-        const float da = ed_s[ta], db = ed_s[tb];
+        // ---- U and U~ = e^{g_C - g_t} U -> shared memory (B operands of P U and K^T U~;
+        // per-channel: the factor is inside K's image and U~ = U)
+        const float da = CH ? 1.f : ed_s[ta], db = CH ? 1.f : ed_s[tb];
 #pragma unroll
         for (int nt = 0; nt < NT; ++nt) {
             const int j = c0 + 8 * nt + 2 * tg;
@@ -1013,14 +1200,16 @@ scan_kernel(const __grid_constant__ ScanMaps maps, const PrefillArgs a) {
                     for (int nt = 0; nt < NT; ++nt)
                         mma16816(ds[kk & 1][mt][nt], af[kk][mt], bf[kk][2 * nt], bf[kk][2 * nt + 1]);
         }
-        const float eC = eg_s[63];                    // e^{g_C}
+        const float *dC = eg_s + 128;                 // per-channel: e^{G_C} of each key dim
 #pragma unroll
         for (int mt = 0; mt < 2; ++mt)
 #pragma unroll
             for (int nt = 0; nt < NT; ++nt)
 #pragma unroll
-                for (int i = 0; i < 4; ++i)
+                for (int i = 0; i < 4; ++i) {
+                    const float eC = CH ? dC[32 * rg + 16 * mt + g + 8 * (i >> 1)] : eg_s[63];     // e^{g_C}
                     S[mt][nt][i] = fmaf(eC, S[mt][nt][i], ds[0][mt][nt][i] + ds[1][mt][nt][i]);
+                }
         // ---- O += P U for rows t = 16rg .. 16rg+15, then the store (masked tail)
         {
             const uint32_t uub = smb + L::UU;
@@ -1145,20 +1334,20 @@ int choose_nv(long units, int Dv) {
     return units * (Dv / 32) >= 148 ? 32 : 16;
 }
 
-template <int NV>
+template <int NV, bool CH>
 cudaError_t init_attrs() {
     static std::once_flag once;
     static cudaError_t attr = cudaSuccess;
     std::call_once(once, [] {
-        attr = set_smem(prep_kernel<NV>, kPrepSmem);
-        if (attr == cudaSuccess) attr = set_smem(scan_kernel<NV>, ScanSmem<NV>::BYTES);
+        attr = set_smem(prep_kernel<NV, CH>, CH ? kPrepSmemCh : kPrepSmem);
+        if (attr == cudaSuccess) attr = set_smem(scan_kernel<NV, CH>, ScanSmem<NV>::BYTES);
     });
     return attr;
 }
 
-template <int NV>
+template <int NV, bool CH>
 cudaError_t launch_nv(const PrefillArgs &a, long chunks_grid, cudaStream_t s) {
-    cudaError_t e = init_attrs<NV>();
+    cudaError_t e = init_attrs<NV, CH>();
     if (e != cudaSuccess) return e;
     PrepMaps pm;
     ScanMaps sm;
@@ -1176,7 +1365,7 @@ cudaError_t launch_nv(const PrefillArgs &a, long chunks_grid, cudaStream_t s) {
     const dim3 chunk_grid((unsigned)chunks_grid, a.H, 1);
 
     if (chunks_grid > 0) {
-        prep_kernel<NV><<<chunk_grid, kPrepThreads, kPrepSmem, s>>>(pm, a);
+        prep_kernel<NV, CH><<<chunk_grid, kPrepThreads, CH ? kPrepSmemCh : kPrepSmem, s>>>(pm, a);
         if ((e = cudaGetLastError()) != cudaSuccess) return e;
     }
     // programmatic stream serialization: the scan's launch and prologue overlap
@@ -1191,10 +1380,14 @@ cudaError_t launch_nv(const PrefillArgs &a, long chunks_grid, cudaStream_t s) {
     attr[0].val.programmaticStreamSerializationAllowed = chunks_grid > 0 ? 1 : 0;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
-    return cudaLaunchKernelEx(&cfg, scan_kernel<NV>, sm, a);
+    return cudaLaunchKernelEx(&cfg, scan_kernel<NV, CH>, sm, a);
 }
 
-size_t image_bytes(int Dv) { return (size_t)kImgU + 64 * (size_t)Dv * 2 + 512; }
+// Bytes of one (chunk, head) image: -W, P, U', the decay factors; with a decay
+// per key dim, e^{G_C} and the K and Q images too.
+size_t image_bytes(int Dv, bool channel) {
+    return channel ? (size_t)img_qt(Dv) + 16384 : (size_t)kImgU + 64 * (size_t)Dv * 2 + 512;
+}
 
 size_t header_bytes(int num_seqs) {
     size_t b = 4 * (size_t)(num_seqs + 1);
@@ -1207,11 +1400,11 @@ bool chunked_supported(rda_dtype_t dtype, int Dk, int Dv) {
     return dtype == RDA_BF16 && Dk == kDK && (Dv == 64 || Dv == 128);
 }
 
-size_t chunked_workspace_bytes(long total_T, int T, int B, int H, int Dv, int num_seqs) {
+size_t chunked_workspace_bytes(long total_T, int T, int B, int H, int Dv, int num_seqs, bool channel) {
     long chunks;
     if (num_seqs > 0) chunks = (total_T + kC - 1) / kC + num_seqs;     // packed: upper bound
     else chunks = (long)B * ((T + kC - 1) / kC);
-    return header_bytes(num_seqs) + (size_t)chunks * H * image_bytes(Dv);
+    return header_bytes(num_seqs) + (size_t)chunks * H * image_bytes(Dv, channel);
 }
 
 cudaError_t launch_chunked(const PrefillArgs &a0, void *scratch, cudaStream_t s) {
@@ -1219,7 +1412,7 @@ cudaError_t launch_chunked(const PrefillArgs &a0, void *scratch, cudaStream_t s)
     uint8_t *ws = static_cast<uint8_t *>(scratch);
     const int nseq_hdr = a.cu_seqlens ? a.num_seqs : 0;
     a.workspace_chunks = ws + header_bytes(nseq_hdr);
-    a.chunk_bytes = image_bytes(a.Dv);
+    a.chunk_bytes = image_bytes(a.Dv, a.channel_decay);
     long chunks_grid;
     if (a.cu_seqlens) {
         int32_t *chunk_base = reinterpret_cast<int32_t *>(ws);
@@ -1234,7 +1427,10 @@ cudaError_t launch_chunked(const PrefillArgs &a0, void *scratch, cudaStream_t s)
     }
     if (a.total_T == 0) chunks_grid = 0;
     const long units = (long)a.num_seqs * a.H;
-    return choose_nv(units, a.Dv) == 32 ? launch_nv<32>(a, chunks_grid, s) : launch_nv<16>(a, chunks_grid, s);
+    const bool wide = choose_nv(units, a.Dv) == 32;
+    if (a.channel_decay)
+        return wide ? launch_nv<32, true>(a, chunks_grid, s) : launch_nv<16, true>(a, chunks_grid, s);
+    return wide ? launch_nv<32, false>(a, chunks_grid, s) : launch_nv<16, false>(a, chunks_grid, s);
 }
 
 }  // namespace rda

@@ -102,7 +102,7 @@ cudaError_t launch_decode_tokens(const DecodeArgs &a, rda_dtype_t dtype, cudaStr
 cudaError_t launch_chunked(const PrefillArgs &a, void *scratch, cudaStream_t s);
 bool chunked_supported(rda_dtype_t dtype, int Dk, int Dv);
 // Scratch the chunked path needs: fixed-length batches pass num_seqs = 0.
-size_t chunked_workspace_bytes(long total_T, int T, int B, int H, int Dv, int num_seqs);
+size_t chunked_workspace_bytes(long total_T, int T, int B, int H, int Dv, int num_seqs, bool channel = false);
 
 // Host-side argument checks of rda_prefill_chunked except those of the
 // workspace; enqueues nothing.  On RDA_OK, *scratch_bytes is the workspace

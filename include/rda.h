@@ -231,10 +231,16 @@ rda_status_t rda_decode_tokens(const void *q, const void *k, const void *v,
  * layouts, results and errors are those of the scalar calls except:
  *   log_alpha  device fp32 [B,T,H,Dk] (varlen: [total_T,H,Dk]; decode: [B,H,Dk]),
  *              each value in [-5, 0] (precondition, not checked)
- * The prefill calls evaluate the rule token by token in fp32 (any dtype,
- * Dk and Dv in {64, 128}); they need only the error word of the workspace
- * but accept any workspace of at least rda_prefill_workspace_bytes(...).
+ * The prefill calls take the chunked tensor-core path for bf16 with Dk = 128
+ * (the decayed Grams split around a reference token of each 16-token block,
+ * and the decayed K and Q of each chunk stored as images next to -W, P and
+ * U'), and evaluate the rule token by token in fp32 otherwise (fp32, or
+ * Dk = 64).  Their workspace is rda_prefill_channel_workspace_bytes(...) bytes
+ * (256-byte aligned; larger than the scalar calls' on the chunked path);
+ * RDA_ERR_WORKSPACE when it is missing or smaller.
  */
+size_t rda_prefill_channel_workspace_bytes(int B, int T, int H, int Dk, int Dv, int num_seqs);
+
 rda_status_t rda_prefill_chunked_channel(const void *q, const void *k, const void *v,
                                          const float *log_alpha, const float *beta,
                                          const float *write_gate,

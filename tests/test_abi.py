@@ -28,7 +28,8 @@ def test_header_declares_the_entry_points():
                  "rda_prefill_chunked_noalloc", "rda_debug_set_wait_fault",
                  "rda_prep_inputs", "rda_output_gate_norm", "rda_backward",
                  "rda_backward_workspace_bytes",
-                 "rda_prefill_workspace_bytes", "rda_read_device_error", "rda_status_string",
+                 "rda_prefill_workspace_bytes", "rda_prefill_channel_workspace_bytes",
+                 "rda_read_device_error", "rda_status_string",
                  "rda_version"]:
         assert want in names
 
@@ -54,6 +55,12 @@ def test_workspace_query():
     assert rda.rda_prefill_workspace_bytes(1, 100, 16, 128, 128, 64) >= 256 + 64 * 4
     assert rda.rda_prefill_workspace_bytes(1, 100, 16, 96, 128, 0) == 0
     assert rda.rda_prefill_workspace_bytes(-1, 100, 16, 128, 128, 0) == 0
+    # per-key-channel decay: the decayed K and Q images (32 KiB per chunk and head) on top
+    ch = rda.rda_prefill_channel_workspace_bytes(1, 4096, 16, 128, 128, 0)
+    assert ch >= rda.rda_prefill_workspace_bytes(1, 4096, 16, 128, 128, 0) + 64 * 16 * 32 * 1024
+    assert rda.rda_prefill_channel_workspace_bytes(1, 4096, 16, 64, 64, 0) == \
+        rda.rda_prefill_workspace_bytes(1, 4096, 16, 64, 64, 0)
+    assert rda.rda_prefill_channel_workspace_bytes(1, 100, 16, 96, 128, 0) == 0
 
 
 # Fake device addresses: never dereferenced, because validation fails first.

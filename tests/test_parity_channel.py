@@ -1,5 +1,8 @@
 """GPU parity of the per-key-channel decay entry points against the fp64
 oracle (log alpha with one value per key dimension), through the C ABI.
+bf16 with Dk = 128 runs the chunked tensor-core path (decayed Grams split
+around reference tokens, decayed K and Q images); fp32 and Dk = 64 run the
+token-sequential kernel.
 
 Relative L2 over the whole returned tensors: <= 1e-5 for fp32 inputs, <= 1e-2
 for bf16 inputs, outputs and final states both.
@@ -19,7 +22,7 @@ def _gpu(inp, scale=1.0):
     import gated_delta_rule_rda_b200 as rda
     d = inp.to("cuda")
     B, T, H, Dk = d.q.shape
-    ws = rda.new_workspace(rda.rda_prefill_workspace_bytes(B, T, H, Dk, d.v.shape[-1], 0), "cuda")
+    ws = rda.new_workspace(rda.rda_prefill_channel_workspace_bytes(B, T, H, Dk, d.v.shape[-1], 0), "cuda")
     out, sf = rda.rda_prefill_chunked(d.q, d.k, d.v, d.log_alpha, d.beta, write_gate=d.gamma,
                                       initial_state=d.initial_state, scale=scale, workspace=ws)
     torch.cuda.synchronize()
@@ -51,6 +54,52 @@ def test_channel_bf16_ragged(cuda_device, T):
     inp = rda_gen.fixed_inputs(2, T, 3, 128, 128, dtype=torch.bfloat16, seed=310 + T, s0=True,
                                channel=True)
     _check(inp)
+
+
+@pytest.mark.parametrize("B,T,H,Dv", [(1, 1, 1, 64), (3, 129, 2, 64), (1, 320, 4, 128)])
+def test_channel_bf16_chunked_shapes(cuda_device, B, T, H, Dv):
+    inp = rda_gen.fixed_inputs(B, T, H, 128, Dv, dtype=torch.bfloat16, seed=305 + T + Dv, s0=True,
+                               gamma=True, channel=True)
+    _check(inp, scale=0.5)
+
+
+def test_channel_bf16_mixed_channels(cuda_device):
+    """Within every token, key dims that do not decay (log alpha 0) next to dims
+    at the bound (-5) and in between: the split factors of the Grams span their
+    whole range."""
+    inp = rda_gen.fixed_inputs(2, 200, 2, 128, 128, dtype=torch.bfloat16, seed=315, s0=True,
+                               gamma=True, channel=True)
+    la = inp.log_alpha.clone()
+    la[..., 0::4] = 0.0
+    la[..., 1::4] = -5.0
+    inp.log_alpha = la
+    _check(inp)
+
+
+def test_channel_bf16_equal_channels_match_scalar(cuda_device):
+    """Both chunked paths: per-channel with log alpha repeated over the key dims
+    against the scalar call (different roundings of the same quantities)."""
+    import gated_delta_rule_rda_b200 as rda
+    inp = rda_gen.fixed_inputs(2, 300, 2, 128, 128, dtype=torch.bfloat16, seed=325, s0=True, gamma=True)
+    d = inp.to("cuda")
+    la_ch = d.log_alpha[..., None].expand(-1, -1, -1, 128).contiguous()
+    o_s, s_s = rda.rda_prefill_chunked(d.q, d.k, d.v, d.log_alpha, d.beta, write_gate=d.gamma,
+                                       initial_state=d.initial_state)
+    o_c, s_c = rda.rda_prefill_chunked(d.q, d.k, d.v, la_ch, d.beta, write_gate=d.gamma,
+                                       initial_state=d.initial_state)
+    torch.cuda.synchronize()
+    assert rel_l2(to_np(o_c), to_np(o_s)) <= 1e-2 and rel_l2(to_np(s_c), to_np(s_s)) <= 1e-2
+
+
+def test_channel_workspace_checked(cuda_device):
+    """The chunked per-channel path needs its own (larger) workspace."""
+    import gated_delta_rule_rda_b200 as rda
+    inp = rda_gen.fixed_inputs(1, 128, 2, 128, 128, dtype=torch.bfloat16, seed=335, channel=True).to("cuda")
+    small = rda.rda_prefill_workspace_bytes(1, 128, 2, 128, 128, 0)
+    assert rda.rda_prefill_channel_workspace_bytes(1, 128, 2, 128, 128, 0) > small
+    with pytest.raises(RuntimeError, match="RDA_ERR_WORKSPACE"):
+        rda.rda_prefill_chunked(inp.q, inp.k, inp.v, inp.log_alpha, inp.beta,
+                                workspace=rda.new_workspace(small, "cuda"))
 
 
 @pytest.mark.parametrize("dtype", [torch.float32, torch.bfloat16])
