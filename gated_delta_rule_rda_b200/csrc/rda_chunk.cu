@@ -649,11 +649,21 @@ prep_kernel(const __grid_constant__ PrepMaps maps, const PrefillArgs a) {
     float *g_s = reinterpret_cast<float *>(sm + PS_G);
     const float *b_s = g_s + 64, *bg_s = g_s + 128, *eg_s = g_s + 256;
 
+    const int r0 = (int)row0;
     if (threadIdx.x == 0) {
         for (int i = 0; i < kPrepBars; ++i) mbar_init(&bars[i], 1);
         *abort_flag = 0;
         *agent_flag = 0;
         fence_mbar_init();
+        fence_proxy_async_smem();
+        // K and Q before the rest of the setup (their latency heads the chunk's
+        // chain); V once the solve has freed A's region (the load overlaps the
+        // T images, W and its extraction)
+        mbar_arrive_expect_tx(&bars[PB_FULL], 32768);
+        tma_load_3d(sm + PS_K, &maps.k, &bars[PB_FULL], 0, h, r0);
+        tma_load_3d(sm + PS_K + 8192, &maps.k, &bars[PB_FULL], 64, h, r0);
+        tma_load_3d(sm + PS_Q, &maps.q, &bars[PB_FULL], 0, h, r0);
+        tma_load_3d(sm + PS_Q + 8192, &maps.q, &bars[PB_FULL], 64, h, r0);
     }
     if (warp == 0) {
         tmem_alloc(tmem_ptr, kPrepTmemCols);
@@ -667,14 +677,6 @@ prep_kernel(const __grid_constant__ PrepMaps maps, const PrefillArgs a) {
 
     if (warp == 0) {
         if (lane == 0) {
-            // K and Q now; V once the solve has freed A's region (the load overlaps
-            // the T images, W and its extraction)
-            const int r0 = (int)row0;
-            mbar_arrive_expect_tx(&bars[PB_FULL], 32768);
-            tma_load_3d(sm + PS_K, &maps.k, &bars[PB_FULL], 0, h, r0);
-            tma_load_3d(sm + PS_K + 8192, &maps.k, &bars[PB_FULL], 64, h, r0);
-            tma_load_3d(sm + PS_Q, &maps.q, &bars[PB_FULL], 0, h, r0);
-            tma_load_3d(sm + PS_Q + 8192, &maps.q, &bars[PB_FULL], 64, h, r0);
             bool v_issued = false;
             const uint32_t kk_ = smem_u32(sm + PS_K), qq = smem_u32(sm + PS_Q), vv = smem_u32(sm + PS_V);
             const uint32_t tbg = smem_u32(sm + PS_TBG), tb = smem_u32(sm + PS_TB);
