@@ -236,15 +236,6 @@ constexpr uint32_t kTcStateBytes = kTcD * kTcRow * 4;
 constexpr uint32_t kTcRawBytes = 3 * kMaxT * kTcD * 4;                    // k, q, v rows (fp32 at most)
 constexpr uint32_t kTcSmem = kTcStateBytes + kTcRawBytes + 3 * kMaxT * 4; // + the gates
 
-__device__ __forceinline__ void cp_async16(uint32_t dst, const void *src) {
-    asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(dst), "l"(src) : "memory");
-}
-__device__ __forceinline__ void cp_async4(uint32_t dst, const void *src) {
-    asm volatile("cp.async.ca.shared.global [%0], [%1], 4;" ::"r"(dst), "l"(src) : "memory");
-}
-__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
-__device__ __forceinline__ void cp_async_wait_all() { asm volatile("cp.async.wait_group 0;" ::: "memory"); }
-
 // Everything unit bh needs, copied into shared memory: its state (4,096
 // 16-byte pieces into the padded buffer), the raw rows of its T keys, queries
 // and values, and its gates (log alpha, beta, gamma).

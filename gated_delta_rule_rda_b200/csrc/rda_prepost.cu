@@ -21,6 +21,8 @@
 // Both are bound by HBM: each token-head is read and written once.
 #include <cuda_bf16.h>
 
+#include <mutex>
+
 #include "rda_internal.h"
 #include "rda_io.cuh"
 
@@ -28,7 +30,6 @@ namespace rda {
 namespace {
 
 constexpr int kTok = 64;          // tokens per pre-kernel CTA (one sequence)
-constexpr int kGrp = 2;           // tokens per step of the rolled token loop
 
 __device__ __forceinline__ float sigmoid_f(float x) { return __frcp_rn(1.f + __expf(-x)); }
 // Hardware tanh (PTX tanh.approx.f32, relative error about 2^-11).
@@ -146,19 +147,48 @@ template <int ACT, bool FAST> __device__ __forceinline__ float2 act2(float2 x) {
     }
 }
 
-// One tensor (q, k or v) of one head over one tile of a sequence, by one warp:
-// 2 NP channels per lane; `norm`: L2-normalise each token over the head (q, k).
-// q, k and v share this one code path (kept small for the instruction cache).
+// One CTA per (head, 64-token tile of a sequence): the tile's raw q, k and v
+// rows of this head, with the two rows before it (the conv's history), go to
+// shared memory first, all as 16-byte asynchronous copies issued up front
+// (~50 KiB in flight per CTA for bf16 at D = 128, four CTAs per SM), then six
+// warps compute from there: warps 2i and 2i+1 own tensor i (q, k, v) for the
+// tile's first and second 32 tokens; a lane owns 2 NP channels of a token row.
+constexpr int kRowsT = kTok + 2;      // tile rows in shared memory: positions p0 - 2 .. p0 + 63
+constexpr int kPrepWarps = 6;
+constexpr int kTokW = kTok / 2;       // tokens per warp
+constexpr int kUnroll = 4;            // tokens per step of a warp's loop (independent reductions)
+
+template <typename Tio, int DK, int DV>
+struct PrepSmem {
+    static constexpr uint32_t Q = 0;
+    static constexpr uint32_t K = Q + kRowsT * DK * sizeof(Tio);
+    static constexpr uint32_t V = K + kRowsT * DK * sizeof(Tio);
+    static constexpr uint32_t BYTES = V + kRowsT * DV * sizeof(Tio);
+};
+
+// Tile rows [r_lo, r_hi) of head h of one tensor [rows, H, D] (tile row r =
+// tensor row base_row + r) into shared memory, 16 bytes per copy.
+template <typename Tio, int D>
+__device__ __forceinline__ void issue_rows(uint32_t dst, const Tio *raw, int H, int h, long base_row, int r_lo,
+                                           int r_hi) {
+    constexpr int CPR = D * (int)sizeof(Tio) / 16;         // copies per row
+    const int n = (r_hi - r_lo) * CPR;
+    for (int e = threadIdx.x; e < n; e += kPrepWarps * 32) {
+        const int r = r_lo + e / CPR, c = e % CPR;
+        cp_async16(dst + (uint32_t)(r * D * sizeof(Tio) + c * 16),
+                   reinterpret_cast<const char *>(raw + ((size_t)(base_row + r) * H + h) * D) + c * 16);
+    }
+}
+
+// One warp's tokens [i0, i1) of one tensor: y_t = act(w0 x_{t-2} + w1 x_{t-1} +
+// w2 x_t) from the rows in shared memory (row i + 2 holds x at tile position i),
+// L2-normalised over the head for q and k, stored to the core's input.
 template <typename Tio, int NP, int ACT>
-__device__ __forceinline__ void conv_tile(const Tio *raw, Tio *out, const float *w, const PrepArgs &a, int n, int h,
-                                          int tile, long t0, long len, long p0, int pend, int coff, int lane,
-                                          bool norm) {
+__device__ __forceinline__ void conv_rows(const Tio *rows, Tio *dst, size_t stride, const float *w, int ch0,
+                                          int i0, int i1, int lane, bool norm) {
     constexpr int NC = 2 * NP;
     constexpr int D = 32 * NC;
     constexpr bool FAST = sizeof(Tio) == 2;
-    const int H = a.H;
-    const int ch0 = h * D + lane * NC;                     // channel within the tensor
-    const size_t stride = (size_t)H * D;                   // elements between tokens
     float2 w0[NP], w1[NP], w2[NP];
 #pragma unroll
     for (int j = 0; j < NP; ++j) {
@@ -167,107 +197,55 @@ __device__ __forceinline__ void conv_tile(const Tio *raw, Tio *out, const float 
         w1[j] = make_float2(wj[1], wj[4]);
         w2[j] = make_float2(wj[2], wj[5]);
     }
-    const Tio *in = raw + (size_t)(t0 + p0) * stride + ch0;
-    Tio *dst = out + (size_t)(t0 + p0) * stride + ch0;
-    // window rows (positions -3, -2, -1 of the sequence), or zeros; tile 0 only
-    float2 win[3][NP];
-#pragma unroll
-    for (int r = 0; r < 3; ++r)
-#pragma unroll
-        for (int j = 0; j < NP; ++j) {
-            win[r][j] = make_float2(0.f, 0.f);
-            if (tile == 0 && a.win_in) {
-                const __nv_bfloat16 *pw = a.win_in + ((size_t)n * 3 + r) * a.C + coff + ch0 + 2 * j;
-                win[r][j] = make_float2(__bfloat162float(pw[0]), __bfloat162float(pw[1]));
-            }
-        }
-    // the two inputs before the tile's first token
+    const Tio *src = rows + lane * NC;
     float2 xm2[NP], xm1[NP];
-    if (p0 >= 2) {
-        Pairs<Tio, NP>::ld(in - 2 * stride, xm2);
-        Pairs<Tio, NP>::ld(in - stride, xm1);
-    } else {
+    Pairs<Tio, NP>::ld(src + (size_t)i0 * D, xm2);
+    Pairs<Tio, NP>::ld(src + (size_t)(i0 + 1) * D, xm1);
+#pragma unroll 1
+    for (int i = i0; i < i1; i += kUnroll) {
+        float2 x[kUnroll][NP], y[kUnroll][NP];
+        float ss[kUnroll];
 #pragma unroll
-        for (int j = 0; j < NP; ++j) {
-            xm2[j] = win[1][j];
-            xm1[j] = win[2][j];
-        }
-    }
-    auto load_grp = [&](int g0, float2 (&x)[kGrp][NP]) {
+        for (int u = 0; u < kUnroll; ++u) Pairs<Tio, NP>::ld(src + (size_t)(i + u + 2) * D, x[u]);
 #pragma unroll
-        for (int i = 0; i < kGrp; ++i) {
-            if (g0 + i < pend) Pairs<Tio, NP>::ld(in + (size_t)(g0 + i) * stride, x[i]);
-            else {
-#pragma unroll
-                for (int j = 0; j < NP; ++j) x[i][j] = make_float2(0.f, 0.f);
-            }
-        }
-    };
-    auto run_grp = [&](int g0, const float2 (&x)[kGrp][NP]) {
-#pragma unroll
-        for (int i = 0; i < kGrp; ++i) {
-            float2 y[NP], ss2 = make_float2(0.f, 0.f);
+        for (int u = 0; u < kUnroll; ++u) {
+            float2 s2 = make_float2(0.f, 0.f);
 #pragma unroll
             for (int j = 0; j < NP; ++j) {
-                float2 t = __fmul2_rn(w2[j], x[i][j]);
+                float2 t = __fmul2_rn(w2[j], x[u][j]);
                 t = __ffma2_rn(w1[j], xm1[j], t);
                 t = __ffma2_rn(w0[j], xm2[j], t);
-                y[j] = act2<ACT, FAST>(t);
-                ss2 = __ffma2_rn(y[j], y[j], ss2);
+                y[u][j] = act2<ACT, FAST>(t);
+                s2 = __ffma2_rn(y[u][j], y[u][j], s2);
                 xm2[j] = xm1[j];
-                xm1[j] = x[i][j];
+                xm1[j] = x[u][j];
             }
-            if (norm) {
-                const float r = rsqrtf(warp_sum(ss2.x + ss2.y));
-#pragma unroll
-                for (int j = 0; j < NP; ++j) y[j] = __fmul2_rn(y[j], make_float2(r, r));
-            }
-            if (g0 + i < pend) Pairs<Tio, NP>::st(dst + (size_t)(g0 + i) * stride, y);
+            ss[u] = s2.x + s2.y;
         }
-    };
-    // a rolled loop over pairs of token groups (a small body the instruction
-    // cache keeps); each group's loads go out while the previous one computes
-    float2 xa[kGrp][NP], xb[kGrp][NP];
-    load_grp(0, xa);
-#pragma unroll 1
-    for (int g0 = 0; g0 < pend; g0 += 2 * kGrp) {
-        load_grp(g0 + kGrp, xb);
-        run_grp(g0, xa);
-        if (g0 + kGrp >= pend) break;
-        load_grp(g0 + 2 * kGrp, xa);
-        run_grp(g0 + kGrp, xb);
-    }
-    // the new window: the last three raw inputs of the sequence (shifting the old
-    // window for sequences shorter than three); written by the first tile only,
-    // after its own reads of the old window
-    if (tile == 0 && a.win_out) {
-        const Tio *seq = raw + (size_t)t0 * stride + ch0;
+        if (norm) {
 #pragma unroll
-        for (int r = 0; r < 3; ++r) {
-            const long p = len - 3 + r;
-            float2 v[NP];
-            if (p >= 0) {
-                Pairs<Tio, NP>::ld(seq + (size_t)p * stride, v);
-            } else {
-                const long src = len + r;           // 0 .. 2: a row of the old window
+            for (int off = 16; off > 0; off >>= 1)
 #pragma unroll
-                for (int j = 0; j < NP; ++j) v[j] = src == 0 ? win[0][j] : (src == 1 ? win[1][j] : win[2][j]);
-            }
+                for (int u = 0; u < kUnroll; ++u) ss[u] += __shfl_xor_sync(0xffffffffu, ss[u], off);
 #pragma unroll
-            for (int j = 0; j < NP; ++j) {
-                __nv_bfloat16 *pw = a.win_out + ((size_t)n * 3 + r) * a.C + coff + ch0 + 2 * j;
-                pw[0] = __float2bfloat16_rn(v[j].x);
-                pw[1] = __float2bfloat16_rn(v[j].y);
+            for (int u = 0; u < kUnroll; ++u) {
+                const float r = rsqrtf(ss[u]);
+#pragma unroll
+                for (int j = 0; j < NP; ++j) y[u][j] = __fmul2_rn(y[u][j], make_float2(r, r));
             }
         }
+#pragma unroll
+        for (int u = 0; u < kUnroll; ++u)
+            if (i + u < i1) Pairs<Tio, NP>::st(dst + (size_t)(i + u) * stride + lane * NC, y[u]);
     }
 }
 
 // grid (H, tiles of the longest sequence, sequences): the CTAs of one tile of
-// all heads run side by side and read whole token rows; warps 0, 1, 2 own q,
-// k, v.
-template <typename Tio, int NCK, int NCV, int ACT>
-__global__ void __launch_bounds__(96) prep_inputs_kernel(PrepArgs a) {
+// all heads run side by side and read whole token rows.
+template <typename Tio, int DK, int DV, int ACT>
+__global__ void __launch_bounds__(kPrepWarps * 32, sizeof(Tio) == 2 ? 4 : 2) prep_inputs_kernel(PrepArgs a) {
+    using L = PrepSmem<Tio, DK, DV>;
+    extern __shared__ __align__(16) uint8_t psm[];
     const int n = blockIdx.z, h = blockIdx.x, tile = blockIdx.y;
     long t0, len;
     if (a.cu_seqlens) {
@@ -282,16 +260,30 @@ __global__ void __launch_bounds__(96) prep_inputs_kernel(PrepArgs a) {
     const int pend = (int)min((long)kTok, len - p0);
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int H = a.H;
-    const int coff = warp == 0 ? 0 : (warp == 1 ? H * a.Dk : 2 * H * a.Dk);
-    const Tio *raw = static_cast<const Tio *>(warp == 0 ? a.raw[0] : (warp == 1 ? a.raw[1] : a.raw[2]));
-    Tio *out = static_cast<Tio *>(warp == 0 ? a.out[0] : (warp == 1 ? a.out[1] : a.out[2]));
-    const float *w = warp == 0 ? a.w[0] : (warp == 1 ? a.w[1] : a.w[2]);
-    if (NCK == NCV || warp < 2)
-        conv_tile<Tio, NCK / 2, ACT>(raw, out, w, a, n, h, tile, t0, len, p0, pend, coff, lane, warp < 2);
-    else
-        conv_tile<Tio, NCV / 2, ACT>(raw, out, w, a, n, h, tile, t0, len, p0, pend, coff, lane, false);
-
-    // ---- gates of the tile's tokens
+    const uint32_t sb = static_cast<uint32_t>(__cvta_generic_to_shared(psm));
+    const long base_row = t0 + p0 - 2;                      // sequence row of tile row 0
+    // ---- the tile's rows: history rows from the sequence, or (first tile) from the window
+    const int r_lo = tile == 0 ? 2 : 0;
+    issue_rows<Tio, DK>(sb + L::Q, static_cast<const Tio *>(a.raw[0]), H, h, base_row, r_lo, pend + 2);
+    issue_rows<Tio, DK>(sb + L::K, static_cast<const Tio *>(a.raw[1]), H, h, base_row, r_lo, pend + 2);
+    issue_rows<Tio, DV>(sb + L::V, static_cast<const Tio *>(a.raw[2]), H, h, base_row, r_lo, pend + 2);
+    cp_async_commit();
+    if (tile == 0) {
+        // positions -2 and -1: rows 1 and 2 of the carried window (oldest first), or zeros
+        constexpr int CQ = DK, CV = DV;
+        for (int e = threadIdx.x; e < 2 * (2 * CQ + CV); e += kPrepWarps * 32) {
+            const int r = e / (2 * CQ + CV), c = e % (2 * CQ + CV);
+            const int ti = c < CQ ? 0 : (c < 2 * CQ ? 1 : 2);
+            const int d = ti == 0 ? c : (ti == 1 ? c - CQ : c - 2 * CQ);
+            const int D = ti == 2 ? DV : DK;
+            const int coff = ti == 0 ? 0 : (ti == 1 ? H * DK : 2 * H * DK);
+            float x = 0.f;
+            if (a.win_in) x = __bfloat162float(a.win_in[((size_t)n * 3 + r + 1) * a.C + coff + h * D + d]);
+            Tio *rowp = reinterpret_cast<Tio *>(psm + (ti == 0 ? L::Q : (ti == 1 ? L::K : L::V)));
+            Io<Tio>::st(rowp + r * D + d, x);
+        }
+    }
+    // ---- the gates of the tile's tokens (their loads overlap the copies in flight)
     for (int i = threadIdx.x; i < pend; i += blockDim.x) {
         const size_t row = (size_t)(t0 + p0 + i) * H + h;
         const float br = a.beta_raw[row];
@@ -301,9 +293,50 @@ __global__ void __launch_bounds__(96) prep_inputs_kernel(PrepArgs a) {
         if (!a.channel) a.log_alpha[row] = fminf(fmaxf(a.la_raw[row], -5.f), 0.f);
     }
     if (a.channel) {
-        for (int i = threadIdx.x; i < pend * a.Dk; i += blockDim.x) {
-            const size_t e = ((size_t)(t0 + p0 + i / a.Dk) * H + h) * a.Dk + i % a.Dk;
+        for (int i = threadIdx.x; i < pend * DK; i += blockDim.x) {
+            const size_t e = ((size_t)(t0 + p0 + i / DK) * H + h) * DK + i % DK;
             a.log_alpha[e] = fminf(fmaxf(a.la_raw[e], -5.f), 0.f);
+        }
+    }
+    cp_async_wait_all();
+    __syncthreads();
+    // ---- q, k, v of the tile
+    const int ti = warp >> 1;
+    const int i0 = (warp & 1) * kTokW, i1 = min(i0 + kTokW, pend);
+    if (i0 < i1) {
+        const size_t row0 = (size_t)(t0 + p0) * H + h;
+        if (ti < 2) {
+            const Tio *rows = reinterpret_cast<const Tio *>(psm + (ti == 0 ? L::Q : L::K));
+            Tio *dst = static_cast<Tio *>(a.out[ti]) + row0 * DK;
+            conv_rows<Tio, DK / 64, ACT>(rows, dst, (size_t)H * DK, a.w[ti], h * DK + lane * (DK / 32), i0, i1,
+                                         lane, true);
+        } else {
+            const Tio *rows = reinterpret_cast<const Tio *>(psm + L::V);
+            Tio *dst = static_cast<Tio *>(a.out[2]) + row0 * DV;
+            conv_rows<Tio, DV / 64, ACT>(rows, dst, (size_t)H * DV, a.w[2], h * DV + lane * (DV / 32), i0, i1,
+                                         lane, false);
+        }
+    }
+    // ---- the new window: the last three raw inputs of the sequence (shifting the
+    // old window for sequences shorter than three); written by the first tile only,
+    // after its own reads of the old window (the barrier above)
+    if (tile == 0 && a.win_out) {
+        const int CH = 2 * DK + DV;
+        for (int e = threadIdx.x; e < 3 * CH; e += blockDim.x) {
+            const int r = e / CH, c = e % CH;
+            const int ti2 = c < DK ? 0 : (c < 2 * DK ? 1 : 2);
+            const int d = ti2 == 0 ? c : (ti2 == 1 ? c - DK : c - 2 * DK);
+            const int D = ti2 == 2 ? DV : DK;
+            const int coff = ti2 == 0 ? 0 : (ti2 == 1 ? H * DK : 2 * H * DK);
+            const long p = len - 3 + r;
+            float x;
+            if (p >= 0) {
+                x = Io<Tio>::ld(static_cast<const Tio *>(a.raw[ti2]) + ((size_t)(t0 + p) * H + h) * D + d);
+            } else {
+                const long src = len + r;           // 0 .. 2: a row of the old window
+                x = a.win_in ? __bfloat162float(a.win_in[((size_t)n * 3 + src) * a.C + coff + h * D + d]) : 0.f;
+            }
+            a.win_out[((size_t)n * 3 + r) * a.C + coff + h * D + d] = __float2bfloat16_rn(x);
         }
     }
 }
@@ -351,6 +384,19 @@ __global__ void __launch_bounds__(256) output_gate_norm_kernel(PostArgs a) {
     }
 }
 
+template <typename T, int DK, int DV, int ACT>
+cudaError_t launch_prep(dim3 grid, uint32_t smem, const PrepArgs &a, cudaStream_t s) {
+    static std::once_flag once;
+    static cudaError_t attr = cudaSuccess;
+    std::call_once(once, [smem] {
+        attr = cudaFuncSetAttribute(prep_inputs_kernel<T, DK, DV, ACT>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                    (int)smem);
+    });
+    if (attr != cudaSuccess) return attr;
+    prep_inputs_kernel<T, DK, DV, ACT><<<grid, kPrepWarps * 32, smem, s>>>(a);
+    return cudaSuccess;
+}
+
 }  // namespace
 
 cudaError_t launch_prep_inputs(const PrepLaunch &l, cudaStream_t s) {
@@ -371,17 +417,19 @@ cudaError_t launch_prep_inputs(const PrepLaunch &l, cudaStream_t s) {
     const long tiles = (l.max_seqlen + kTok - 1) / kTok;
     const dim3 grid(l.H, (unsigned)(tiles > 0 ? tiles : 1), l.num_seqs);
     const bool f32 = l.dtype == RDA_F32;
-#define RDA_PREP(T, NK, NV)                                                         \
-    do {                                                                            \
-        if (l.act == RDA_ACT_SILU) prep_inputs_kernel<T, NK, NV, RDA_ACT_SILU><<<grid, 96, 0, s>>>(a); \
-        else prep_inputs_kernel<T, NK, NV, RDA_ACT_NONE><<<grid, 96, 0, s>>>(a);   \
+    cudaError_t e = cudaSuccess;
+#define RDA_PREP(T, DK, DV)                                                                     \
+    do {                                                                                        \
+        constexpr uint32_t smem = PrepSmem<T, DK, DV>::BYTES;                                   \
+        if (l.act == RDA_ACT_SILU) e = launch_prep<T, DK, DV, RDA_ACT_SILU>(grid, smem, a, s);   \
+        else e = launch_prep<T, DK, DV, RDA_ACT_NONE>(grid, smem, a, s);                         \
     } while (0)
-    if (l.Dk == 128 && l.Dv == 128) { if (f32) RDA_PREP(float, 4, 4); else RDA_PREP(__nv_bfloat16, 4, 4); }
-    else if (l.Dk == 128) { if (f32) RDA_PREP(float, 4, 2); else RDA_PREP(__nv_bfloat16, 4, 2); }
-    else if (l.Dv == 128) { if (f32) RDA_PREP(float, 2, 4); else RDA_PREP(__nv_bfloat16, 2, 4); }
-    else { if (f32) RDA_PREP(float, 2, 2); else RDA_PREP(__nv_bfloat16, 2, 2); }
+    if (l.Dk == 128 && l.Dv == 128) { if (f32) RDA_PREP(float, 128, 128); else RDA_PREP(__nv_bfloat16, 128, 128); }
+    else if (l.Dk == 128) { if (f32) RDA_PREP(float, 128, 64); else RDA_PREP(__nv_bfloat16, 128, 64); }
+    else if (l.Dv == 128) { if (f32) RDA_PREP(float, 64, 128); else RDA_PREP(__nv_bfloat16, 64, 128); }
+    else { if (f32) RDA_PREP(float, 64, 64); else RDA_PREP(__nv_bfloat16, 64, 64); }
 #undef RDA_PREP
-    return cudaGetLastError();
+    return e != cudaSuccess ? e : cudaGetLastError();
 }
 
 cudaError_t launch_output_gate_norm(const void *o, const void *g, const float *w, void *out, long rows, int Dv,
