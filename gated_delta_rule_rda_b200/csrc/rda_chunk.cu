@@ -464,14 +464,16 @@ __device__ __forceinline__ void gram_rows(uint32_t taddr, int ta, int lane, cons
 // With one decay per key dim, the chunk's Gram entries are
 //     X[t] . (K[s] o e^{G[t] - G[s]})   (X = K for A, Q for P),
 // not a plain product times a mask.  Split the factor around a reference token
-// r of the column block, e^{G[t] - G[r]} on the row operand and e^{G[r] - G[s]}
-// on the column operand, and each 16 x 16 block is an ordinary product of
-// scaled operands.  References: for an off-diagonal block the last token of the
-// column block (both factors <= 1), for a diagonal block its first token (row
-// factors <= 1, column factors at most e^{15 x 5}, well inside the range of
-// bf16 and fp32).  A factor that underflows belongs to an entry far below
-// every other one in the row.  The operands are scaled in fp32 and rounded to
-// bf16 in the MMA fragments (mma.sync m16n8k16, fp32 accumulation).
+// r, e^{G[t] - G[r]} on the row operand and e^{G[r] - G[s]} on the column
+// operand, and each 16 x 16 block is an ordinary product of scaled operands.
+// The reference of every block of a row block is that row block's first token
+// 16 rb: row factors <= 1; column factors <= 1 off the diagonal (s < r) and at
+// most e^{15 x 5} on it (well inside the range of bf16 and fp32).  A factor
+// that underflows belongs to an entry far below every other one in the row.
+// So a row block's K and Q row operands serve all its blocks, and each column
+// operand serves both the A and the P block of a pair.  The operands are scaled
+// in fp32 and rounded to bf16 in the MMA fragments (mma.sync m16n8k16, fp32
+// accumulation).
 // ---------------------------------------------------------------------------
 __device__ __forceinline__ void mma16816_g(float *d, const uint32_t *a, uint32_t b0, uint32_t b1) {
     asm volatile(
@@ -492,26 +494,36 @@ __device__ __forceinline__ uint32_t scaled_pair(const uint8_t *tile, const float
     const float2 gr = *reinterpret_cast<const float2 *>(Gm + ref * kGld + d);
     return pack_bf16(x.x * __expf(sgn * (gt.x - gr.x)), x.y * __expf(sgn * (gt.y - gr.y)));
 }
-// acc[nt] (n-tiles of 8 columns) += the 16 x 16 block (rows 16 rb.., columns
-// 16 cb..) of sum_d X[t][d] K[s][d] e^{G[t][d] - G[s][d]}, split around `ref`.
-__device__ __forceinline__ void gram_block_ch(const uint8_t *xt, const uint8_t *kt, const float *Gm, int rb, int cb,
-                                              int ref, int lane, float (&acc)[2][4]) {
+// Row block rb of the decayed Grams, by one warp: accK[cb] (A, before beta and
+// the mask) and accQ[cb] (P, before the mask) for the column blocks cb <= rb,
+// n-tiles of 8 columns, mma.sync accumulator layout.
+__device__ __forceinline__ void gram_rowblock_ch(const uint8_t *kt, const uint8_t *qt, const float *Gm, int rb,
+                                                 int lane, float (&accK)[4][2][4], float (&accQ)[4][2][4]) {
     const int g = lane >> 2, tg = lane & 3;
-    const int t0 = 16 * rb + g, t1 = t0 + 8;
-#pragma unroll 2
+    const int t0 = 16 * rb + g, t1 = t0 + 8, ref = 16 * rb;
+#pragma unroll 1
     for (int ks = 0; ks < 8; ++ks) {
         const int d = 16 * ks + 2 * tg;
-        uint32_t af[4];
-        af[0] = scaled_pair(xt, Gm, t0, d, ref, 1.f);
-        af[1] = scaled_pair(xt, Gm, t1, d, ref, 1.f);
-        af[2] = scaled_pair(xt, Gm, t0, d + 8, ref, 1.f);
-        af[3] = scaled_pair(xt, Gm, t1, d + 8, ref, 1.f);
+        uint32_t ak[4], aq[4];
+        ak[0] = scaled_pair(kt, Gm, t0, d, ref, 1.f);
+        ak[1] = scaled_pair(kt, Gm, t1, d, ref, 1.f);
+        ak[2] = scaled_pair(kt, Gm, t0, d + 8, ref, 1.f);
+        ak[3] = scaled_pair(kt, Gm, t1, d + 8, ref, 1.f);
+        aq[0] = scaled_pair(qt, Gm, t0, d, ref, 1.f);
+        aq[1] = scaled_pair(qt, Gm, t1, d, ref, 1.f);
+        aq[2] = scaled_pair(qt, Gm, t0, d + 8, ref, 1.f);
+        aq[3] = scaled_pair(qt, Gm, t1, d + 8, ref, 1.f);
 #pragma unroll
-        for (int nt = 0; nt < 2; ++nt) {
-            const int sc = 16 * cb + 8 * nt + g;
-            const uint32_t b0 = scaled_pair(kt, Gm, sc, d, ref, -1.f);
-            const uint32_t b1 = scaled_pair(kt, Gm, sc, d + 8, ref, -1.f);
-            mma16816_g(acc[nt], af, b0, b1);
+        for (int cb = 0; cb < 4; ++cb) {
+            if (cb > rb) continue;
+#pragma unroll
+            for (int nt = 0; nt < 2; ++nt) {
+                const int sc = 16 * cb + 8 * nt + g;
+                const uint32_t b0 = scaled_pair(kt, Gm, sc, d, ref, -1.f);
+                const uint32_t b1 = scaled_pair(kt, Gm, sc, d + 8, ref, -1.f);
+                mma16816_g(accK[cb][nt], ak, b0, b1);
+                mma16816_g(accQ[cb][nt], aq, b0, b1);
+            }
         }
     }
 }
@@ -561,34 +573,34 @@ __device__ __forceinline__ void prep_channel_front(const PrefillArgs &a, uint8_t
     float *Af = reinterpret_cast<float *>(sm + PS_AF);
     const uint8_t *kt = sm + PS_K, *qt = sm + PS_Q;
     const int g = lane >> 2, tg = lane & 3;
-    for (int task = wq; go && task < 20; task += 4) {
-        const bool isP = task >= 10;
-        int idx = isP ? task - 10 : task, rb = 0;            // block pairs (rb, cb), cb <= rb, in order
-        while (idx > rb) {
-            idx -= rb + 1;
-            ++rb;
-        }
-        const int cb = idx;
-        const int ref = rb == cb ? 16 * cb : 16 * cb + 15;
-        float acc[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
-        gram_block_ch(isP ? qt : kt, kt, Gm, rb, cb, ref, lane, acc);
+    if (go) {
+        // warp wq owns row block 3 - wq: the largest first
+        const int rb = 3 - wq;
+        float accK[4][2][4], accQ[4][2][4];
 #pragma unroll
-        for (int nt = 0; nt < 2; ++nt)
+        for (int cb = 0; cb < 4; ++cb)
 #pragma unroll
-            for (int hh = 0; hh < 2; ++hh) {
-                const int t = 16 * rb + g + 8 * hh, s0 = 16 * cb + 8 * nt + 2 * tg;
-                float v0 = acc[nt][2 * hh], v1 = acc[nt][2 * hh + 1];
-                if (isP) {
-                    v0 = s0 <= t ? v0 : 0.f;
-                    v1 = s0 + 1 <= t ? v1 : 0.f;
-                    *reinterpret_cast<uint32_t *>(img + kImgP + swz(t, s0 >> 3, 128) + (s0 & 7) * 2) =
-                        pack_bf16(v0, v1);
-                } else {
+            for (int nt = 0; nt < 2; ++nt)
+#pragma unroll
+                for (int i = 0; i < 4; ++i) accK[cb][nt][i] = accQ[cb][nt][i] = 0.f;
+        gram_rowblock_ch(kt, qt, Gm, rb, lane, accK, accQ);
+#pragma unroll
+        for (int cb = 0; cb < 4; ++cb) {
+            if (cb > rb) continue;
+#pragma unroll
+            for (int nt = 0; nt < 2; ++nt)
+#pragma unroll
+                for (int hh = 0; hh < 2; ++hh) {
+                    const int t = 16 * rb + g + 8 * hh, s0 = 16 * cb + 8 * nt + 2 * tg;
+                    const float k0 = accK[cb][nt][2 * hh], k1 = accK[cb][nt][2 * hh + 1];
+                    const float q0 = accQ[cb][nt][2 * hh], q1 = accQ[cb][nt][2 * hh + 1];
                     const float be = b_s[t];
                     *reinterpret_cast<float2 *>(Af + t * kLd + s0) =
-                        make_float2(s0 < t ? be * v0 : 0.f, s0 + 1 < t ? be * v1 : 0.f);
+                        make_float2(s0 < t ? be * k0 : 0.f, s0 + 1 < t ? be * k1 : 0.f);
+                    *reinterpret_cast<uint32_t *>(img + kImgP + swz(t, s0 >> 3, 128) + (s0 & 7) * 2) =
+                        pack_bf16(s0 <= t ? q0 : 0.f, s0 + 1 <= t ? q1 : 0.f);
                 }
-            }
+        }
     }
     // the blocks of P's image above the diagonal are zero (the scan multiplies by all 64 columns)
     for (int i = cw; go && i < 6 * 16 * 8; i += 128) {
