@@ -637,16 +637,18 @@ def profile_decode_tokens(T, steps, warmup):
     print(json.dumps({"decode_tokens_T": T, "ms_per_call": s.elapsed_time(e) / steps}), flush=True)
 
 
-def profile_prefill(steps, warmup):
-    """Only the nano prefill: `warmup` + `steps` eager calls, L2 flushed before
-    each (a short, self-contained run for a profiler)."""
+def profile_prefill(steps, warmup, workload=WORKLOAD):
+    """Only the nano prefill (or the per-key-channel one): `warmup` + `steps`
+    eager calls, L2 flushed before each (a short, self-contained run for a
+    profiler)."""
     import torch
     import gated_delta_rule_rda_b200 as rda
     import rda_gen
-    inp = rda_gen.workload(WORKLOAD).to("cuda")
+    inp = rda_gen.workload(workload).to("cuda")
     B, T, H, Dk = inp.q.shape
     Dv = inp.v.shape[-1]
-    ws = rda.new_workspace(rda.rda_prefill_workspace_bytes(B, T, H, Dk, Dv, 0), "cuda")
+    wb = rda.rda_prefill_channel_workspace_bytes if inp.log_alpha.dim() == 4 else rda.rda_prefill_workspace_bytes
+    ws = rda.new_workspace(wb(B, T, H, Dk, Dv, 0), "cuda")
     out = torch.empty_like(inp.v)
     sf = torch.empty(B, H, Dk, Dv, device="cuda")
     flush = torch.empty(256 << 20, dtype=torch.uint8, device="cuda")
@@ -690,6 +692,8 @@ def main():
                     help="also time the long-context and packed (varlen) prefill workloads")
     ap.add_argument("--profile-decode-tokens", type=int, default=0, metavar="T",
                     help="run only the multi-token decode with T tokens per call (for a profiler)")
+    ap.add_argument("--profile-prefill-channel", action="store_true",
+                    help="run only warmup + steps per-key-channel nano prefill calls, L2 flushed (for a profiler)")
     ap.add_argument("--profile-prefill", action="store_true",
                     help="run only warmup + steps nano prefill calls, L2 flushed (for a profiler)")
     ap.add_argument("--profile-prepost", action="store_true",
@@ -702,6 +706,9 @@ def main():
         return
     if args.profile_prefill:
         profile_prefill(args.steps, args.warmup)
+        return
+    if args.profile_prefill_channel:
+        profile_prefill(args.steps, args.warmup, "nano_prefill_channel_b1_t4096_h16_d128")
         return
     if args.profile_prepost:
         profile_prepost(args.steps, args.warmup)
