@@ -76,3 +76,27 @@ def test_varlen_scan_wait_runs_out(cuda_device):
     ro, rs = oracle.varlen(vin.q, vin.k, vin.v, vin.log_alpha, vin.beta, vin.cu_seqlens,
                            initial_states=vin.initial_states)
     assert rel_l2(out, ro) <= 1e-2 and rel_l2(sf, rs) <= 1e-2
+
+
+def test_channel_scan_wait_runs_out(cuda_device):
+    """The per-key-channel chunked prefill (its scan has the same bounded waits,
+    fed from the K~ and Q~ images): the stalled chunk records the timeout, the
+    chunks before it are stored, and the next normal call is correct."""
+    import oracle
+    import gated_delta_rule_rda_b200 as rda
+    inp = rda_gen.fixed_inputs(1, 320, 2, 128, 128, dtype=torch.bfloat16, seed=93, s0=True, channel=True)
+    ro, rs = oracle.forward(inp.q, inp.k, inp.v, inp.log_alpha, inp.beta, initial_state=inp.initial_state)
+    d = inp.to("cuda")
+    ws = rda.new_workspace(rda.rda_prefill_channel_workspace_bytes(1, 320, 2, 128, 128, 0), "cuda")
+    try:
+        rda.rda_debug_set_wait_fault(drop_chunk=2, wait_limit_ns=20_000_000)
+        out, _ = _call(rda, d, ws)
+        torch.cuda.synchronize()
+    finally:
+        rda.rda_debug_set_wait_fault()
+    assert rda.rda_read_device_error(ws) == RDA_ERR_TIMEOUT
+    assert rel_l2(to_np(out)[:, :128], ro[:, :128]) <= 1e-2
+    out2, sf2 = _call(rda, d, ws)
+    torch.cuda.synchronize()
+    assert rda.rda_read_device_error(ws) == 0
+    assert rel_l2(to_np(out2), ro) <= 1e-2 and rel_l2(to_np(sf2), rs) <= 1e-2

@@ -192,3 +192,26 @@ def test_channel_decode_continues_prefill(cuda_device):
     got = torch.stack(outs, 1)
     assert rel_l2(to_np(got), to_np(full_o[:, 100:])) <= 1e-5
     assert rel_l2(to_np(st), to_np(full_s)) <= 1e-5
+
+
+def test_channel_bf16_decode_continues_chunked_prefill(cuda_device):
+    """bf16, Dk = 128: the chunked per-channel prefill of T tokens, then 5
+    per-channel decode steps from its final state, equals the chunked prefill of
+    T + 5 tokens (the state the chunked path hands over is the rule's state)."""
+    import gated_delta_rule_rda_b200 as rda
+    inp = rda_gen.fixed_inputs(2, 135, 2, 128, 128, dtype=torch.bfloat16, seed=365, s0=True,
+                               gamma=True, channel=True).to("cuda")
+    full_o, full_s = rda.rda_prefill_chunked(inp.q, inp.k, inp.v, inp.log_alpha, inp.beta,
+                                             write_gate=inp.gamma, initial_state=inp.initial_state)
+    c = lambda t: t[:, :130].contiguous()
+    _, st = rda.rda_prefill_chunked(c(inp.q), c(inp.k), c(inp.v), c(inp.log_alpha), c(inp.beta),
+                                    write_gate=c(inp.gamma), initial_state=inp.initial_state)
+    outs = []
+    for t in range(130, 135):
+        s = lambda x: x[:, t].contiguous()
+        outs.append(rda.rda_decode_step(s(inp.q), s(inp.k), s(inp.v), s(inp.log_alpha), s(inp.beta), st,
+                                        write_gate=s(inp.gamma)))
+    torch.cuda.synchronize()
+    got = torch.stack(outs, 1)
+    assert rel_l2(to_np(got), to_np(full_o[:, 130:])) <= 1e-2
+    assert rel_l2(to_np(st), to_np(full_s)) <= 1e-2
