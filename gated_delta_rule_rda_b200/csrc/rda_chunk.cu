@@ -307,7 +307,8 @@ __device__ __forceinline__ void ut_solve(float *Af, float *Tf, float *Xs, int cw
 // Four CTAs share an SM (shared memory <= 55 KiB, 128 TMEM columns, <= 96
 // registers): three regions are reused as the chunk's work moves along.
 // ---------------------------------------------------------------------------
-constexpr int kPrepThreads = 160;     // warp 0 TMA + MMA issue, warps 1..4 compute
+constexpr int kPrepThreads = 160;     // warp 0: TMEM and the tile loads; warps 1..4 compute (one of
+                                      // their threads issues the MMAs and the V load)
 constexpr uint32_t kPrepTmemCols = 128;
 // shared memory (bytes from a 1024-aligned base)
 constexpr uint32_t PS_K = 0;           // K [64 x 128]: halves of 8 KiB (SW128); later the -W image
@@ -337,7 +338,7 @@ constexpr uint32_t kPrepSmemCh = PS_GCH + 64 * kGld * 4 + 1024;
 static_assert(2 * (kPrepSmemCh + 1024) <= 233472, "two per-channel prep CTAs per SM");
 // TMEM columns: K K^T and Q K^T side by side, then W, then U' (one at a time)
 constexpr uint32_t PT_KK = 0, PT_QK = 64, PT_W = 0, PT_U = 0;
-enum PrepBar { PB_FULL = 0, PB_VFULL, PB_KK, PB_QK, PB_TREADY, PB_W, PB_WFREE, PB_U, PB_DRAIN, kPrepBars };
+enum PrepBar { PB_FULL = 0, PB_VFULL, PB_KK, PB_QK, PB_W, PB_U, PB_DRAIN, kPrepBars };
 static_assert(kPrepBars <= 10, "barrier area");
 
 struct PrepMaps {
@@ -657,7 +658,6 @@ prep_kernel(const __grid_constant__ PrepMaps maps, const PrefillArgs a) {
     uint64_t *bars = reinterpret_cast<uint64_t *>(sm + PS_BAR);
     uint32_t *tmem_ptr = reinterpret_cast<uint32_t *>(sm + PS_TMEMPTR);
     volatile int *abort_flag = reinterpret_cast<volatile int *>(sm + PS_FLAGS);
-    volatile int *agent_flag = abort_flag + 1;
     float *g_s = reinterpret_cast<float *>(sm + PS_G);
     const float *b_s = g_s + 64, *bg_s = g_s + 128, *eg_s = g_s + 256;
 
@@ -665,7 +665,6 @@ prep_kernel(const __grid_constant__ PrepMaps maps, const PrefillArgs a) {
     if (threadIdx.x == 0) {
         for (int i = 0; i < kPrepBars; ++i) mbar_init(&bars[i], 1);
         *abort_flag = 0;
-        *agent_flag = 0;
         fence_mbar_init();
         fence_proxy_async_smem();
         // K and Q before the rest of the setup (their latency heads the chunk's
@@ -687,64 +686,10 @@ prep_kernel(const __grid_constant__ PrepMaps maps, const PrefillArgs a) {
     const uint32_t tmem = *tmem_ptr;
     uint8_t *img = a.workspace_chunks + ((size_t)gc * H + h) * a.chunk_bytes;
 
-    if (warp == 0) {
-        if (lane == 0) {
-            bool v_issued = false;
-            const uint32_t kk_ = smem_u32(sm + PS_K), qq = smem_u32(sm + PS_Q), vv = smem_u32(sm + PS_V);
-            const uint32_t tbg = smem_u32(sm + PS_TBG), tb = smem_u32(sm + PS_TB);
-            constexpr uint32_t ID_KK = idesc_bf16(64, 64, 0, 0);
-            constexpr uint32_t ID_W = idesc_bf16(64, 128, 0, 1);
-            const uint32_t ID_U = Dv == 128 ? idesc_bf16(64, 128, 0, 1) : idesc_bf16(64, 64, 0, 1);
-            bool ok = wait_bar2(&bars[PB_FULL], 0, abort_flag, agent_flag, a.err, a.wait_ns);
-            if (ok && CH) ok = wait_bar2(&bars[PB_TREADY], 0, abort_flag, agent_flag, a.err, a.wait_ns);
-            if (ok && !CH) {
-                tc_fence_after();
-#pragma unroll
-                for (int kk = 0; kk < 8; ++kk) {     // K K^T: A = B = the K tile (K-major)
-                    const uint32_t off = (kk >> 2) * 8192 + (kk & 3) * 32;
-                    mma_bf16(tmem + PT_KK, smem_desc(kk_ + off, 16, 1024, kSw128),
-                             smem_desc(kk_ + off, 16, 1024, kSw128), ID_KK, kk > 0);
-                }
-                mma_commit(&bars[PB_KK]);
-#pragma unroll
-                for (int kk = 0; kk < 8; ++kk) {     // Q K^T: A = the Q tile, B = the K tile (K-major)
-                    const uint32_t off = (kk >> 2) * 8192 + (kk & 3) * 32;
-                    mma_bf16(tmem + PT_QK, smem_desc(qq + off, 16, 1024, kSw128),
-                             smem_desc(kk_ + off, 16, 1024, kSw128), ID_KK, kk > 0);
-                }
-                mma_commit(&bars[PB_QK]);
-                ok = wait_bar2(&bars[PB_TREADY], 0, abort_flag, agent_flag, a.err, a.wait_ns);
-            }
-            if (ok) {
-                // the compute threads fenced their generic accesses to A's region
-                // before the barrier that preceded TREADY
-                mbar_arrive_expect_tx(&bars[PB_VFULL], 64 * Dv * 2);
-                tma_load_3d(sm + PS_V, &maps.v, &bars[PB_VFULL], 0, h, r0);
-                if (Dv == 128) tma_load_3d(sm + PS_V + 8192, &maps.v, &bars[PB_VFULL], 64, h, r0);
-                v_issued = true;
-                tc_fence_after();
-#pragma unroll
-                for (int kk = 0; kk < 4; ++kk)       // W = T diag(beta e^g) K  (B = K, MN-major)
-                    mma_bf16(tmem + PT_W, smem_desc(tbg + kk * 32, 16, 1024, kSw128),
-                             smem_desc(kk_ + kk * 2048, 8192, 1024, kSw128), ID_W, kk > 0);
-                mma_commit(&bars[PB_W]);
-                ok = wait_bar2(&bars[PB_WFREE], 0, abort_flag, agent_flag, a.err, a.wait_ns) &&
-                     wait_bar2(&bars[PB_VFULL], 0, abort_flag, agent_flag, a.err, a.wait_ns);
-            }
-            if (ok) {
-                tc_fence_after();
-#pragma unroll
-                for (int kk = 0; kk < 4; ++kk)       // U' = T diag(beta gamma) V  (B = V, MN-major)
-                    mma_bf16(tmem + PT_U, smem_desc(tb + kk * 32, 16, 1024, kSw128),
-                             smem_desc(vv + kk * 2048, 8192, 1024, kSw128), ID_U, kk > 0);
-                mma_commit(&bars[PB_U]);
-            }
-            mma_commit(&bars[PB_DRAIN]);      // every MMA issued has completed before TMEM is freed
-            drain_bar(&bars[PB_DRAIN], 0, a.wait_ns);
-            drain_bar(&bars[PB_FULL], 0, a.wait_ns);     // the CTA may not exit with copies in flight
-            if (v_issued) drain_bar(&bars[PB_VFULL], 0, a.wait_ns);
-        }
-    } else {
+    // Warp 0 allocated TMEM and (thread 0) issued the tile loads; compute thread 0
+    // issues the MMAs and the V load itself, where its warps' work makes them
+    // ready (no hand-off through another warp), and drains them at the end.
+    if (warp > 0) {
         const int cw = threadIdx.x - 32;
         // rows ta, ta + 8 and column pairs 8 kb + j2 of the M=64 accumulators (16x256b loads)
         const int ta = 16 * q4 + (lane >> 2), j2 = 2 * (lane & 3);
@@ -752,12 +697,36 @@ prep_kernel(const __grid_constant__ PrepMaps maps, const PrefillArgs a) {
         float *Af = reinterpret_cast<float *>(sm + PS_AF);
         float *Tf = reinterpret_cast<float *>(sm + PS_TF);
         float *Xs = reinterpret_cast<float *>(sm + PS_XS);
+        // MMA operands (shared-memory addresses) and instruction descriptors
+        const uint32_t kk_ = smem_u32(sm + PS_K), qq = smem_u32(sm + PS_Q), vv = smem_u32(sm + PS_V);
+        const uint32_t tbg = smem_u32(sm + PS_TBG), tb = smem_u32(sm + PS_TB);
+        constexpr uint32_t ID_KK = idesc_bf16(64, 64, 0, 0);
+        constexpr uint32_t ID_W = idesc_bf16(64, 128, 0, 1);
+        const uint32_t ID_U = Dv == 128 ? idesc_bf16(64, 128, 0, 1) : idesc_bf16(64, 64, 0, 1);
+        bool v_issued = false;           // compute thread 0's: copies and MMAs to drain
 
         if constexpr (CH) {
             prep_channel_front(a, sm, g_s, gates, cw, r, lenc, row0, h, img, bars, abort_flag);
         } else {
         chunk_gates(gates, r, lane, g_s);
-        if (cw == 0 && !wait_bar(&bars[PB_KK], 0, abort_flag, a.err, a.wait_ns)) *abort_flag = 1;
+        if (cw == 0 && wait_bar(&bars[PB_FULL], 0, abort_flag, a.err, a.wait_ns)) {
+            tc_fence_after();
+#pragma unroll
+            for (int kk = 0; kk < 8; ++kk) {     // K K^T: A = B = the K tile (K-major)
+                const uint32_t off = (kk >> 2) * 8192 + (kk & 3) * 32;
+                mma_bf16(tmem + PT_KK, smem_desc(kk_ + off, 16, 1024, kSw128),
+                         smem_desc(kk_ + off, 16, 1024, kSw128), ID_KK, kk > 0);
+            }
+            mma_commit(&bars[PB_KK]);
+#pragma unroll
+            for (int kk = 0; kk < 8; ++kk) {     // Q K^T: A = the Q tile, B = the K tile (K-major)
+                const uint32_t off = (kk >> 2) * 8192 + (kk & 3) * 32;
+                mma_bf16(tmem + PT_QK, smem_desc(qq + off, 16, 1024, kSw128),
+                         smem_desc(kk_ + off, 16, 1024, kSw128), ID_KK, kk > 0);
+            }
+            mma_commit(&bars[PB_QK]);
+            if (!wait_bar(&bars[PB_KK], 0, abort_flag, a.err, a.wait_ns)) *abort_flag = 1;
+        }
         named_bar_sync(1, 128);
         if (!*abort_flag) {
             tc_fence_after();
@@ -826,7 +795,18 @@ prep_kernel(const __grid_constant__ PrepMaps maps, const PrefillArgs a) {
         fence_proxy_async_smem();
         named_bar_sync(1, 128);
         if (cw == 0 && !*abort_flag) {
-            mbar_arrive(&bars[PB_TREADY]);
+            // V into A's region (dead since the solve; the fence above ordered the
+            // generic accesses to it), then W = T diag(beta e^g) K  (B = K, MN-major)
+            mbar_arrive_expect_tx(&bars[PB_VFULL], 64 * Dv * 2);
+            tma_load_3d(sm + PS_V, &maps.v, &bars[PB_VFULL], 0, h, r0);
+            if (Dv == 128) tma_load_3d(sm + PS_V + 8192, &maps.v, &bars[PB_VFULL], 64, h, r0);
+            v_issued = true;
+            tc_fence_after();
+#pragma unroll
+            for (int kk = 0; kk < 4; ++kk)
+                mma_bf16(tmem + PT_W, smem_desc(tbg + kk * 32, 16, 1024, kSw128),
+                         smem_desc(kk_ + kk * 2048, 8192, 1024, kSw128), ID_W, kk > 0);
+            mma_commit(&bars[PB_W]);
             if (!wait_bar(&bars[PB_W], 0, abort_flag, a.err, a.wait_ns)) *abort_flag = 1;
         }
         named_bar_sync(1, 128);
@@ -852,10 +832,18 @@ prep_kernel(const __grid_constant__ PrepMaps maps, const PrefillArgs a) {
         }
         named_bar_sync(1, 128);
         if (cw == 0 && !*abort_flag) {
-            mbar_arrive(&bars[PB_WFREE]);
             bulk_store(img + kImgW, sm + PS_WIMG, 16384);
             bulk_commit();
-            if (!wait_bar(&bars[PB_U], 0, abort_flag, a.err, a.wait_ns)) *abort_flag = 1;
+            // U' = T diag(beta gamma) V  (B = V, MN-major), into the columns W has left
+            if (wait_bar(&bars[PB_VFULL], 0, abort_flag, a.err, a.wait_ns)) {
+                tc_fence_after();
+#pragma unroll
+                for (int kk = 0; kk < 4; ++kk)
+                    mma_bf16(tmem + PT_U, smem_desc(tb + kk * 32, 16, 1024, kSw128),
+                             smem_desc(vv + kk * 2048, 8192, 1024, kSw128), ID_U, kk > 0);
+                mma_commit(&bars[PB_U]);
+                if (!wait_bar(&bars[PB_U], 0, abort_flag, a.err, a.wait_ns)) *abort_flag = 1;
+            }
         }
         named_bar_sync(1, 128);
         if (!*abort_flag) {
@@ -884,6 +872,11 @@ prep_kernel(const __grid_constant__ PrepMaps maps, const PrefillArgs a) {
                 bulk_commit();
             }
             bulk_wait_reads();
+            // the CTA may not exit (nor free TMEM) with copies or MMAs in flight
+            mma_commit(&bars[PB_DRAIN]);
+            drain_bar(&bars[PB_DRAIN], 0, a.wait_ns);
+            drain_bar(&bars[PB_FULL], 0, a.wait_ns);
+            if (v_issued) drain_bar(&bars[PB_VFULL], 0, a.wait_ns);
         }
     }
 
