@@ -229,25 +229,31 @@ __device__ __forceinline__ void mma_f32_split(float *acc, const float *a, uint32
 // Persistent form: each CTA loops over (sequence, head) units.  A unit's state
 // (64 KiB) is copied into shared memory with 16-byte asynchronous copies
 // (cp.async, completed by a hardware wait, no spin) and from there into the
-// registers; the copy of the CTA's next unit is issued as soon as the buffer is
-// free, so every SM always has state bytes in flight while it computes.
+// registers; the copy of the CTA's next unit is issued while the current one
+// computes, so every SM always has state bytes in flight.  The next unit's rows
+// and gates go out as soon as their buffer is free; its state by the 128
+// threads that the token recurrence leaves idle (4,096 copies issued at once
+// back up the load queue: ~3,200 cycles of a ~16,400-cycle unit when every
+// thread issued them in the chain).
 constexpr int kTcRow = kTcD + 4;    // padded smem row (528 B): conflict-free 8-byte fragment reads
 constexpr uint32_t kTcStateBytes = kTcD * kTcRow * 4;
 constexpr uint32_t kTcRawBytes = 3 * kMaxT * kTcD * 4;                    // k, q, v rows (fp32 at most)
 constexpr uint32_t kTcSmem = kTcStateBytes + kTcRawBytes + 3 * kMaxT * 4; // + the gates
 
-// Everything unit bh needs, copied into shared memory: its state (4,096
-// 16-byte pieces into the padded buffer), the raw rows of its T keys, queries
-// and values, and its gates (log alpha, beta, gamma).
-template <typename Tio>
-__device__ __forceinline__ void issue_unit_copy(const DecodeArgs &a, int bh, uint32_t smem) {
+// Unit bh's state into shared memory: 4,096 16-byte pieces into the padded
+// buffer, by `nthr` threads (thread index `tid` among them).
+__device__ __forceinline__ void issue_unit_state(const DecodeArgs &a, int bh, uint32_t smem, int tid, int nthr) {
     const float *st = a.state + (size_t)bh * kTcD * kTcD;
-#pragma unroll
-    for (int i = 0; i < 16; ++i) {
-        const int id = i * kThreads + threadIdx.x;
+    for (int id = tid; id < kTcD * kTcD / 4; id += nthr) {
         const int row = id >> 5, c16 = id & 31;
         cp_async16(smem + (row * kTcRow + c16 * 4) * 4, st + row * kTcD + c16 * 4);
     }
+    cp_async_commit();
+}
+// The raw rows of unit bh's T keys, queries and values, and its gates (log
+// alpha, beta, gamma), into shared memory.
+template <typename Tio>
+__device__ __forceinline__ void issue_unit_rows(const DecodeArgs &a, int bh, uint32_t smem) {
     const int T = a.T, H = a.H, b = bh / H, h = bh % H;
     constexpr int PR = kTcD * (int)sizeof(Tio) / 16;      // 16-byte pieces per row
     const uint32_t raw = smem + kTcStateBytes;
@@ -292,7 +298,10 @@ decode_tokens_tc_kernel(DecodeArgs a) {
     const Tio *raw_s = reinterpret_cast<const Tio *>(reinterpret_cast<const char *>(sbuf) + kTcStateBytes);
     const float *graw_s = reinterpret_cast<const float *>(reinterpret_cast<const char *>(sbuf) + kTcStateBytes +
                                                           kTcRawBytes);
-    if ((int)blockIdx.x < units) issue_unit_copy<Tio>(a, blockIdx.x, buf);
+    if ((int)blockIdx.x < units) {
+        issue_unit_rows<Tio>(a, blockIdx.x, buf);
+        issue_unit_state(a, blockIdx.x, buf, threadIdx.x, kThreads);
+    }
     for (int bh = blockIdx.x; bh < units; bh += gridDim.x) {
         const int b = bh / H, h = bh % H;
         float *st = a.state + (size_t)bh * D * D;
@@ -327,7 +336,8 @@ decode_tokens_tc_kernel(DecodeArgs a) {
             if (live) v_s[t][d] = Io<Tio>::ld(raw_s + (2 * kMaxT + t) * D + d);
         }
         __syncthreads();
-        if (bh + (int)gridDim.x < units) issue_unit_copy<Tio>(a, bh + gridDim.x, buf);
+        const bool has_next = bh + (int)gridDim.x < units;
+        if (has_next) issue_unit_rows<Tio>(a, bh + gridDim.x, buf);
         __syncthreads();
 
         {
@@ -413,6 +423,10 @@ decode_tokens_tc_kernel(DecodeArgs a) {
 #pragma unroll
             for (int t = 0; t < kMaxT; ++t) w_s[t][j] = t < T ? w[t] : 0.f;
             if (j == 0) c_s = c;
+        } else if (has_next) {
+            // the next unit's state, by the threads the recurrence leaves idle (its
+            // buffer has been free since this unit's state moved into registers)
+            issue_unit_state(a, bh + gridDim.x, buf, threadIdx.x - D, kThreads - D);
         }
         __syncthreads();
 
