@@ -215,3 +215,25 @@ def test_channel_bf16_decode_continues_chunked_prefill(cuda_device):
     got = torch.stack(outs, 1)
     assert rel_l2(to_np(got), to_np(full_o[:, 130:])) <= 1e-2
     assert rel_l2(to_np(st), to_np(full_s)) <= 1e-2
+
+
+def test_channel_bf16_no_initial_state(cuda_device):
+    """The chunked per-channel path from a zero state (no initial state given)."""
+    inp = rda_gen.fixed_inputs(2, 193, 2, 128, 128, dtype=torch.bfloat16, seed=370, s0=False,
+                               gamma=True, channel=True)
+    assert inp.initial_state is None
+    _check(inp)
+
+
+def test_channel_bf16_in_place_final_state(cuda_device):
+    """final_state may alias initial_state on the chunked per-channel path, over
+    an odd number of chunks with a ragged tail."""
+    import gated_delta_rule_rda_b200 as rda
+    inp = rda_gen.fixed_inputs(2, 64 * 9 + 7, 3, 128, 64, dtype=torch.bfloat16, seed=375, s0=True,
+                               channel=True)
+    ro, rs = oracle.forward(inp.q, inp.k, inp.v, inp.log_alpha, inp.beta, initial_state=inp.initial_state)
+    d = inp.to("cuda")
+    st = d.initial_state.clone()
+    out, _ = rda.rda_prefill_chunked(d.q, d.k, d.v, d.log_alpha, d.beta, initial_state=st, final_state=st)
+    torch.cuda.synchronize()
+    assert rel_l2(to_np(st), rs) <= 1e-2 and rel_l2(to_np(out), ro) <= 1e-2
