@@ -29,7 +29,7 @@
 namespace rda {
 namespace {
 
-constexpr int kTok = 64;          // tokens per pre-kernel CTA (one sequence)
+constexpr int kTok = 32;          // tokens per pre-kernel CTA (one sequence)
 
 __device__ __forceinline__ float sigmoid_f(float x) { return __frcp_rn(1.f + __expf(-x)); }
 // Hardware tanh (PTX tanh.approx.f32, relative error about 2^-11).
@@ -147,15 +147,15 @@ template <int ACT, bool FAST> __device__ __forceinline__ float2 act2(float2 x) {
     }
 }
 
-// One CTA per (head, 64-token tile of a sequence): the tile's raw q, k and v
+// One CTA per (head, 32-token tile of a sequence): the tile's raw q, k and v
 // rows of this head, with the two rows before it (the conv's history), go to
 // shared memory first, all as 16-byte asynchronous copies issued up front
-// (~50 KiB in flight per CTA for bf16 at D = 128, four CTAs per SM), then six
-// warps compute from there: warps 2i and 2i+1 own tensor i (q, k, v) for the
-// tile's first and second 32 tokens; a lane owns 2 NP channels of a token row.
-constexpr int kRowsT = kTok + 2;      // tile rows in shared memory: positions p0 - 2 .. p0 + 63
-constexpr int kPrepWarps = 6;
-constexpr int kTokW = kTok / 2;       // tokens per warp
+// (~26 KiB per CTA for bf16 at D = 128, eight CTAs per SM, whose load and
+// compute phases interleave), then three warps compute from there: warp i owns
+// tensor i (q, k, v); a lane owns 2 NP channels of a token row.
+constexpr int kRowsT = kTok + 2;      // tile rows in shared memory: positions p0 - 2 .. p0 + kTok - 1
+constexpr int kPrepWarps = 3;
+constexpr int kTokW = kTok;           // tokens per warp
 constexpr int kUnroll = 4;            // tokens per step of a warp's loop (independent reductions)
 
 template <typename Tio, int DK, int DV>
@@ -243,7 +243,7 @@ __device__ __forceinline__ void conv_rows(const Tio *rows, Tio *dst, size_t stri
 // grid (H, tiles of the longest sequence, sequences): the CTAs of one tile of
 // all heads run side by side and read whole token rows.
 template <typename Tio, int DK, int DV, int ACT>
-__global__ void __launch_bounds__(kPrepWarps * 32, sizeof(Tio) == 2 ? 4 : 2) prep_inputs_kernel(PrepArgs a) {
+__global__ void __launch_bounds__(kPrepWarps * 32, sizeof(Tio) == 2 ? 8 : 4) prep_inputs_kernel(PrepArgs a) {
     using L = PrepSmem<Tio, DK, DV>;
     extern __shared__ __align__(16) uint8_t psm[];
     const int n = blockIdx.z, h = blockIdx.x, tile = blockIdx.y;
@@ -301,8 +301,8 @@ __global__ void __launch_bounds__(kPrepWarps * 32, sizeof(Tio) == 2 ? 4 : 2) pre
     cp_async_wait_all();
     __syncthreads();
     // ---- q, k, v of the tile
-    const int ti = warp >> 1;
-    const int i0 = (warp & 1) * kTokW, i1 = min(i0 + kTokW, pend);
+    const int ti = warp;
+    const int i0 = 0, i1 = min(kTokW, pend);
     if (i0 < i1) {
         const size_t row0 = (size_t)(t0 + p0) * H + h;
         if (ti < 2) {
