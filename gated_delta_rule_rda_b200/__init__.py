@@ -7,10 +7,16 @@ been built, and every call requires CUDA tensors.
 
 Functions mirror the C entry points of ``include/rda.h``:
 
-- :func:`rda_prefill_chunked` -- fixed-length prefill ``[B,T,H,D]``;
+- :func:`rda_prefill_chunked` -- fixed-length prefill ``[B,T,H,D]`` (a log alpha
+  ``[B,T,H,Dk]`` selects the per-key-channel decay);
 - :func:`rda_prefill_varlen` -- packed sequences with ``cu_seqlens``;
 - :func:`rda_decode_step` -- one token per sequence, state updated in place;
-- :func:`rda_read_device_error`, :func:`rda_prefill_workspace_bytes`.
+- :func:`rda_decode_tokens` -- 1..8 tokens per sequence in one pass over the state;
+- :func:`rda_prep_inputs`, :func:`rda_output_gate_norm` -- the steps either side of
+  the core (short convolutions, q/k norms, gates; output RMSNorm times the gate);
+- :func:`rda_backward` -- the gradients of the core;
+- :func:`rda_read_device_error`, :func:`rda_prefill_workspace_bytes`,
+  :func:`rda_prefill_channel_workspace_bytes`.
 
 The raw ctypes handle is :data:`lib` (``lib.rda_prefill_chunked(...)`` takes
 plain pointers and sizes, including host-pointer use for the varlen schedule).

@@ -61,6 +61,11 @@ def test_workspace_query():
     assert rda.rda_prefill_channel_workspace_bytes(1, 4096, 16, 64, 64, 0) == \
         rda.rda_prefill_workspace_bytes(1, 4096, 16, 64, 64, 0)
     assert rda.rda_prefill_channel_workspace_bytes(1, 100, 16, 96, 128, 0) == 0
+    # packed batches: the schedule and the chunk offsets on top, more than the fixed-length figure
+    assert rda.rda_prefill_channel_workspace_bytes(1, 4096, 16, 128, 128, 8) > \
+        rda.rda_prefill_channel_workspace_bytes(1, 4096, 16, 128, 128, 0)
+    assert rda.rda_prefill_channel_workspace_bytes(1, 4096, 16, 128, 128, 8) > \
+        rda.rda_prefill_workspace_bytes(1, 4096, 16, 128, 128, 8)
 
 
 # Fake device addresses: never dereferenced, because validation fails first.
